@@ -1,0 +1,154 @@
+"""CPU oracle for the tree-verification step (fp64, plain C).
+
+TEST INFRASTRUCTURE ONLY.  The tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may call it; the library under test never does.
+It shares no code with the CUDA path; both read inputs from ``synth``.
+
+Functions and what each follows (all pages are about tree-based speculative
+decoding):
+
+* :func:`tree_mask` -- the mask definition M[i][j] = 1 iff node j is node i or
+  an ancestor of i (glossary page, "Tree attention"), whose 5-node instance is
+  the blog's "Tree Attention Verification Matrix" (section 3).
+* :func:`tree_attention` -- every node attends to the whole prefix plus its own
+  root path in one pass (glossary, "Tree attention"); plain masked softmax
+  attention with a dense mask, accumulated in fp64.
+* :func:`verify_sample` -- the acceptance rule min(1, p/q) and the
+  renormalised residual max(0, p - q) (blog section 2, "Rejection Sampling
+  Acceptance Condition"), applied root-down with sibling retries (glossary,
+  "SpecInfer").
+
+Every function is pinned by ``tests/test_oracle_*.py`` against values the
+pages print, closed forms and library routines.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+OK, ERR_ARG, ERR_TREE, ERR_BLOCK = 0, 1, 3, 4
+
+
+def build(force: bool = False, extra_flags=(), out: str | None = None) -> str:
+    """Compile the oracle with gcc (fp64, OpenMP, no fast-math)."""
+    src = os.path.join(_HERE, "oracle.c")
+    out = out or _LIB_PATH
+    if force or extra_flags or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", *extra_flags, "-o", out, src, "-lm"])
+    return out
+
+
+def _bind(path):
+    L = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    i32, i64, dbl = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
+    L.or_tree_mask.argtypes = [i32, P, P]
+    L.or_tree_attention.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, dbl, i64, P, P]
+    L.or_verify_sample.argtypes = [i32, i32, i64, P, P, P, P, P, dbl, P, P, P, P, P]
+    L.or_set_threads.argtypes = [ctypes.c_int]
+    L.or_max_threads.restype = ctypes.c_int
+    return L
+
+
+_lib = None
+
+
+def lib():
+    """The oracle library; ``ORACLE_LIB`` may name another build of
+    ``oracle.c`` (the mutation tests point it at planted-mistake builds)."""
+    global _lib
+    if _lib is None:
+        _lib = _bind(os.environ.get("ORACLE_LIB") or build())
+    return _lib
+
+
+def load_variant(path: str):
+    """Bind a separately compiled oracle build (used by the mutation tests)."""
+    return _bind(path)
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def set_threads(n: int) -> None:
+    lib().or_set_threads(int(n))
+
+
+def max_threads() -> int:
+    return int(lib().or_max_threads())
+
+
+def tree_mask(parent, L=None) -> np.ndarray:
+    parent = np.ascontiguousarray(parent, dtype=np.int32)
+    n = parent.shape[0]
+    m = np.zeros((n, n), dtype=np.uint8)
+    rc = (L or lib()).or_tree_mask(n, _p(parent), _p(m))
+    if rc:
+        raise ValueError(f"invalid tree (code {rc})")
+    return m
+
+
+def tree_attention(query, k_cache, v_cache, block_table, prefix_lens, parent_idx, num_kv_heads,
+                   dtype: str, scale: float | None = None, rows=None, L=None) -> np.ndarray:
+    """fp64 tree attention.
+
+    query [B][N][Hq][D], caches [num_blocks][bs][Hkv][D] (float32 arrays, or
+    uint16 bfloat16 bits when dtype == "bf16"), block_table [B][max_blocks],
+    prefix_lens [B], parent_idx [B][N].  ``rows`` is an optional int array of
+    (b, i, h) triples; the result is then [n_rows][D], else [B][N][Hq][D]."""
+    B, N, Hq, D = query.shape
+    nb, bs, Hkv, D2 = k_cache.shape
+    assert D2 == D and Hkv == num_kv_heads
+    code = 0 if dtype == "bf16" else 1
+    want = np.uint16 if code == 0 else np.float32
+    q = np.ascontiguousarray(query, dtype=want)
+    kc = np.ascontiguousarray(k_cache, dtype=want)
+    vc = np.ascontiguousarray(v_cache, dtype=want)
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    pl = np.ascontiguousarray(prefix_lens, dtype=np.int32)
+    pa = np.ascontiguousarray(parent_idx, dtype=np.int32)
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    if rows is not None:
+        r = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 3))
+        out = np.zeros((r.shape[0], D), dtype=np.float64)
+        n_rows = r.shape[0]
+    else:
+        r = None
+        out = np.zeros((B, N, Hq, D), dtype=np.float64)
+        n_rows = B * N * Hq
+    rc = (L or lib()).or_tree_attention(B, N, Hq, Hkv, D, bs, bt.shape[1], nb, code, _p(q), _p(kc), _p(vc),
+                                        _p(bt), _p(pl), _p(pa), float(scale), n_rows, _p(r), _p(out))
+    if rc:
+        raise ValueError(f"oracle tree_attention failed (code {rc})")
+    return out
+
+
+def verify_sample(p, q, tree_tokens, parent_idx, uniforms, eps: float = 1e-6, L=None):
+    """Literal root-down acceptance walk in fp64.
+
+    Returns a dict with accepted_path [B][N] (-1 padded), accepted_len [B],
+    bonus_token [B], near [B] (threshold events within ``eps``), rows [B]
+    (vocabulary rows read in full) and rc (0, or 3 when some tree was
+    invalid)."""
+    B, N, V = p.shape
+    pp = np.ascontiguousarray(p, dtype=np.float32)
+    qq = np.ascontiguousarray(q, dtype=np.float32)
+    tt = np.ascontiguousarray(tree_tokens, dtype=np.int32)
+    pa = np.ascontiguousarray(parent_idx, dtype=np.int32)
+    uu = np.ascontiguousarray(uniforms, dtype=np.float32)
+    path = np.zeros((B, N), dtype=np.int32)
+    alen = np.zeros(B, dtype=np.int32)
+    bonus = np.zeros(B, dtype=np.int32)
+    near = np.zeros(B, dtype=np.int32)
+    rows = np.zeros(B, dtype=np.int32)
+    rc = (L or lib()).or_verify_sample(B, N, V, _p(pp), _p(qq), _p(tt), _p(pa), _p(uu), float(eps),
+                                       _p(path), _p(alen), _p(bonus), _p(near), _p(rows))
+    return {"accepted_path": path, "accepted_len": alen, "bonus_token": bonus, "near": near, "rows": rows, "rc": rc}
