@@ -1,0 +1,423 @@
+#!/usr/bin/env python3
+"""Benchmark of the tree-verification step: one tree-attention call (one
+layer) plus one acceptance walk, on seeded synthetic inputs.
+
+Default workload (one GPU): the Llama-3-8B attention shape -- batch 1,
+prefix 4096 (contiguous blocks), 32 query / 8 KV heads, head_dim 128, bf16,
+a 64-node top-k [4,3,2,2,1,1] tree, vocabulary 128256 with fp32 p/q.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU runs (launched with torch.distributed.run) give every rank its own
+independent sequences (weak scaling, no data-path collective); time is the
+maximum over ranks.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "tree nodes verified/s and µs per verify step; achieved HBM GB/s vs B200 peak"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 512 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured", d
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback", {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "tree_speculative_decoding_07_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    kernel sources changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[kernel_key][workload]
+        if e.get("source_hash") != kernel_source_hash():
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ inputs
+
+def make_inputs(workload: str, seed: int):
+    import synth
+    wl = synth.make(workload, seed=seed)
+    p, q = wl.pq()
+    return wl, {
+        "query": wl.query(), "k": wl.k_cache(), "v": wl.v_cache(), "block_table": wl.block_table,
+        "prefix_lens": wl.prefix_lens, "parent_idx": wl.parent_idx, "p": p, "q": q,
+        "tokens": wl.tree_tokens, "uniforms": wl.uniforms(),
+    }
+
+
+def attention_bytes(wl) -> int:
+    """Algorithmic HBM bytes of one tree-attention call: every cached K and V
+    row the call must read (prefix plus tree block, per KV head), the queries
+    and the outputs."""
+    el = 2 if wl.dtype == "bf16" else 4
+    kv = 2 * int((wl.prefix_lens.astype(np.int64) + wl.num_nodes).sum()) * wl.num_kv_heads * wl.head_dim * el
+    qo = 2 * wl.batch * wl.num_nodes * wl.num_q_heads * wl.head_dim * el
+    return kv + qo
+
+
+def sampler_bytes(wl, h) -> int:
+    """Algorithmic bytes of the acceptance walk: 8 bytes (p and q) per tested
+    child plus both rows of every node whose row the walk reads in full
+    (as logged by the oracle), plus tree metadata."""
+    import oracle
+    r = oracle.verify_sample(h["p"], h["q"], h["tokens"], h["parent_idx"], h["uniforms"])
+    rows = int(r["rows"].sum())
+    tested = int((h["parent_idx"] >= 0).sum())
+    return rows * 8 * wl.vocab + tested * 12 + h["parent_idx"].size * 8
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import tree_speculative_decoding_07_b200 as tv
+
+    torch.cuda.set_device(local_rank)
+    wl, h = make_inputs(args.workload, seed=1 + 1000 * rank)
+
+    def dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+    d = {k: dev(v) for k, v in h.items()}
+    out = torch.empty_like(d["query"])
+    B, N = wl.batch, wl.num_nodes
+    path = torch.empty((B, N), dtype=torch.int32, device="cuda")
+    alen = torch.empty((B,), dtype=torch.int32, device="cuda")
+    bonus = torch.empty((B,), dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    adesc = tv.attn_desc(d["query"], d["k"], d["block_table"])
+    aplan = tv.tv_tree_attention_plan(adesc)
+    ws_bytes = aplan.workspace_bytes
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
+    sdesc = tv.TvSampleDesc(B, N, wl.vocab)
+    splan = tv.tv_verify_sample_plan(sdesc)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(dd, o, pth, ln, bn, mid):
+        s1 = tv.tv_tree_attention(adesc, dd["query"], dd["k"], dd["v"], dd["block_table"], dd["prefix_lens"],
+                                  dd["parent_idx"], o, ws, ws_bytes, status, stream)
+        mid.record(stream)
+        s2 = tv.tv_verify_sample(sdesc, dd["p"], dd["q"], dd["tokens"], dd["parent_idx"], dd["uniforms"], pth, ln,
+                                 bn, None, 0, status, stream)
+        if s1 or s2:
+            raise tv.TreeVerifyError(s1 or s2, "verify step")
+
+    # ---- device-resident timing (L2 flushed before every step)
+    W, K = args.warmup, args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for _ in range(W):
+        flush.zero_()
+        step(d, out, path, alen, bonus, torch.cuda.Event())
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_wall = time.perf_counter()
+    for k in range(K):
+        flush.zero_()
+        e0, mid, e1 = ev[k]
+        e0.record(stream)
+        step(d, out, path, alen, bonus, mid)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    attn_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
+    samp_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
+    step_ms = [ev[k][0].elapsed_time(ev[k][2]) for k in range(K)]
+    total_ms = float(sum(step_ms))
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())}")
+
+    # ---- end to end: host (pinned) inputs -> device -> results back, every step
+    pin = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16) if v.dtype == np.uint16
+                               else np.ascontiguousarray(v)).pin_memory() for k, v in h.items()}
+    h2d = int(sum(v.numel() * v.element_size() for v in pin.values()))
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    path_h = torch.empty(path.shape, dtype=torch.int32).pin_memory()
+    alen_h = torch.empty(alen.shape, dtype=torch.int32).pin_memory()
+    bonus_h = torch.empty(bonus.shape, dtype=torch.int32).pin_memory()
+    d2h = sum(t.numel() * t.element_size() for t in (out_h, path_h, alen_h, bonus_h))
+    K2 = max(3, min(K, 50))
+
+    def e2e_step():
+        for key, t in pin.items():
+            dst = d[key]
+            (dst.view(torch.int16) if dst.dtype == torch.bfloat16 else dst).copy_(t, non_blocking=True)
+        step(d, out, path, alen, bonus, torch.cuda.Event())
+        out_h.copy_(out, non_blocking=True)
+        path_h.copy_(path, non_blocking=True)
+        alen_h.copy_(alen, non_blocking=True)
+        bonus_h.copy_(bonus, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(K2):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a0.elapsed_time(a1)
+
+    times = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = float(times[0]), float(times[1])
+    if rank != 0:
+        return None
+
+    nodes = B * N
+    ms_step = total_ms / K
+    value = world * nodes * K / (total_ms / 1e3)
+    e2e_value = world * nodes * K2 / (e2e_ms / 1e3)
+    peak, peak_kind, _ = load_peaks()
+    a_bytes = attention_bytes(wl)
+    s_bytes = sampler_bytes(wl, h)
+    attn_avg_s = (sum(attn_ms) / K) / 1e3
+    achieved = a_bytes / attn_avg_s / 1e9
+    kernel_key = "attn_tc" if aplan.kernel == 0 else "attn_simt"
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "nodes/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": ms_step,
+        "us_per_step": ms_step * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": wl.dtype,
+        "data": "synthetic (Philox4x32-10 seeded; no dataset)",
+        "config": {"workload": f"{args.workload}: batch {wl.batch}, prefix {int(wl.prefix_lens[0])}, "
+                               f"Hq {wl.num_q_heads}/Hkv {wl.num_kv_heads}, D {wl.head_dim}, {wl.dtype}, "
+                               f"{N}-node tree, vocab {wl.vocab}",
+                   "global_batch": world * B, "tree_nodes": N, "seq_len": int(wl.prefix_lens.max()) + N,
+                   "parallelism": f"replicas x{world} (independent sequences per GPU)",
+                   "l2": f"flushed before every step ({L2_FLUSH_BYTES >> 20} MB write, outside the step events)"},
+        "attention_us": attn_avg_s * 1e6,
+        "sample_us": (sum(samp_ms) / K) * 1e3,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": ncu_traffic(kernel_key, args.workload), "kernel": kernel_key,
+                     "algorithmic_bytes": a_bytes, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_kind == "measured" else "fallback 6.65 TB/s"},
+        "step_roofline": {"bytes": a_bytes + s_bytes, "sampler_bytes": s_bytes,
+                          "frac": (a_bytes + s_bytes) / (ms_step / 1e3) / 1e9 / peak},
+        "e2e": {"value": e2e_value, "unit": "nodes/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": K2},
+        "gpu_launches": K * (aplan.launches + splan.launches),
+        "clocks": clk,
+        "wall_s": t_wall,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, h, budget_s=args.cpu_budget)
+    return line
+
+
+# ------------------------------------------------------------------ oracle timing
+
+def oracle_step_times(wl, h, rows_frac: float):
+    """Time the oracle on one step: attention over a deterministic fraction of
+    the query rows (extrapolated to all rows) plus the full acceptance walk."""
+    import oracle
+    B, N, Hq = wl.batch, wl.num_nodes, wl.num_q_heads
+    total_rows = B * N * Hq
+    n = max(1, int(round(total_rows * rows_frac)))
+    sel = np.linspace(0, total_rows - 1, n).astype(np.int64)
+    rows = np.stack([sel // (N * Hq), (sel // Hq) % N, sel % Hq], axis=1).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.tree_attention(h["query"], h["k"], h["v"], h["block_table"], h["prefix_lens"], h["parent_idx"],
+                          wl.num_kv_heads, wl.dtype, rows=rows)
+    t_attn = (time.perf_counter() - t0) * total_rows / n
+    t0 = time.perf_counter()
+    oracle.verify_sample(h["p"], h["q"], h["tokens"], h["parent_idx"], h["uniforms"])
+    t_walk = time.perf_counter() - t0
+    return t_attn + t_walk, n, total_rows
+
+
+def cpu_baseline(wl, h, budget_s: float = 20.0):
+    import oracle
+    cores = oracle.max_threads()
+    # calibrate with a small fraction, then size the sample to the budget
+    t_est, n, total = oracle_step_times(wl, h, 1.0 / 64)
+    frac = min(1.0, max(1.0 / 64, budget_s / max(t_est, 1e-9)))
+    steps, t_sum, rows_done = 0, 0.0, 0
+    t_start = time.perf_counter()
+    while time.perf_counter() - t_start < budget_s or steps == 0:
+        t, n, total = oracle_step_times(wl, h, frac)
+        t_sum += t
+        rows_done += n
+        steps += 1
+        if frac >= 1.0 and time.perf_counter() - t_start > budget_s / 2:
+            break
+    per_step = t_sum / steps
+    return {"value": wl.batch * wl.num_nodes / per_step, "unit": "nodes/s", "cores": cores, "kind": "oracle",
+            "sample": f"{steps} oracle step(s): attention on {rows_done // steps} of {total} query rows "
+                      f"(time scaled to all rows) plus the full fp64 acceptance walk; "
+                      f"{per_step * 1e3:.1f} ms per full step"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    wl, h = make_inputs(args.workload, seed=1)
+    K, W = args.steps, args.warmup
+    budget = 150.0
+    t_est, _, _ = oracle_step_times(wl, h, 1.0 / 64)
+    frac = min(1.0, max(1.0 / 1024, budget / max(1, K + W) / max(t_est, 1e-9)))
+    for _ in range(W):
+        oracle_step_times(wl, h, frac)
+    times = []
+    n_rows = 0
+    for _ in range(K):
+        t, n_rows, total = oracle_step_times(wl, h, frac)
+        times.append(t)
+    per_step = sum(times) / K
+    value = wl.batch * wl.num_nodes / per_step
+    cores = oracle.max_threads()
+    sample = (f"each step: oracle attention on {n_rows} of {total} query rows (time scaled to all rows) "
+              f"plus the full fp64 acceptance walk")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "nodes/s", "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (Philox4x32-10 seeded; no dataset)",
+            "config": {"workload": args.workload}, "cpu_baseline": {"value": value, "unit": "nodes/s",
+                                                                  "cores": cores, "kind": "oracle",
+                                                                  "sample": sample},
+            "e2e": {"value": value, "unit": "nodes/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="l8b", choices=("tiny", "l8b", "l70b", "mix", "long"))
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        import datetime
+
+        import torch.distributed as dist
+        if world > 1:
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=None)
+        try:
+            line = run_ours(args, rank, world, local_rank)
+        finally:
+            if world > 1:
+                dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

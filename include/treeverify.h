@@ -1,0 +1,182 @@
+/*
+ * treeverify.h -- C ABI of libtreeverify, the target model's verification
+ * step of tree-based speculative decoding on one NVIDIA B200 (sm_100a).
+ *
+ * The step has two parts, each one call:
+ *
+ *  tv_tree_attention  every draft-tree node attends to its sequence's cached
+ *                     prefix and to its own root path, in one pass.  Defined
+ *                     by the glossary page "Tree-based speculative decoding"
+ *                     (jisaku.com), section "Tree attention": the mask
+ *                     M[i][j] = 1 iff node j is node i or one of its
+ *                     ancestors; its 5-node instance is the blog "Speculative
+ *                     decoding x tree attention" (radar-34b), section 3,
+ *                     figure "Tree Attention Verification Matrix".
+ *
+ *  tv_verify_sample   the lossless acceptance walk.  Defined by the same blog,
+ *                     section 2, table "Rejection Sampling Acceptance
+ *                     Condition" (accept x with probability min(1, p(x)/q(x)),
+ *                     on rejection resample from max(0, p - q) normalised) and
+ *                     the glossary's section "SpecInfer" (the tree is verified
+ *                     root-down, depth first; a rejected child hands the
+ *                     renormalised residual to its next sibling).
+ *
+ * Conventions shared by all calls
+ *  - Every array pointer is a caller-owned DEVICE pointer unless stated
+ *    otherwise; descriptors and plan structs are host memory.  The library
+ *    never allocates device memory and never synchronises the stream.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Work is enqueued asynchronously on it.
+ *  - Host-checkable errors (shapes, dtype, null pointers, workspace size)
+ *    return a status before anything is launched.
+ *  - Data-dependent errors (a malformed tree, a block id or token id out of
+ *    range) are written by the kernels to `*dev_status` (a device int32 the
+ *    caller zeroes; may be NULL) with the first error code winning; the
+ *    affected sequence gets sentinel outputs (NaN attention rows, -1 tokens)
+ *    and the kernels exit normally.  Kernels never trap.
+ *  - Results are deterministic: the same inputs give bit-identical outputs.
+ */
+#ifndef TREEVERIFY_H
+#define TREEVERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TV_API __attribute__((visibility("default")))
+#else
+#define TV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TV_OK = 0,
+    TV_ERR_INVALID_ARG = 1,   /* bad descriptor field, null pointer, bad size */
+    TV_ERR_UNSUPPORTED = 2,   /* valid but not supported by this build (e.g. head_dim) */
+    TV_ERR_TREE = 3,          /* device: parent_idx not topological, or token out of range */
+    TV_ERR_BLOCK_TABLE = 4,   /* device: block id outside [0, num_blocks) */
+    TV_ERR_WORKSPACE = 5,     /* workspace null or smaller than the *_workspace_size value */
+    TV_ERR_CUDA = 6,          /* a CUDA runtime call failed (launch configuration etc.) */
+    TV_ERR_TIMEOUT = 7        /* device: a bounded wait ran out */
+} tv_status;
+
+typedef enum { TV_BF16 = 0, TV_F32 = 1 } tv_dtype;
+
+/*
+ * Tree attention problem.
+ *   q, out      [batch][num_nodes][num_q_heads][head_dim], dtype, contiguous
+ *   paged_k/v   [num_blocks][block_size][num_kv_heads][head_dim], dtype
+ *   block_table [batch][max_blocks_per_seq] int32: logical block j of
+ *               sequence b lives in physical block block_table[b][j]
+ *   prefix_lens [batch] int32: L_b, committed tokens before the tree
+ *   parent_idx  [batch][num_nodes] int32: parent_idx[b][0] = -1 (the root,
+ *               i.e. the last committed token), 0 <= parent_idx[b][i] < i
+ * Node i's key/value sit at logical position L_b + i of the paged cache;
+ * the caller writes them before the call.  Query head h reads KV head
+ * h / (num_q_heads / num_kv_heads).  Row (b, i, h) of `out` is softmax
+ * attention of q[b][i][h] over positions t < L_b and the positions L_b + j
+ * of the nodes j on i's root path, with scores scaled by softmax_scale
+ * (0 means 1/sqrt(head_dim)).  Cache slots at positions >= L_b + num_nodes
+ * inside an allocated block are never used.  For bf16 with head_dim 128
+ * (the tensor-core path) q, paged_k, paged_v and out must be 16-byte
+ * aligned, else TV_ERR_INVALID_ARG.
+ */
+typedef struct {
+    int32_t batch;
+    int32_t num_nodes;           /* 1..128 */
+    int32_t num_q_heads;
+    int32_t num_kv_heads;        /* divides num_q_heads */
+    int32_t head_dim;            /* 64 or 128 */
+    int32_t block_size;          /* 16 */
+    int32_t max_blocks_per_seq;  /* >= ceil((L_b + num_nodes) / block_size) for every b */
+    int32_t num_blocks;          /* physical blocks in paged_k / paged_v */
+    int32_t dtype;               /* tv_dtype of q, paged_k, paged_v and out */
+    float softmax_scale;         /* 0 => 1/sqrt(head_dim) */
+} tv_attn_desc;
+
+/* How a call will run (host-side query; launches nothing). */
+typedef struct {
+    int32_t kernel;              /* 0 = tensor-core (tcgen05) bf16 path, 1 = CUDA-core path */
+    int32_t num_splits;          /* KV splits per (sequence, KV head, row tile) */
+    int32_t row_tiles;           /* 128-row query tiles per (sequence, KV head) */
+    int32_t grid_ctas;           /* CTAs in the main launch */
+    int32_t launches;            /* kernel launches per call */
+    size_t workspace_bytes;      /* same value as tv_tree_attention_workspace_size */
+} tv_attn_plan;
+
+TV_API tv_status tv_tree_attention_plan(const tv_attn_desc *desc, tv_attn_plan *plan);
+
+/* Device workspace the call needs, in bytes (0 when none).  Ownership stays
+ * with the caller; it must be 256-byte aligned and may be reused across
+ * calls that are ordered on one stream. */
+TV_API size_t tv_tree_attention_workspace_size(const tv_attn_desc *desc);
+
+TV_API tv_status tv_tree_attention(const tv_attn_desc *desc, const void *q, const void *paged_k,
+                            const void *paged_v, const int32_t *block_table,
+                            const int32_t *prefix_lens, const int32_t *parent_idx, void *out,
+                            void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                            void *stream);
+
+/*
+ * Acceptance walk problem.
+ *   p, q         [batch][num_nodes][vocab] float32 probabilities:
+ *                p[b][u] = target distribution after node u's path,
+ *                q[b][u] = draft distribution node u's children were drawn from
+ *   tree_tokens  [batch][num_nodes] int32 draft token of each node (the
+ *                root's entry is ignored)
+ *   parent_idx   [batch][num_nodes] int32 as for tv_tree_attention
+ *   uniforms     [batch][num_nodes] float32 in [0,1): uniforms[b][c] (c >= 1)
+ *                is node c's acceptance draw, uniforms[b][0] the bonus draw
+ * Walk: from the root, children of the current node u are tried in
+ * ascending index; child c with token x is accepted iff
+ * uniforms[b][c] < P(x) / q[b][u][x], P being p[b][u] renormalised after
+ * each rejected sibling to max(0, P - q[b][u]) / sum(max(0, P - q[b][u]))
+ * (q(x) = 0 accepts iff P(x) > 0; a zero residual keeps P).  Acceptance
+ * descends into c.  When no child is accepted (or u is a leaf) the bonus
+ * token is the first index whose running sum of P exceeds
+ * uniforms[b][0] * sum(P) (the last positive index if rounding leaves none).
+ * Outputs:
+ *   accepted_path [batch][num_nodes] int32: accepted node indices, root
+ *                 excluded, in walk order, padded with -1
+ *   accepted_len  [batch] int32, bonus_token [batch] int32
+ * A malformed tree or token gives accepted_len = -1, bonus = -1 and
+ * TV_ERR_TREE in *dev_status.
+ */
+typedef struct {
+    int32_t batch;
+    int32_t num_nodes;           /* 1..1024 */
+    int32_t vocab;               /* 1..(16 * 24576) */
+} tv_sample_desc;
+
+typedef struct {
+    int32_t cluster_ctas;        /* CTAs cooperating on one sequence's rows */
+    int32_t threads;             /* threads per CTA */
+    int32_t slice;               /* vocabulary entries held per CTA */
+    int32_t smem_bytes;          /* dynamic shared memory per CTA */
+    int32_t launches;            /* kernel launches per call */
+} tv_sample_plan;
+
+TV_API tv_status tv_verify_sample_plan(const tv_sample_desc *desc, tv_sample_plan *plan);
+
+TV_API size_t tv_verify_sample_workspace_size(const tv_sample_desc *desc);
+
+TV_API tv_status tv_verify_sample(const tv_sample_desc *desc, const float *p, const float *q,
+                           const int32_t *tree_tokens, const int32_t *parent_idx,
+                           const float *uniforms, int32_t *accepted_path, int32_t *accepted_len,
+                           int32_t *bonus_token, void *workspace, size_t workspace_bytes,
+                           int32_t *dev_status, void *stream);
+
+/* Static string for a status code. */
+TV_API const char *tv_status_string(int32_t status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+TV_API int32_t tv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TREEVERIFY_H */

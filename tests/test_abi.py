@@ -1,0 +1,105 @@
+"""The C-ABI library loads, exports every symbol ``include/*.h`` declares,
+and rejects bad arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import tree_speculative_decoding_07_b200 as tv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names += re.findall(r"TV_API\s+[\w\s\*]*?\b(tv_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    L = tv.lib()
+    names = declared_symbols()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+
+
+def test_version_and_status_strings():
+    assert tv.tv_version() >= 100
+    for s in range(8):
+        assert tv.tv_status_string(s)
+    assert "unknown" in tv.tv_status_string(99)
+
+
+def _desc(**kw):
+    base = dict(batch=1, num_nodes=5, num_q_heads=8, num_kv_heads=2, head_dim=64, block_size=16,
+                max_blocks_per_seq=9, num_blocks=9, dtype=tv.TV_F32, softmax_scale=0.0)
+    base.update(kw)
+    return tv.TvAttnDesc(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(batch=0), tv.TV_ERR_INVALID_ARG),
+    (dict(num_q_heads=6, num_kv_heads=4), tv.TV_ERR_INVALID_ARG),
+    (dict(num_nodes=129), tv.TV_ERR_UNSUPPORTED),
+    (dict(head_dim=96), tv.TV_ERR_UNSUPPORTED),
+    (dict(block_size=32), tv.TV_ERR_UNSUPPORTED),
+    (dict(dtype=7), tv.TV_ERR_INVALID_ARG),
+    (dict(softmax_scale=-1.0), tv.TV_ERR_INVALID_ARG),
+    (dict(max_blocks_per_seq=0), tv.TV_ERR_INVALID_ARG),
+])
+def test_attention_rejects_bad_descriptors(kw, status):
+    d = _desc(**kw)
+    plan = tv.TvAttnPlan()
+    assert tv.lib().tv_tree_attention_plan(ctypes.byref(d), ctypes.byref(plan)) == status
+    dummy = 256
+    assert tv.tv_tree_attention(d, dummy, dummy, dummy, dummy, dummy, dummy, dummy, stream=0) == status
+
+
+def test_attention_rejects_null_pointers_and_small_workspace():
+    d = _desc()
+    assert tv.tv_tree_attention(d, None, 256, 256, 256, 256, 256, 256, stream=0) == tv.TV_ERR_INVALID_ARG
+    d = _desc(batch=1, num_nodes=64, num_q_heads=32, num_kv_heads=8, head_dim=128, max_blocks_per_seq=4096,
+              num_blocks=4096, dtype=tv.TV_F32)
+    need = tv.tv_tree_attention_workspace_size(d)
+    plan = tv.tv_tree_attention_plan(d)
+    assert plan.workspace_bytes == need
+    if need:
+        assert tv.tv_tree_attention(d, 256, 256, 256, 256, 256, 256, 256, 256, need - 1, stream=0) == tv.TV_ERR_WORKSPACE
+        assert tv.tv_tree_attention(d, 256, 256, 256, 256, 256, 256, 256, None, need, stream=0) == tv.TV_ERR_WORKSPACE
+
+
+def test_attention_plans():
+    # bf16 head_dim 128 runs on the tensor-core kernel, fp32 on the CUDA-core kernel
+    d = _desc(num_nodes=64, num_q_heads=32, num_kv_heads=8, head_dim=128, max_blocks_per_seq=260,
+              num_blocks=260, dtype=tv.TV_BF16)
+    p = tv.tv_tree_attention_plan(d)
+    assert p.num_splits >= 1 and p.grid_ctas >= 1 and p.launches >= 1
+    d = _desc()
+    p = tv.tv_tree_attention_plan(d)
+    assert p.kernel == 1 and p.row_tiles == 1
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(batch=0, num_nodes=4, vocab=10), tv.TV_ERR_INVALID_ARG),
+    (dict(batch=1, num_nodes=0, vocab=10), tv.TV_ERR_INVALID_ARG),
+    (dict(batch=1, num_nodes=1025, vocab=10), tv.TV_ERR_UNSUPPORTED),
+    (dict(batch=1, num_nodes=4, vocab=16 * 24576 + 1), tv.TV_ERR_UNSUPPORTED),
+])
+def test_sampler_rejects_bad_descriptors(kw, status):
+    d = tv.TvSampleDesc(**kw)
+    dummy = 256
+    assert tv.tv_verify_sample(d, *([dummy] * 8), stream=0) == status
+
+
+def test_sampler_plan_covers_vocab():
+    for V in (8, 1000, 128256, 151936):
+        p = tv.tv_verify_sample_plan(tv.TvSampleDesc(1, 64, V))
+        assert p.cluster_ctas * p.slice >= V and p.slice % 4 == 0
+        assert 32 <= p.threads <= 512 and p.threads % 32 == 0
+        assert p.smem_bytes == 8 * p.slice
+    assert tv.tv_verify_sample_workspace_size(tv.TvSampleDesc(1, 64, 1000)) == 0

@@ -1,0 +1,213 @@
+"""libtreeverify: the target model's verification step of tree-based
+speculative decoding, as a CUDA library for one B200 (sm_100a).
+
+This module is a thin ctypes binding over the C ABI in
+``include/treeverify.h``: the functions named ``tv_*`` take the same
+arguments as the C calls (device pointers taken from torch tensors, the
+current torch CUDA stream unless another is given) and return the C status.
+All computation happens in the library's kernels; torch only provides
+device memory and streams.
+
+Convenience wrappers :func:`tree_attention` and :func:`verify_sample`
+allocate outputs/workspace with torch and raise on a non-OK status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtreeverify.so")
+
+TV_OK, TV_ERR_INVALID_ARG, TV_ERR_UNSUPPORTED, TV_ERR_TREE = 0, 1, 2, 3
+TV_ERR_BLOCK_TABLE, TV_ERR_WORKSPACE, TV_ERR_CUDA, TV_ERR_TIMEOUT = 4, 5, 6, 7
+TV_BF16, TV_F32 = 0, 1
+
+
+class TvAttnDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_nodes", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("max_blocks_per_seq", ctypes.c_int32), ("num_blocks", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float)]
+
+
+class TvAttnPlan(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_int32), ("num_splits", ctypes.c_int32), ("row_tiles", ctypes.c_int32),
+                ("grid_ctas", ctypes.c_int32), ("launches", ctypes.c_int32), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class TvSampleDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_nodes", ctypes.c_int32), ("vocab", ctypes.c_int32)]
+
+
+class TvSamplePlan(ctypes.Structure):
+    _fields_ = [("cluster_ctas", ctypes.c_int32), ("threads", ctypes.c_int32), ("slice", ctypes.c_int32),
+                ("smem_bytes", ctypes.c_int32), ("launches", ctypes.c_int32)]
+
+
+class TreeVerifyError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {tv_status_string(status)} (status {status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libtreeverify.so; raises if the library has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libtreeverify.so not built at {LIB_PATH}; run __graft_entry__.build() "
+                              "or python -m tree_speculative_decoding_07_b200.build_lib")
+        L = ctypes.CDLL(LIB_PATH)
+        P, sz = ctypes.c_void_p, ctypes.c_size_t
+        L.tv_tree_attention_plan.argtypes = [ctypes.POINTER(TvAttnDesc), ctypes.POINTER(TvAttnPlan)]
+        L.tv_tree_attention_workspace_size.argtypes = [ctypes.POINTER(TvAttnDesc)]
+        L.tv_tree_attention_workspace_size.restype = sz
+        L.tv_tree_attention.argtypes = [ctypes.POINTER(TvAttnDesc), P, P, P, P, P, P, P, P, sz, P, P]
+        L.tv_verify_sample_plan.argtypes = [ctypes.POINTER(TvSampleDesc), ctypes.POINTER(TvSamplePlan)]
+        L.tv_verify_sample_workspace_size.argtypes = [ctypes.POINTER(TvSampleDesc)]
+        L.tv_verify_sample_workspace_size.restype = sz
+        L.tv_verify_sample.argtypes = [ctypes.POINTER(TvSampleDesc), P, P, P, P, P, P, P, P, P, sz, P, P]
+        L.tv_status_string.argtypes = [ctypes.c_int32]
+        L.tv_status_string.restype = ctypes.c_char_p
+        L.tv_version.restype = ctypes.c_int32
+        for name in ("tv_tree_attention_plan", "tv_tree_attention", "tv_verify_sample_plan", "tv_verify_sample"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(t) -> ctypes.c_void_p | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p | None:
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# ------------------------------------------------------------ C ABI, same names
+
+def tv_version() -> int:
+    return int(lib().tv_version())
+
+
+def tv_status_string(status: int) -> str:
+    return lib().tv_status_string(int(status)).decode()
+
+
+def tv_tree_attention_plan(desc: TvAttnDesc) -> TvAttnPlan:
+    plan = TvAttnPlan()
+    s = lib().tv_tree_attention_plan(ctypes.byref(desc), ctypes.byref(plan))
+    if s != TV_OK:
+        raise TreeVerifyError(s, "tv_tree_attention_plan")
+    return plan
+
+
+def tv_tree_attention_workspace_size(desc: TvAttnDesc) -> int:
+    return int(lib().tv_tree_attention_workspace_size(ctypes.byref(desc)))
+
+
+def tv_tree_attention(desc, q, paged_k, paged_v, block_table, prefix_lens, parent_idx, out,
+                      workspace=None, workspace_bytes: int = 0, dev_status=None, stream=None) -> int:
+    return int(lib().tv_tree_attention(ctypes.byref(desc), _ptr(q), _ptr(paged_k), _ptr(paged_v), _ptr(block_table),
+                                       _ptr(prefix_lens), _ptr(parent_idx), _ptr(out), _ptr(workspace),
+                                       int(workspace_bytes), _ptr(dev_status), _stream(stream)))
+
+
+def tv_verify_sample_plan(desc: TvSampleDesc) -> TvSamplePlan:
+    plan = TvSamplePlan()
+    s = lib().tv_verify_sample_plan(ctypes.byref(desc), ctypes.byref(plan))
+    if s != TV_OK:
+        raise TreeVerifyError(s, "tv_verify_sample_plan")
+    return plan
+
+
+def tv_verify_sample_workspace_size(desc: TvSampleDesc) -> int:
+    return int(lib().tv_verify_sample_workspace_size(ctypes.byref(desc)))
+
+
+def tv_verify_sample(desc, p, q, tree_tokens, parent_idx, uniforms, accepted_path, accepted_len, bonus_token,
+                     workspace=None, workspace_bytes: int = 0, dev_status=None, stream=None) -> int:
+    return int(lib().tv_verify_sample(ctypes.byref(desc), _ptr(p), _ptr(q), _ptr(tree_tokens), _ptr(parent_idx),
+                                      _ptr(uniforms), _ptr(accepted_path), _ptr(accepted_len), _ptr(bonus_token),
+                                      _ptr(workspace), int(workspace_bytes), _ptr(dev_status), _stream(stream)))
+
+
+# ------------------------------------------------------------ torch conveniences
+
+def attn_desc(q, k_cache, block_table, softmax_scale: float = 0.0) -> TvAttnDesc:
+    """Descriptor from tensors: q [B][N][Hq][D], cache [nb][16][Hkv][D],
+    block_table [B][max_blocks]."""
+    import torch
+    B, N, Hq, D = q.shape
+    nb, bs, Hkv, D2 = k_cache.shape
+    if D2 != D:
+        raise ValueError("head_dim mismatch between q and cache")
+    dt = {torch.bfloat16: TV_BF16, torch.float32: TV_F32}.get(q.dtype)
+    if dt is None:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    return TvAttnDesc(B, N, Hq, Hkv, D, bs, block_table.shape[1], nb, dt, float(softmax_scale))
+
+
+def _check_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("all tensors must be contiguous CUDA tensors")
+
+
+def tree_attention(q, k_cache, v_cache, block_table, prefix_lens, parent_idx, softmax_scale: float = 0.0,
+                   out=None, workspace=None, dev_status=None, stream=None):
+    """Run tv_tree_attention; allocates `out` (and workspace) when not given."""
+    import torch
+    _check_cuda(q, k_cache, v_cache, block_table, prefix_lens, parent_idx, out, workspace, dev_status)
+    if k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
+        raise TypeError("q, k_cache and v_cache must share a dtype")
+    for t in (block_table, prefix_lens, parent_idx):
+        if t.dtype != torch.int32:
+            raise TypeError("block_table, prefix_lens and parent_idx must be int32")
+    desc = attn_desc(q, k_cache, block_table, softmax_scale)
+    if out is None:
+        out = torch.empty_like(q)
+    ws_bytes = tv_tree_attention_workspace_size(desc)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    s = tv_tree_attention(desc, q, k_cache, v_cache, block_table, prefix_lens, parent_idx, out, workspace,
+                          workspace.numel() if workspace is not None else 0, dev_status, stream)
+    if s != TV_OK:
+        raise TreeVerifyError(s, "tv_tree_attention")
+    return out
+
+
+def verify_sample(p, q, tree_tokens, parent_idx, uniforms, accepted_path=None, accepted_len=None,
+                  bonus_token=None, dev_status=None, stream=None):
+    """Run tv_verify_sample; returns (accepted_path, accepted_len, bonus_token)."""
+    import torch
+    _check_cuda(p, q, tree_tokens, parent_idx, uniforms, dev_status)
+    if p.dtype != torch.float32 or q.dtype != torch.float32 or uniforms.dtype != torch.float32:
+        raise TypeError("p, q and uniforms must be float32")
+    B, N, V = p.shape
+    dev = p.device
+    if accepted_path is None:
+        accepted_path = torch.empty((B, N), dtype=torch.int32, device=dev)
+    if accepted_len is None:
+        accepted_len = torch.empty((B,), dtype=torch.int32, device=dev)
+    if bonus_token is None:
+        bonus_token = torch.empty((B,), dtype=torch.int32, device=dev)
+    desc = TvSampleDesc(B, N, V)
+    s = tv_verify_sample(desc, p, q, tree_tokens, parent_idx, uniforms, accepted_path, accepted_len, bonus_token,
+                         None, 0, dev_status, stream)
+    if s != TV_OK:
+        raise TreeVerifyError(s, "tv_verify_sample")
+    return accepted_path, accepted_len, bonus_token

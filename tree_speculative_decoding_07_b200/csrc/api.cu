@@ -1,0 +1,218 @@
+// api.cu -- host side of libtreeverify: argument checks, launch planning and
+// the extern "C" entry points declared in include/treeverify.h.
+#include <math.h>
+#include <stdint.h>
+
+#include "kernels.h"
+#include "tv_common.cuh"
+
+namespace {
+
+int device_sms() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+        return sms;
+    cudaGetLastError();
+    return 148;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+tv_status check_attn_desc(const tv_attn_desc* d) {
+    if (!d) return TV_ERR_INVALID_ARG;
+    if (d->batch < 1 || d->num_nodes < 1 || d->num_q_heads < 1 || d->num_kv_heads < 1) return TV_ERR_INVALID_ARG;
+    if (d->num_q_heads % d->num_kv_heads) return TV_ERR_INVALID_ARG;
+    if (d->num_nodes > TV_MAX_NODES_ATTN) return TV_ERR_UNSUPPORTED;
+    if (d->head_dim != 64 && d->head_dim != 128) return TV_ERR_UNSUPPORTED;
+    if (d->block_size != TV_BLOCK) return TV_ERR_UNSUPPORTED;
+    if (d->max_blocks_per_seq < 1 || d->num_blocks < 1) return TV_ERR_INVALID_ARG;
+    if (d->dtype != TV_BF16 && d->dtype != TV_F32) return TV_ERR_INVALID_ARG;
+    if (!(d->softmax_scale >= 0.f) || isinf(d->softmax_scale)) return TV_ERR_INVALID_ARG;
+    if ((int64_t)d->max_blocks_per_seq * TV_BLOCK > INT32_MAX / 2) return TV_ERR_UNSUPPORTED;
+    return TV_OK;
+}
+
+// Which kernel runs and how the KV range is split.
+//  - bf16 with head_dim 128 runs on the tensor cores: 128-row query tiles,
+//    the KV splits of one tile form a thread-block cluster that merges its
+//    partial results through distributed shared memory (no workspace).
+//  - everything else runs on the CUDA cores: 32-row tiles, splits merged by
+//    a second kernel through a global workspace.
+// Splits are chosen so the main launch covers the SMs about once, and never
+// below 256 tokens per split.
+void make_plan(const tv_attn_desc* d, tv_attn_plan* p) {
+    const int G = d->num_q_heads / d->num_kv_heads;
+    const int rows = G * d->num_nodes;
+    const int sms = device_sms();
+    const int64_t max_tokens = (int64_t)d->max_blocks_per_seq * TV_BLOCK;
+    const bool tc = d->dtype == TV_BF16 && d->head_dim == 128;
+    p->kernel = tc ? 0 : 1;
+    const int tile_rows = tc ? tv::tc_rows_per_tile() : tv::simt_rows_per_tile();
+    p->row_tiles = (rows + tile_rows - 1) / tile_rows;
+    const int64_t base = (int64_t)d->batch * d->num_kv_heads * p->row_tiles;
+    int64_t splits = base >= sms ? 1 : (sms / base);
+    const int64_t by_len = (max_tokens + 255) / 256;
+    if (splits > by_len) splits = by_len;
+    if (splits < 1) splits = 1;
+    if (tc) {
+        // cluster sizes 1, 2, 4 or 8
+        if (splits > tv::tc_max_cluster()) splits = tv::tc_max_cluster();
+        int64_t pow2 = 1;
+        while (pow2 * 2 <= splits) pow2 *= 2;
+        splits = pow2;
+    }
+    if (!tc && splits > 64) splits = 64;
+    p->num_splits = (int32_t)splits;
+    p->grid_ctas = (int32_t)(base * splits);
+    p->launches = (!tc && splits > 1) ? 2 : 1;
+    size_t ws = 0;
+    if (!tc && splits > 1) {
+        const size_t rows_all = (size_t)d->batch * d->num_nodes * d->num_q_heads;
+        ws = align256(sizeof(float) * splits * rows_all * d->head_dim) + align256(sizeof(float) * splits * rows_all);
+    }
+    p->workspace_bytes = ws;
+}
+
+tv_status check_sample_desc(const tv_sample_desc* d) {
+    if (!d) return TV_ERR_INVALID_ARG;
+    if (d->batch < 1 || d->num_nodes < 1 || d->vocab < 1) return TV_ERR_INVALID_ARG;
+    if (d->num_nodes > 1024) return TV_ERR_UNSUPPORTED;
+    if (d->vocab > 16 * 24576) return TV_ERR_UNSUPPORTED;
+    if ((int64_t)d->batch * 16 > INT32_MAX) return TV_ERR_UNSUPPORTED;
+    return TV_OK;
+}
+
+// One cluster per sequence; each CTA caches a slice of about 8K entries of
+// a row's p and q (64 KB) so a 128K-entry row spreads over 16 SMs.
+void make_sample_plan(const tv_sample_desc* d, tv_sample_plan* p) {
+    const int max_c = tv::sample_max_cluster();
+    int c = (d->vocab + 8191) / 8192;
+    if (c > max_c) c = max_c;
+    if (c < 1) c = 1;
+    int slice = (d->vocab + c - 1) / c;
+    slice = (slice + 3) / 4 * 4;
+    int threads = ((slice + 7) / 8 + 31) / 32 * 32;
+    if (threads < 64) threads = 64;
+    if (threads > 512) threads = 512;
+    p->cluster_ctas = c;
+    p->threads = threads;
+    p->slice = slice;
+    p->smem_bytes = (int32_t)(2 * sizeof(float) * (size_t)slice);
+    p->launches = 1;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t tv_version(void) { return 100; }
+
+const char* tv_status_string(int32_t s) {
+    switch (s) {
+        case TV_OK: return "ok";
+        case TV_ERR_INVALID_ARG: return "invalid argument";
+        case TV_ERR_UNSUPPORTED: return "unsupported configuration";
+        case TV_ERR_TREE: return "malformed tree (parent not before child, bad root, or token out of range)";
+        case TV_ERR_BLOCK_TABLE: return "block table entry out of range or sequence longer than the table";
+        case TV_ERR_WORKSPACE: return "workspace missing or too small";
+        case TV_ERR_CUDA: return "CUDA runtime error";
+        case TV_ERR_TIMEOUT: return "bounded device wait ran out";
+        default: return "unknown status";
+    }
+}
+
+tv_status tv_tree_attention_plan(const tv_attn_desc* desc, tv_attn_plan* plan) {
+    tv_status s = check_attn_desc(desc);
+    if (s != TV_OK) return s;
+    if (!plan) return TV_ERR_INVALID_ARG;
+    make_plan(desc, plan);
+    return TV_OK;
+}
+
+size_t tv_tree_attention_workspace_size(const tv_attn_desc* desc) {
+    if (check_attn_desc(desc) != TV_OK) return 0;
+    tv_attn_plan p;
+    make_plan(desc, &p);
+    return p.workspace_bytes;
+}
+
+tv_status tv_tree_attention(const tv_attn_desc* desc, const void* q, const void* paged_k, const void* paged_v,
+                            const int32_t* block_table, const int32_t* prefix_lens, const int32_t* parent_idx,
+                            void* out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                            void* stream) {
+    tv_status s = check_attn_desc(desc);
+    if (s != TV_OK) return s;
+    if (!q || !paged_k || !paged_v || !block_table || !prefix_lens || !parent_idx || !out)
+        return TV_ERR_INVALID_ARG;
+    tv_attn_plan plan;
+    make_plan(desc, &plan);
+    if (plan.kernel == 0) {
+        // the tensor-core path reads q, K and V with 16-byte vector loads / TMA
+        const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(paged_k) |
+                              reinterpret_cast<uintptr_t>(paged_v) | reinterpret_cast<uintptr_t>(out);
+        if (mis & 15) return TV_ERR_INVALID_ARG;
+    }
+    if (plan.workspace_bytes) {
+        if (!workspace || workspace_bytes < plan.workspace_bytes) return TV_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(workspace) & 255) return TV_ERR_WORKSPACE;
+    }
+    tv::AttnArgs a = {};
+    a.q = q; a.k = paged_k; a.v = paged_v;
+    a.block_table = block_table; a.prefix_lens = prefix_lens; a.parent = parent_idx;
+    a.out = out; a.status = dev_status;
+    a.B = desc->batch; a.N = desc->num_nodes; a.Hq = desc->num_q_heads; a.Hkv = desc->num_kv_heads;
+    a.G = a.Hq / a.Hkv; a.D = desc->head_dim; a.max_blocks = desc->max_blocks_per_seq;
+    a.num_blocks = desc->num_blocks; a.splits = plan.num_splits; a.row_tiles = plan.row_tiles;
+    const float scale = desc->softmax_scale > 0.f ? desc->softmax_scale : 1.0f / sqrtf((float)desc->head_dim);
+    a.scale_log2 = scale * 1.4426950408889634f;
+    if (plan.workspace_bytes) {
+        const size_t rows_all = (size_t)a.B * a.N * a.Hq;
+        a.o_part = static_cast<float*>(workspace);
+        a.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                              align256(sizeof(float) * a.splits * rows_all * a.D));
+    }
+    int launches = 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = plan.kernel == 0 ? tv::launch_attn_tc(a, st, &launches)
+                                     : tv::launch_attn_simt(a, desc->dtype == TV_BF16, st, &launches);
+    return e == cudaSuccess ? TV_OK : TV_ERR_CUDA;
+}
+
+tv_status tv_verify_sample_plan(const tv_sample_desc* desc, tv_sample_plan* plan) {
+    tv_status s = check_sample_desc(desc);
+    if (s != TV_OK) return s;
+    if (!plan) return TV_ERR_INVALID_ARG;
+    make_sample_plan(desc, plan);
+    return TV_OK;
+}
+
+size_t tv_verify_sample_workspace_size(const tv_sample_desc* desc) {
+    (void)desc;
+    return 0;
+}
+
+tv_status tv_verify_sample(const tv_sample_desc* desc, const float* p, const float* q, const int32_t* tree_tokens,
+                           const int32_t* parent_idx, const float* uniforms, int32_t* accepted_path,
+                           int32_t* accepted_len, int32_t* bonus_token, void* workspace, size_t workspace_bytes,
+                           int32_t* dev_status, void* stream) {
+    (void)workspace;
+    (void)workspace_bytes;
+    tv_status s = check_sample_desc(desc);
+    if (s != TV_OK) return s;
+    if (!p || !q || !tree_tokens || !parent_idx || !uniforms || !accepted_path || !accepted_len || !bonus_token)
+        return TV_ERR_INVALID_ARG;
+    tv_sample_plan plan;
+    make_sample_plan(desc, &plan);
+    tv::SampleArgs a = {};
+    a.p = p; a.q = q; a.tokens = tree_tokens; a.parent = parent_idx; a.uniforms = uniforms;
+    a.path = accepted_path; a.len = accepted_len; a.bonus = bonus_token; a.status = dev_status;
+    a.B = desc->batch; a.N = desc->num_nodes; a.V = desc->vocab;
+    a.cluster = plan.cluster_ctas; a.threads = plan.threads; a.slice = plan.slice; a.smem_bytes = plan.smem_bytes;
+    a.vec4 = (desc->vocab % 4 == 0) && !(reinterpret_cast<uintptr_t>(p) & 15) && !(reinterpret_cast<uintptr_t>(q) & 15);
+    int launches = 0;
+    cudaError_t e = tv::launch_verify_sample(a, static_cast<cudaStream_t>(stream), &launches);
+    return e == cudaSuccess ? TV_OK : TV_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,51 @@
+// kernels.h -- launch interfaces between the host API (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tv {
+
+struct AttnArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const int32_t* block_table;
+    const int32_t* prefix_lens;
+    const int32_t* parent;
+    void* out;
+    float* o_part;      // [splits][B][N][Hq][D] fp32 partial outputs (normalised)
+    float* lse_part;    // [splits][B][N][Hq] log2-domain log-sum-exp of each partial
+    int32_t* status;
+    int B, N, Hq, Hkv, G, D, max_blocks, num_blocks, splits, row_tiles;
+    float scale_log2;   // softmax_scale * log2(e)
+};
+
+// CUDA-core split-KV kernel (fp32 or bf16 storage, fp32 math) + LSE combine.
+cudaError_t launch_attn_simt(const AttnArgs& a, bool bf16, cudaStream_t st, int* launches);
+int simt_rows_per_tile();
+
+// Tensor-core (tcgen05 / TMEM / TMA) bf16 kernel, head_dim 128.
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st, int* launches);
+int tc_rows_per_tile();
+int tc_max_cluster();
+
+struct SampleArgs {
+    const float* p;
+    const float* q;
+    const int32_t* tokens;
+    const int32_t* parent;
+    const float* uniforms;
+    int32_t* path;
+    int32_t* len;
+    int32_t* bonus;
+    int32_t* status;
+    int B, N, V;
+    int cluster, threads, slice, smem_bytes;
+    int vec4;           // rows start 16-byte aligned and V % 4 == 0
+};
+
+cudaError_t launch_verify_sample(const SampleArgs& a, cudaStream_t st, int* launches);
+int sample_max_cluster();
+
+}  // namespace tv
