@@ -175,28 +175,47 @@ def run_ours(args, rank, world, local_rank):
     adesc = tv.attn_desc(d["query"], d["k"], d["block_table"])
     aplan = tv.tv_tree_attention_plan(adesc)
     ws_bytes = aplan.workspace_bytes
-    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
     sdesc = tv.TvSampleDesc(B, N, wl.vocab)
     splan = tv.tv_verify_sample_plan(sdesc)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
-    def step(dd, o, pth, ln, bn, mid):
-        s1 = tv.tv_tree_attention(adesc, dd["query"], dd["k"], dd["v"], dd["block_table"], dd["prefix_lens"],
-                                  dd["parent_idx"], o, ws, ws_bytes, status, stream)
-        mid.record(stream)
-        s2 = tv.tv_verify_sample(sdesc, dd["p"], dd["q"], dd["tokens"], dd["parent_idx"], dd["uniforms"], pth, ln,
-                                 bn, None, 0, status, stream)
-        if s1 or s2:
-            raise tv.TreeVerifyError(s1 or s2, "verify step")
+    def attn_call(st):
+        s1 = tv.tv_tree_attention(adesc, d["query"], d["k"], d["v"], d["block_table"], d["prefix_lens"],
+                                  d["parent_idx"], out, ws, ws_bytes, status, st)
+        if s1:
+            raise tv.TreeVerifyError(s1, "tv_tree_attention")
 
-    # ---- device-resident timing (L2 flushed before every step)
+    def sample_call(st):
+        s2 = tv.tv_verify_sample(sdesc, d["p"], d["q"], d["tokens"], d["parent_idx"], d["uniforms"], path, alen,
+                                 bonus, None, 0, status, st)
+        if s2:
+            raise tv.TreeVerifyError(s2, "tv_verify_sample")
+
+    def step(mid):
+        attn_call(stream)
+        mid.record(stream)
+        sample_call(stream)
+
+    # ---- device-resident timing (L2 flushed before every step).  Each call is
+    # replayed from a CUDA graph so host launch work stays out of the events.
     W, K = args.warmup, args.steps
+    for _ in range(2):
+        step(torch.cuda.Event())
+    torch.cuda.synchronize()
+    g_attn, g_samp = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_attn):
+        attn_call(torch.cuda.current_stream())
+    with torch.cuda.graph(g_samp):
+        sample_call(torch.cuda.current_stream())
+    torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     for _ in range(W):
         flush.zero_()
-        step(d, out, path, alen, bonus, torch.cuda.Event())
+        g_attn.replay()
+        g_samp.replay()
     torch.cuda.synchronize()
     clocks = ClockSampler(local_rank)
     if world > 1:
@@ -208,7 +227,9 @@ def run_ours(args, rank, world, local_rank):
         flush.zero_()
         e0, mid, e1 = ev[k]
         e0.record(stream)
-        step(d, out, path, alen, bonus, mid)
+        g_attn.replay()
+        mid.record(stream)
+        g_samp.replay()
         e1.record(stream)
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall
@@ -237,7 +258,7 @@ def run_ours(args, rank, world, local_rank):
         for key, t in pin.items():
             dst = d[key]
             (dst.view(torch.int16) if dst.dtype == torch.bfloat16 else dst).copy_(t, non_blocking=True)
-        step(d, out, path, alen, bonus, torch.cuda.Event())
+        step(torch.cuda.Event())
         out_h.copy_(out, non_blocking=True)
         path_h.copy_(path, non_blocking=True)
         alen_h.copy_(alen, non_blocking=True)

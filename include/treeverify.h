@@ -110,8 +110,10 @@ typedef struct {
 TV_API tv_status tv_tree_attention_plan(const tv_attn_desc *desc, tv_attn_plan *plan);
 
 /* Device workspace the call needs, in bytes (0 when none).  Ownership stays
- * with the caller; it must be 256-byte aligned and may be reused across
- * calls that are ordered on one stream. */
+ * with the caller; it must be 256-byte aligned, zero-filled before its first
+ * use (e.g. one cudaMemset at allocation), and may be reused across calls
+ * that are ordered on one stream: every call leaves its synchronisation
+ * counters at zero again.  Calls that share a workspace must not overlap. */
 TV_API size_t tv_tree_attention_workspace_size(const tv_attn_desc *desc);
 
 TV_API tv_status tv_tree_attention(const tv_attn_desc *desc, const void *q, const void *paged_k,

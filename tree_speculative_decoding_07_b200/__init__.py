@@ -182,7 +182,7 @@ def tree_attention(q, k_cache, v_cache, block_table, prefix_lens, parent_idx, so
         out = torch.empty_like(q)
     ws_bytes = tv_tree_attention_workspace_size(desc)
     if ws_bytes and workspace is None:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+        workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=q.device)
     s = tv_tree_attention(desc, q, k_cache, v_cache, block_table, prefix_lens, parent_idx, out, workspace,
                           workspace.numel() if workspace is not None else 0, dev_status, stream)
     if s != TV_OK:

@@ -34,13 +34,14 @@ tv_status check_attn_desc(const tv_attn_desc* d) {
 }
 
 // Which kernel runs and how the KV range is split.
-//  - bf16 with head_dim 128 runs on the tensor cores: 128-row query tiles,
-//    the KV splits of one tile form a thread-block cluster that merges its
-//    partial results through distributed shared memory (no workspace).
+//  - bf16 with head_dim 128 runs on the tensor cores: 128-row query tiles;
+//    with several KV splits the launch is cooperative and the splits of a
+//    tile merge their partial results through the workspace.
 //  - everything else runs on the CUDA cores: 32-row tiles, splits merged by
 //    a second kernel through a global workspace.
-// Splits are chosen so the main launch covers the SMs about once, and never
-// below 256 tokens per split.
+// Splits are chosen so the main launch covers the SMs about once (for the
+// tensor-core path: as many as keep the whole grid resident), and never below
+// 256 tokens per split.
 void make_plan(const tv_attn_desc* d, tv_attn_plan* p) {
     const int G = d->num_q_heads / d->num_kv_heads;
     const int rows = G * d->num_nodes;
@@ -51,22 +52,21 @@ void make_plan(const tv_attn_desc* d, tv_attn_plan* p) {
     const int tile_rows = tc ? tv::tc_rows_per_tile() : tv::simt_rows_per_tile();
     p->row_tiles = (rows + tile_rows - 1) / tile_rows;
     const int64_t base = (int64_t)d->batch * d->num_kv_heads * p->row_tiles;
-    int64_t splits = base >= sms ? 1 : (sms / base);
-    const int64_t by_len = (max_tokens + 255) / 256;
-    if (splits > by_len) splits = by_len;
-    if (splits < 1) splits = 1;
+    int64_t splits;
     if (tc) {
-        // cluster sizes 1, 2, 4 or 8
-        if (splits > tv::tc_max_cluster()) splits = tv::tc_max_cluster();
-        int64_t pow2 = 1;
-        while (pow2 * 2 <= splits) pow2 *= 2;
-        splits = pow2;
+        splits = tv::tc_pick_splits(base, max_tokens, sms);
+    } else {
+        splits = base >= sms ? 1 : (sms / base);
+        const int64_t by_len = (max_tokens + 255) / 256;
+        if (splits > by_len) splits = by_len;
+        if (splits < 1) splits = 1;
+        if (splits > 64) splits = 64;
     }
-    if (!tc && splits > 64) splits = 64;
     p->num_splits = (int32_t)splits;
     p->grid_ctas = (int32_t)(base * splits);
     p->launches = (!tc && splits > 1) ? 2 : 1;
     size_t ws = 0;
+    if (tc) ws = tv::tc_workspace_bytes(base, (int)splits);
     if (!tc && splits > 1) {
         const size_t rows_all = (size_t)d->batch * d->num_nodes * d->num_q_heads;
         ws = align256(sizeof(float) * splits * rows_all * d->head_dim) + align256(sizeof(float) * splits * rows_all);
@@ -166,7 +166,12 @@ tv_status tv_tree_attention(const tv_attn_desc* desc, const void* q, const void*
     a.num_blocks = desc->num_blocks; a.splits = plan.num_splits; a.row_tiles = plan.row_tiles;
     const float scale = desc->softmax_scale > 0.f ? desc->softmax_scale : 1.0f / sqrtf((float)desc->head_dim);
     a.scale_log2 = scale * 1.4426950408889634f;
-    if (plan.workspace_bytes) {
+    if (plan.workspace_bytes && plan.kernel == 0) {
+        const int64_t groups = (int64_t)a.B * a.Hkv * a.row_tiles;
+        a.o_part = static_cast<float*>(workspace);
+        a.counters = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) +
+                                                 tv::tc_counter_offset(groups, a.splits));
+    } else if (plan.workspace_bytes) {
         const size_t rows_all = (size_t)a.B * a.N * a.Hq;
         a.o_part = static_cast<float*>(workspace);
         a.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +

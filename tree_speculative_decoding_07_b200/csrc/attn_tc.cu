@@ -6,60 +6,80 @@
 //
 // Decomposition.  The G query heads that share a KV head, times the N tree
 // nodes, form the query rows of one (sequence, KV head): row r is node r / G,
-// head r % G.  A CTA owns one 128-row tile of those rows and one KV split;
-// the splits of a tile form a thread-block cluster and merge their partial
-// results through distributed shared memory at the end (flash-decoding
-// log-sum-exp merge), so nothing goes through global scratch memory.
+// head r % G, so each K/V row is read once for all G heads.  A CTA owns one
+// 128-row tile of those rows and one KV split.  With several splits the grid
+// is launched cooperatively (all CTAs resident at once, one per SM); the
+// splits of a tile write their partial results to an L2-resident workspace,
+// count themselves in on a per-tile arrival counter, and once all S have
+// arrived each combines an equal share of the rows (flash-decoding
+// log-sum-exp merge).  The last split to leave resets the counters, so the
+// workspace is ready for the next call.
 //
-// Per 128-token KV tile (8 paged blocks of 16 tokens):
-//   producer warp   TMA-loads the K and V rows of the 8 blocks (one 2 KB box
-//                   per block and 64-column half, 128-byte swizzle) into a
-//                   two-stage ring; block ids come from the block table.
-//   MMA warp        S = Q K^T (tcgen05.mma kind::f16, M 128, N 128, K 16 x 8)
-//                   into one of two TMEM S buffers, then O += P V into the
-//                   TMEM accumulator once the softmax warps published P.
-//   softmax warps   one thread per query row (TMEM lane): read the row of S,
-//                   scale, apply the tree mask on the tree block, keep an
-//                   online max / sum in the log2 domain (the O rescale in
-//                   TMEM is skipped while the max grows by at most 2^8), write
-//                   P as bf16 into shared memory in the MMA's swizzled layout.
-// The tree mask is a 128-bit ancestor set per node, built from parent_idx in
-// the prologue (anc(i) = anc(parent(i)) | {i}) and shifted into column space
-// once per tile.
+// Warp roles (384 threads):
+//   warp 0      TMA producer: K and V rows of 8 paged blocks per 128-token
+//               tile (one 2 KB box per block and 64-column half, 128-byte
+//               swizzle) into a 3-deep K ring and a 2-deep V ring; a K slot
+//               is refilled as soon as its S = Q K^T has finished.
+//   warp 1      MMA issuer: S = Q K^T (tcgen05.mma kind::f16, M 128, N 128,
+//               8 x K16) into one of two TMEM S buffers; then, per softmax
+//               warpgroup, O_x += P_x V_x over that group's 64 tokens.
+//   warp 2      TMEM allocation (all 512 columns).
+//   warps 4-7   softmax group A: columns 0..63 of every S tile
+//   warps 8-11  softmax group B: columns 64..127
+// Each softmax thread owns one query row (its TMEM lane).  The two groups
+// keep separate running maxima / sums and separate O accumulators, so they
+// never wait on each other inside the loop; their halves are merged at the
+// end like two extra splits.  Scores are scaled into the log2 domain by the
+// same FFMA that subtracts the running max; the O rescale in TMEM is skipped
+// while the max grows by at most 2^8.  P is written as bf16 into shared
+// memory in the MMA's swizzled K-major layout.  The tree mask is a 128-bit
+// ancestor set per node (anc(i) = anc(parent(i)) | {i}), shifted into column
+// space once per tile; prefix-only tiles skip it.
 //
-// Every wait on an mbarrier is bounded (about two seconds of clock); on expiry
-// the CTA records TV_ERR_TIMEOUT, stops issuing work, writes NaN rows, frees
-// its TMEM and still takes part in the cluster barriers so no peer is left
-// waiting.
+// Every wait (mbarrier phase or arrival counter) is bounded (about two
+// seconds of clock); on expiry the CTA records TV_ERR_TIMEOUT, stops issuing
+// work, writes NaN rows, frees its TMEM and still counts itself in and out
+// so no peer is left waiting and the counters return to zero.
 #include <cuda.h>
-#include <cooperative_groups.h>
 
 #include "tv_common.cuh"
 #include "kernels.h"
 
-namespace cg = cooperative_groups;
-
 namespace tv {
 namespace {
 
-constexpr int TC_THREADS = 256;
+constexpr int TC_THREADS = 384;
 constexpr int TM = 128;          // query rows per CTA (TMEM lanes)
 constexpr int TN = 128;          // KV tokens per tile
+constexpr int HALF_N = TN / 2;   // tokens per softmax group
 constexpr int HD = 128;          // head dim
 constexpr int BLK_PER_TILE = TN / TV_BLOCK;
-constexpr int STAGES = 2;
-constexpr int MAX_CLUSTER = 8;
-constexpr uint32_t SQ_OFF = 0;           // Q: 2 x [128 rows][128 B], swizzled
-constexpr uint32_t SP_OFF = 32768;       // P: 2 x [128 rows][128 B], swizzled
-constexpr uint32_t SKV_OFF = 65536;      // stage s: K at +0 (32 KB), V at +32 KB
-constexpr uint32_t STAGE_BYTES = 65536;
-constexpr uint32_t HALF_BYTES = 16384;   // one 64-column half of a 128-row operand
-constexpr uint32_t TILE_TX_BYTES = 2 * 2 * BLK_PER_TILE * 2048;  // K and V, 2 halves, 8 blocks
-constexpr uint32_t SMEM_BYTES = SKV_OFF + STAGES * STAGE_BYTES + 1024;
-constexpr int OPITCH = HD + 4;           // floats per row when staging partial outputs
-constexpr uint32_t TMEM_COLS = 512;      // S0 [0,128), S1 [128,256), O [256,384)
+constexpr int KST = 3;           // K ring depth
+constexpr int VST = 3;           // V ring depth
+constexpr int MAX_SPLITS = 16;
+constexpr uint32_t SQ_OFF = 0;             // Q: 2 x [128 rows][128 B], swizzled
+constexpr uint32_t SK_OFF = 32768;         // K ring: KST x 32 KB
+constexpr uint32_t SV_OFF = SK_OFF + KST * 32768u;  // V ring: VST x 32 KB
+constexpr uint32_t TILE_BYTES = 32768;     // one K or V tile: 2 halves x 128 rows x 128 B
+constexpr uint32_t HALF_BYTES = 16384;
+constexpr uint32_t SMEM_BYTES = SV_OFF + VST * 32768u + 1024;
+constexpr int RPITCH = HD + 4;             // floats per workspace partial row: 128 outputs, lse, padding
+constexpr uint32_t TMEM_COLS = 512;        // S0 [0,128), S1 [128,256), O_A [256,384), O_B [384,512)
 constexpr uint32_t O_COL = 256;
 constexpr long long WAIT_LIMIT = 1ll << 32;  // clock cycles (~2 s)
+
+// mbarrier slots, derived from the ring depths
+constexpr int BAR_K_FULL = 0;                    // KST: K tile landed (TMA transaction count)
+constexpr int BAR_K_EMPTY = BAR_K_FULL + KST;    // KST: S = Q K^T done with the K slot
+constexpr int BAR_V_FULL = BAR_K_EMPTY + KST;    // VST: V tile landed
+constexpr int BAR_V_EMPTY = BAR_V_FULL + VST;    // VST: P V done with the V slot
+constexpr int BAR_S_FULL = BAR_V_EMPTY + VST;    // 2: S buffer written
+constexpr int BAR_P_FULL = BAR_S_FULL + 2;       // 2: group's P written (and O rescaled)
+constexpr int BAR_O_DONE = BAR_P_FULL + 2;       // 2: group's P V done
+constexpr int BAR_Q_READY = BAR_O_DONE + 2;      // Q staged
+constexpr int BAR_DRAIN = BAR_Q_READY + 1;       // all MMAs of the CTA done
+constexpr int BAR_COUNT = BAR_DRAIN + 1;
+static_assert(BAR_COUNT == 2 * KST + 2 * VST + 8, "barrier slots overlap");
 
 // instruction descriptor, kind::f16: D fp32, A/B bf16, A K-major,
 // B K-major (S = Q K^T) or MN-major (O += P V), M = 128, N = 128
@@ -135,6 +155,16 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D (TMEM) += A (TMEM, bf16 pairs per 32-bit column) * B (shared memory descriptor)
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
@@ -200,14 +230,96 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
     return __all_sync(0xffffffffu, ok);
 }
 
+// per-tile arrival counter: increment after a release fence, bounded
+// acquire spin for the target count
+__device__ __forceinline__ unsigned count_in(unsigned* cnt) {
+    __threadfence();
+    return atomicAdd(cnt, 1u);
+}
+__device__ __forceinline__ bool wait_count(const unsigned* cnt, unsigned target, volatile int* abort_flag) {
+    const long long t0 = clock64();
+    for (;;) {
+        unsigned v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+        if (v >= target) return true;
+        if (clock64() - t0 > WAIT_LIMIT) {
+            *abort_flag = 1;
+            return false;
+        }
+        __nanosleep(32);
+    }
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+// Combine rows [split * R, split * R + R) of one 128-row tile from the S
+// partials in the workspace (layout [S][128][RPITCH]: 128 outputs, lse):
+// out = sum_s 2^(lse_s - m) o_s / sum_s 2^(lse_s - m), m = max_s lse_s.
+template <int S_>
+__device__ __forceinline__ void merge_rows(const AttnArgs& a, const float* part, int split, int tile, int b, int kvh,
+                                           int tid) {
+    constexpr int R = (TM + S_ - 1) / S_;
+    const int own = max(0, min(TM, (split + 1) * R) - split * R);
+    for (int item = tid; item < own * (HD / 4); item += TC_THREADS) {
+        const int rr = item / (HD / 4), c4 = item % (HD / 4);
+        const int rt = split * R + rr;
+        const int gr = tile * TM + rt;
+        if (gr >= a.G * a.N) continue;
+        float ls[S_];
+        float4 v[S_];
+#pragma unroll
+        for (int k = 0; k < S_; ++k) {
+            const float* prow = part + ((size_t)k * TM + rt) * RPITCH;
+            ls[k] = prow[HD];
+            v[k] = reinterpret_cast<const float4*>(prow)[c4];
+        }
+        float mx = -INFINITY;
+        bool nan = false;
+#pragma unroll
+        for (int k = 0; k < S_; ++k) {
+            nan |= isnan(ls[k]);
+            mx = fmaxf(mx, ls[k]);
+        }
+        float den = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < S_; ++k) {
+            const float w = ls[k] == -INFINITY ? 0.f : ex2(ls[k] - mx);
+            den += w;
+            acc.x = fmaf(w, v[k].x, acc.x);
+            acc.y = fmaf(w, v[k].y, acc.y);
+            acc.z = fmaf(w, v[k].z, acc.z);
+            acc.w = fmaf(w, v[k].w, acc.w);
+        }
+        const bool dead = nan || !(den > 0.f);
+        const float id = dead ? 0.f : 1.f / den;
+        const int node = gr / a.G, head = kvh * a.G + gr % a.G;
+        uint2 ov;
+        ov.x = pack_bf16(dead ? NAN : acc.x * id, dead ? NAN : acc.y * id);
+        ov.y = pack_bf16(dead ? NAN : acc.z * id, dead ? NAN : acc.w * id);
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + (((size_t)b * a.N + node) * a.Hq + head) * HD +
+                                  c4 * 4) = ov;
+    }
+}
+
+template <int NV>
+__device__ __forceinline__ float max_tree(const float (&v)[NV]) {
+    float m[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m[k] = v[k];
+#pragma unroll
+    for (int i = 8; i < NV; ++i) m[i & 7] = fmaxf(m[i & 7], v[i]);
+    return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+
 __global__ void __launch_bounds__(TC_THREADS, 1)
     attn_tc_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
     extern __shared__ uint8_t dsmem[];
-    __shared__ __align__(8) uint64_t bars[12];
+    __shared__ __align__(8) uint64_t bars[BAR_COUNT];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort, s_bad;
     __shared__ int32_t s_par[TV_MAX_NODES_ATTN];
-    __shared__ float s_lse[TM];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int split = blockIdx.x, tile = blockIdx.y;
@@ -216,35 +328,44 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const uint32_t raw = smem_u32(dsmem);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* base_ptr = dsmem + (base - raw);
-    const uint32_t sQ = base + SQ_OFF, sP = base + SP_OFF, sKV = base + SKV_OFF;
+    const uint32_t sQ = base + SQ_OFF;
+    auto sK = [&](int s) { return base + SK_OFF + (uint32_t)s * TILE_BYTES; };
+    auto sV = [&](int s) { return base + SV_OFF + (uint32_t)s * TILE_BYTES; };
     const uint32_t bar0 = smem_u32(&bars[0]);
-    auto kv_full = [&](int s) { return bar0 + 8u * (0 + s); };
-    auto kv_empty = [&](int s) { return bar0 + 8u * (2 + s); };
-    auto s_full = [&](int s) { return bar0 + 8u * (4 + s); };
-    auto s_free = [&](int s) { return bar0 + 8u * (6 + s); };
-    const uint32_t p_full = bar0 + 8u * 8, o_done = bar0 + 8u * 9, q_ready = bar0 + 8u * 10;
-    const uint32_t mma_drain = bar0 + 8u * 11;
+    auto k_full = [&](int s) { return bar0 + 8u * (BAR_K_FULL + s); };
+    auto k_empty = [&](int s) { return bar0 + 8u * (BAR_K_EMPTY + s); };
+    auto v_full = [&](int s) { return bar0 + 8u * (BAR_V_FULL + s); };
+    auto v_empty = [&](int s) { return bar0 + 8u * (BAR_V_EMPTY + s); };
+    auto s_full = [&](int s) { return bar0 + 8u * (BAR_S_FULL + s); };
+    auto p_full = [&](int x) { return bar0 + 8u * (BAR_P_FULL + x); };
+    auto o_done = [&](int x) { return bar0 + 8u * (BAR_O_DONE + x); };
+    const uint32_t q_ready = bar0 + 8u * BAR_Q_READY, mma_drain = bar0 + 8u * BAR_DRAIN;
     volatile int* abort_flag = &s_abort;
+    // results of the softmax groups, consumed by the split merge after the role blocks
+    float o[64];
+    float lse = -INFINITY;
+    const int X = warp >= 4 ? (warp - 4) >> 2 : 0;          // softmax group: tokens X*64 .. X*64+63 of a tile
+    const int r = ((warp & 3) << 5) + lane;                  // query row in the tile (softmax warps)
 
-    const int L = a.prefix_lens[b];
-    const int total = L + N;
-
-    // ---- prologue: tree check, barriers, TMEM
+    // ---- prologue
+    if ((warp == 0 || warp == 3) && lane == 0) prefetch_tensormap(warp == 0 ? &tmk : &tmv);
     if (tid == 0) {
         s_abort = 0;
-        s_bad = (L < 0 || (total + TV_BLOCK - 1) / TV_BLOCK > a.max_blocks) ? TV_ERR_BLOCK_TABLE : 0;
-    }
-    for (int i = tid; i < N; i += TC_THREADS) s_par[i] = a.parent[(size_t)b * N + i];
-    if (tid == 32) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(kv_full(s), 1);
-            mbar_init(kv_empty(s), 1);
-            mbar_init(s_full(s), 1);
-            mbar_init(s_free(s), 128);
+        s_bad = 0;
+        for (int s = 0; s < KST; ++s) {
+            mbar_init(k_full(s), 1);
+            mbar_init(k_empty(s), 1);
         }
-        mbar_init(p_full, 128);
-        mbar_init(o_done, 1);
-        mbar_init(q_ready, 128);
+        for (int s = 0; s < VST; ++s) {
+            mbar_init(v_full(s), 1);
+            mbar_init(v_empty(s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(s_full(s), 1);
+            mbar_init(p_full(s), 128);
+            mbar_init(o_done(s), 1);
+        }
+        mbar_init(q_ready, 256);
         mbar_init(mma_drain, 1);
         fence_barrier_init();
     }
@@ -255,126 +376,143 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
         tc_fence_before();
     }
-    __syncthreads();
-    for (int i = tid; i < N; i += TC_THREADS)
-        if (!parent_ok(s_par, i)) s_bad = TV_ERR_TREE;
-    tc_fence_after();
-    __syncthreads();
-    const uint32_t tmem = s_tmem;
-    const bool bad0 = s_bad != 0;
+    for (int i = tid; i < N; i += TC_THREADS) s_par[i] = a.parent[(size_t)b * N + i];
+    const int L = a.prefix_lens[b];
+    const int total = L + N;
+    const bool bad_len = L < 0 || (total + TV_BLOCK - 1) / TV_BLOCK > a.max_blocks;
     int t0, t1;
-    split_range(total, S, split, t0, t1);
-    if (bad0) t1 = t0;
+    split_range(bad_len ? 0 : total, S, split, t0, t1);
     const int ntiles = (t1 - t0 + TN - 1) / TN;
     const int last_blk = (t1 - 1) / TV_BLOCK;
+    // the producer's first block ids are fetched before the barrier so the
+    // loads overlap barrier set-up and TMEM allocation
+    const int32_t* bt = a.block_table + (size_t)b * a.max_blocks;
+    // producer lane l holds the block id of block l % 8 of tile j + l / 8: four tiles of lookahead
+    bool bad_id = false;
+    auto load_id = [&](int jt) {
+        if (jt >= ntiles) return 0;
+        int bi = (t0 + jt * TN) / TV_BLOCK + (lane & 7);
+        if (bi > last_blk) bi = last_blk;
+        int id = bt[bi];
+        if (id < 0 || id >= a.num_blocks) {
+            bad_id = true;
+            id = 0;
+        }
+        return id;
+    };
+    int ids = (warp == 0 || warp == 3) ? load_id(lane >> 3) : 0;
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
 
-    if (warp == 0) {
-        // ---------------- TMA producer
-        const int32_t* bt = a.block_table + (size_t)b * a.max_blocks;
-        auto fetch = [&](int j) {
-            int id = 0;
-            if (lane < BLK_PER_TILE) {
-                int bi = (t0 + j * TN) / TV_BLOCK + lane;
-                if (bi > last_blk) bi = last_blk;
-                id = bt[bi];
-                if (id < 0 || id >= a.num_blocks) {
-                    s_bad = TV_ERR_BLOCK_TABLE;
-                    id = 0;
-                }
-            }
-            return id;
-        };
-        int ids = ntiles > 0 ? fetch(0) : 0;
+    if (warp == 0 || warp == 3) {
+        // ---------------- TMA producers: warp 0 streams K tiles, warp 3 V tiles
+        const bool is_k = warp == 0;
+        const CUtensorMap* map = is_k ? &tmk : &tmv;
+        const int depth = is_k ? KST : VST;
         int issued = 0;
         for (int j = 0; j < ntiles; ++j) {
-            const int stage = j & 1;
-            if (j >= STAGES && !warp_wait(kv_empty(stage), ((j - STAGES) >> 1) & 1, abort_flag)) break;
+            const int s = j % depth;
+            if (j >= depth && !warp_wait(is_k ? k_empty(s) : v_empty(s), ((j - depth) / depth) & 1, abort_flag)) break;
             int cur[BLK_PER_TILE];
 #pragma unroll
             for (int k = 0; k < BLK_PER_TILE; ++k) cur[k] = __shfl_sync(0xffffffffu, ids, k);
             if (lane == 0) {
-                const uint32_t full = kv_full(stage);
-                mbar_expect_tx(full, TILE_TX_BYTES);
-                const uint32_t sK = sKV + stage * STAGE_BYTES, sV = sK + 32768u;
+                const uint32_t full = is_k ? k_full(s) : v_full(s);
+                const uint32_t dst = is_k ? sK(s) : sV(s);
+                mbar_expect_tx(full, TILE_BYTES);
 #pragma unroll
-                for (int k = 0; k < BLK_PER_TILE; ++k) {
+                for (int k = 0; k < BLK_PER_TILE; ++k)
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        tma_load_4d(sK + h * HALF_BYTES + k * 2048u, &tmk, full, 0, kvh * 2 + h, 0, cur[k]);
-                        tma_load_4d(sV + h * HALF_BYTES + k * 2048u, &tmv, full, 0, kvh * 2 + h, 0, cur[k]);
-                    }
-                }
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_4d(dst + h * HALF_BYTES + k * 2048u, map, full, 0, kvh * 2 + h, 0, cur[k]);
             }
             ++issued;
+            // let the first tile land before streaming the rest, so it does not queue
+            // behind every other tile of the launch
+            if (j == 0 && ntiles > 1 && !warp_wait(is_k ? k_full(0) : v_full(0), 0, abort_flag)) break;
+            // slide the lookahead window by one tile
+            const int nxt = __shfl_down_sync(0xffffffffu, ids, 8);
+            ids = lane < 24 ? nxt : load_id(j + 4);
             __syncwarp();
-            if (j + 1 < ntiles) ids = fetch(j + 1);
         }
-        if (*abort_flag) {
+        if (bad_id) s_bad = TV_ERR_BLOCK_TABLE;
+        if (*abort_flag && lane == 0) {
             // let copies already in flight land before the CTA retires
-            for (int j = max(0, issued - STAGES); j < issued; ++j) {
-                const long long t_0 = clock64();
-                while (!mbar_try(kv_full(j & 1), (j >> 1) & 1) && clock64() - t_0 < (WAIT_LIMIT >> 4)) {
+            for (int j = max(0, issued - depth); j < issued; ++j) {
+                const long long c0 = clock64();
+                const uint32_t full = is_k ? k_full(j % depth) : v_full(j % depth);
+                while (!mbar_try(full, (j / depth) & 1) && clock64() - c0 < (WAIT_LIMIT >> 4)) {
                 }
             }
         }
+        __syncwarp();
     } else if (warp == 1) {
         // ---------------- MMA issuer (one thread)
         if (ntiles > 0 && lane == 0) {
             bool ok = mbar_wait(q_ready, 0, abort_flag);
             bool issued_any = false;
-            for (int j = 0; ok && j <= ntiles; ++j) {
-                if (j < ntiles) {
-                    const int stage = j & 1, sb = j & 1;
-                    ok = mbar_wait(kv_full(stage), (j >> 1) & 1, abort_flag);
-                    if (ok && j >= 2) ok = mbar_wait(s_free(sb), ((j - 2) >> 1) & 1, abort_flag);
+            // S = Q K^T of tile j into S buffer j % 2
+            auto issue_qk = [&](int j) {
+                const int ks = j % KST, sb = j & 1;
+                if (!mbar_wait(k_full(ks), (j / KST) & 1, abort_flag)) return false;
+                // S buffer j % 2 held P of tile j - 2, whose P V was issued before this call
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < HD / 16; ++k) {
+                    const uint32_t off = (k >> 2) * HALF_BYTES + (k & 3) * 32u;
+                    mma_bf16(tmem + sb * TN, sdesc(sQ + off, 16, 1024), sdesc(sK(ks) + off, 16, 1024), IDESC_QK,
+                             k > 0 ? 1u : 0u);
+                }
+                mma_commit(s_full(sb));
+                mma_commit(k_empty(ks));
+                issued_any = true;
+                return true;
+            };
+            // the S tiles run two ahead of P V, so the softmax groups never wait for S
+            for (int j = 0; ok && j < 2 && j < ntiles; ++j) ok = issue_qk(j);
+            for (int t = 0; ok && t < ntiles; ++t) {
+                const int vs = t % VST;
+                ok = mbar_wait(v_full(vs), (t / VST) & 1, abort_flag);
+                for (int x = 0; ok && x < 2; ++x) {
+                    ok = mbar_wait(p_full(x), t & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t sK = sKV + stage * STAGE_BYTES;
 #pragma unroll
-                    for (int k = 0; k < HD / 16; ++k) {
-                        const uint32_t off = (k >> 2) * HALF_BYTES + (k & 3) * 32u;
-                        mma_bf16(tmem + sb * TN, sdesc(sQ + off, 16, 1024), sdesc(sK + off, 16, 1024), IDESC_QK,
-                                 k > 0 ? 1u : 0u);
-                    }
-                    mma_commit(s_full(sb));
-                    issued_any = true;
+                    for (int k = 0; k < HALF_N / 16; ++k)
+                        mma_bf16_ts(tmem + O_COL + x * HD, tmem + (t & 1) * TN + x * HALF_N + k * 8,
+                                    sdesc(sV(vs) + (x * 4 + k) * 2048u, HALF_BYTES, 1024), IDESC_PV,
+                                    (t > 0 || k > 0) ? 1u : 0u);
+                    mma_commit(o_done(x));
                 }
-                if (j >= 1) {
-                    const int t = j - 1, stage = t & 1;
-                    ok = mbar_wait(p_full, t & 1, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t sV = sKV + stage * STAGE_BYTES + 32768u;
-#pragma unroll
-                    for (int k = 0; k < TN / 16; ++k) {
-                        const uint32_t off = (k >> 2) * HALF_BYTES + (k & 3) * 32u;
-                        mma_bf16(tmem + O_COL, sdesc(sP + off, 16, 1024), sdesc(sV + k * 2048u, HALF_BYTES, 1024),
-                                 IDESC_PV, (t > 0 || k > 0) ? 1u : 0u);
-                    }
-                    mma_commit(o_done);
-                    mma_commit(kv_empty(stage));
-                }
+                if (!ok) break;
+                mma_commit(v_empty(vs));
+                if (t + 2 < ntiles) ok = issue_qk(t + 2);
             }
             if (issued_any) {
                 // every MMA issued by this thread has finished before TMEM is released
                 mma_commit(mma_drain);
-                const long long t_0 = clock64();
-                while (!mbar_try(mma_drain, 0) && clock64() - t_0 < WAIT_LIMIT) {
+                const long long c0 = clock64();
+                while (!mbar_try(mma_drain, 0) && clock64() - c0 < WAIT_LIMIT) {
                 }
             }
         }
         __syncwarp();
     } else if (warp >= 4) {
-        // ---------------- softmax: one thread per query row / TMEM lane
-        const int r = tid - 128;
+        // ---------------- softmax groups: one thread per query row / TMEM lane
+        const int st = tid - 128;  // 0..255
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        for (int i = st; i < N; i += 256)
+            if (!parent_ok(s_par, i)) s_bad = TV_ERR_TREE;
+        if (st == 0 && bad_len) s_bad = TV_ERR_BLOCK_TABLE;
         const int gr = tile * TM + r;
         const bool row_ok = gr < G * N;
         const int node = row_ok ? gr / G : 0;
         const int head = kvh * G + (row_ok ? gr % G : 0);
         uint32_t an0 = 0, an1 = 0, an2 = 0, an3 = 0;
-        if (!bad0 && row_ok)
-            for (int jn = node; jn >= 0; jn = s_par[jn]) {
+        if (row_ok) {
+            int steps = 0;
+            for (int jn = node; jn >= 0 && jn < N && steps <= N; jn = s_par[jn], ++steps) {
                 const uint32_t bit = 1u << (jn & 31);
                 const int w = jn >> 5;
                 an0 |= w == 0 ? bit : 0u;
@@ -382,217 +520,220 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 an2 |= w == 2 ? bit : 0u;
                 an3 |= w == 3 ? bit : 0u;
             }
+        }
         {
             const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
-                                                              (((size_t)b * N + node) * a.Hq + head) * HD);
+                                                              (((size_t)b * N + node) * a.Hq + head) * HD + X * 64);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
+            for (int c = 0; c < 8; ++c) {
                 const uint4 v = row_ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-                st_shared_v4(sQ + (c >> 3) * HALF_BYTES + r * 128 + (((c & 7) ^ (r & 7)) << 4), v);
+                st_shared_v4(sQ + X * HALF_BYTES + r * 128 + ((c ^ (r & 7)) << 4), v);
             }
             fence_proxy_async();
             mbar_arrive(q_ready);
         }
-        float m_run = -INFINITY, l_run = 0.f;
+        float m_run = -INFINITY, l_run = 0.f;  // running max in the scaled log2 domain, running sum
         const float sl = a.scale_log2;
         for (int j = 0; j < ntiles; ++j) {
-            const int sb = j & 1, stage = j & 1;
+            const int sb = j & 1;
             if (!warp_wait(s_full(sb), (j >> 1) & 1, abort_flag)) break;
             tc_fence_after();
-            float x[TN];
+            float x[HALF_N];
 #pragma unroll
-            for (int c4 = 0; c4 < TN / 32; ++c4) {
+            for (int c32 = 0; c32 < HALF_N / 32; ++c32) {
                 uint32_t rr[32];
-                tmem_ld_x32(tmem + lane_base + sb * TN + c4 * 32, rr);
+                tmem_ld_x32(tmem + lane_base + sb * TN + X * HALF_N + c32 * 32, rr);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) x[c4 * 32 + i] = __uint_as_float(rr[i]);
+                for (int i = 0; i < 32; ++i) x[c32 * 32 + i] = __uint_as_float(rr[i]);
             }
-            tc_fence_before();
-            mbar_arrive(s_free(sb));
             const int tstart = t0 + j * TN;
-            const int lim = t1 - tstart;  // columns >= lim lie past the split
-            const int tree0 = L - tstart; // columns >= tree0 are tree nodes (node = column - tree0)
-            float mt = -INFINITY;
-            if (lim >= TN && tree0 >= TN) {
+            const int lim = t1 - tstart;   // tile columns >= lim lie past the split
+            const int tree0 = L - tstart;  // tile columns >= tree0 are tree nodes
+            if (lim < TN || tree0 < TN) {
+                uint32_t cm[2];
 #pragma unroll
-                for (int c = 0; c < TN; ++c) {
-                    x[c] *= sl;
-                    mt = fmaxf(mt, x[c]);
-                }
-            } else {
-                uint32_t cm[4];
+                for (int w = 0; w < 2; ++w)
+                    cm[w] = (below(tree0, 2 * X + w) | shifted_word(an0, an1, an2, an3, tree0, 2 * X + w)) &
+                            below(lim, 2 * X + w);
 #pragma unroll
-                for (int w = 0; w < 4; ++w)
-                    cm[w] = (below(tree0, w) | shifted_word(an0, an1, an2, an3, tree0, w)) & below(lim, w);
-#pragma unroll
-                for (int c = 0; c < TN; ++c) {
-                    const bool ok = (cm[c >> 5] >> (c & 31)) & 1u;
-                    x[c] = ok ? x[c] * sl : -INFINITY;
-                    mt = fmaxf(mt, x[c]);
-                }
+                for (int i = 0; i < HALF_N; ++i)
+                    if (!((cm[i >> 5] >> (i & 31)) & 1u)) x[i] = -INFINITY;
             }
-            // the previous P V must be done: it frees P and settles O
-            if (j > 0 && !warp_wait(o_done, (j - 1) & 1, abort_flag)) break;
-            if (mt > m_run + 8.f) {
-                if (m_run != -INFINITY) {
-                    const float f = ex2(m_run - mt);
-                    l_run *= f;
-                    if (j > 0) {
-                        tc_fence_after();
-#pragma unroll
-                        for (int c4 = 0; c4 < HD / 32; ++c4) {
-                            uint32_t rr[32];
-                            tmem_ld_x32(tmem + lane_base + O_COL + c4 * 32, rr);
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * f);
-                            tmem_st_x32(tmem + lane_base + O_COL + c4 * 32, rr);
-                        }
-                        tmem_wait_st();
-                    }
-                }
+            const float mt = max_tree(x) * sl;
+            float f = 1.f;
+            if (mt > m_run + 8.f) {  // grow the reference max (also the first finite tile)
+                if (m_run != -INFINITY) f = ex2(m_run - mt);
                 m_run = mt;
             }
             const float mu = m_run == -INFINITY ? 0.f : m_run;
-            float ls = 0.f;
+            float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int cc = 0; cc < TN / 8; ++cc) {
-                float p[8];
+            for (int i = 0; i < HALF_N; ++i) {
+                x[i] = ex2(fmaf(x[i], sl, -mu));
+                s4[i & 3] += x[i];
+            }
+            l_run = l_run * f + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+            // P as bf16 pairs (token 2i in the low half of column i) over the first 32 of
+            // this group's S columns of the tile, whose scores were read above
+            {
+                uint32_t pk[32];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    p[e] = ex2(x[cc * 8 + e] - mu);
-                    ls += p[e];
+                for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(x[2 * i], x[2 * i + 1]);
+                tmem_st_x32(tmem + lane_base + sb * TN + X * HALF_N, pk);
+            }
+            if (lim < TN) {
+                // value rows past the split end may hold stale data: clear this group's ones
+                const int tok = X * HALF_N + (r & 63);
+                if (tok >= lim) {
+                    const int vs = j % VST;
+                    mbar_wait(v_full(vs), (j / VST) & 1, abort_flag);
+                    const uint32_t row = sV(vs) + (r >> 6) * HALF_BYTES + tok * 128;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) st_shared_v4(row + c * 16, make_uint4(0, 0, 0, 0));
                 }
-                uint4 v;
-                v.x = pack_bf16(p[0], p[1]);
-                v.y = pack_bf16(p[2], p[3]);
-                v.z = pack_bf16(p[4], p[5]);
-                v.w = pack_bf16(p[6], p[7]);
-                st_shared_v4(sP + (cc >> 3) * HALF_BYTES + r * 128 + (((cc & 7) ^ (r & 7)) << 4), v);
+                fence_proxy_async();
             }
-            l_run += ls;
-            if (lim < TN && r >= lim) {
-                // value rows past the split end may hold stale data: clear them before P V
-                mbar_wait(kv_full(stage), (j >> 1) & 1, abort_flag);
-                const uint32_t sV = sKV + stage * STAGE_BYTES + 32768u;
+            // this group's previous P V must be complete before O is rescaled and
+            // before P V of this tile is released (every phase is waited, in order)
+            if (j > 0 && !warp_wait(o_done(X), (j - 1) & 1, abort_flag)) break;
+            if (f != 1.f && j > 0) {
+                tc_fence_after();
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
+                for (int c4 = 0; c4 < HD / 32; ++c4) {
+                    uint32_t rr[32];
+                    tmem_ld_x32(tmem + lane_base + O_COL + X * HD + c4 * 32, rr);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) st_shared_v4(sV + h * HALF_BYTES + r * 128 + c * 16, make_uint4(0, 0, 0, 0));
+                    for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * f);
+                    tmem_st_x32(tmem + lane_base + O_COL + X * HD + c4 * 32, rr);
+                }
             }
-            fence_proxy_async();
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(p_full);
+            mbar_arrive(p_full(X));
         }
-        // ---- epilogue: normalise this CTA's partial output
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        bool fail = *abort_flag != 0;
-        if (ntiles > 0 && !fail) fail = !warp_wait(o_done, (ntiles - 1) & 1, abort_flag);
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        // one decision per warp: tcgen05.ld below is warp-collective
+        // ---- epilogue: merge the two groups' halves into this CTA's partial output
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        bool fail = __any_sync(0xffffffffu, *abort_flag != 0);
+        if (ntiles > 0 && !fail) fail = !warp_wait(o_done(X), (ntiles - 1) & 1, abort_flag);
+        // per-row (max, sum) of each group, exchanged through that group's half of the Q
+        // buffer: every S = Q K^T finished before this group's last P V
+        float* pm = reinterpret_cast<float*>(base_ptr + SQ_OFF);
+        auto s_m = [&](int g) { return pm + g * (HALF_BYTES / 4); };
+        auto s_l = [&](int g) { return pm + g * (HALF_BYTES / 4) + TM; };
+        s_m(X)[r] = m_run;
+        s_l(X)[r] = l_run;
+        asm volatile("bar.sync 1, 256;" ::: "memory");
         const bool bad = __any_sync(0xffffffffu, *abort_flag != 0 || s_bad != 0);
-        tc_fence_after();
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        const float lse = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
+        const float mA = s_m(0)[r], mB = s_m(1)[r];
+        const float m = fmaxf(mA, mB);
+        const float wA = mA == -INFINITY ? 0.f : ex2(mA - m);
+        const float wB = mB == -INFINITY ? 0.f : ex2(mB - m);
+        const float l = wA * s_l(0)[r] + wB * s_l(1)[r];
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        lse = bad ? NAN : (l > 0.f ? m + log2f(l) : -INFINITY);
         const bool have_o = ntiles > 0 && !bad;
-        if (S == 1) {
-            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + (((size_t)b * N + node) * a.Hq + head) * HD;
+        tc_fence_after();
 #pragma unroll
-            for (int c4 = 0; c4 < HD / 32; ++c4) {
-                uint32_t rr[32];
-                if (have_o) {
-                    tmem_ld_x32(tmem + lane_base + O_COL + c4 * 32, rr);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) rr[i] = 0u;
-                }
-                if (row_ok) {
-#pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8) {
-                        float o[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) o[e] = bad ? NAN : __uint_as_float(rr[q8 * 8 + e]) * inv;
-                        uint4 v;
-                        v.x = pack_bf16(o[0], o[1]);
-                        v.y = pack_bf16(o[2], o[3]);
-                        v.z = pack_bf16(o[4], o[5]);
-                        v.w = pack_bf16(o[6], o[7]);
-                        reinterpret_cast<uint4*>(dst + c4 * 32)[q8] = v;
-                    }
-                }
+        for (int c32 = 0; c32 < 2; ++c32) {
+            uint32_t ra[32], rb[32];
+            if (have_o) {
+                tmem_ld_x32(tmem + lane_base + O_COL + X * 64 + c32 * 32, ra);
+                tmem_ld_x32(tmem + lane_base + O_COL + HD + X * 64 + c32 * 32, rb);
             }
-        } else {
-            float* stage_o = reinterpret_cast<float*>(base_ptr + SKV_OFF);
 #pragma unroll
-            for (int c4 = 0; c4 < HD / 32; ++c4) {
-                uint32_t rr[32];
-                if (have_o) {
-                    tmem_ld_x32(tmem + lane_base + O_COL + c4 * 32, rr);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) rr[i] = 0u;
-                }
-#pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4) {
-                    float4 v;
-                    v.x = __uint_as_float(rr[q4 * 4 + 0]) * inv;
-                    v.y = __uint_as_float(rr[q4 * 4 + 1]) * inv;
-                    v.z = __uint_as_float(rr[q4 * 4 + 2]) * inv;
-                    v.w = __uint_as_float(rr[q4 * 4 + 3]) * inv;
-                    *reinterpret_cast<float4*>(stage_o + r * OPITCH + c4 * 32 + q4 * 4) = v;
-                }
-            }
-            s_lse[r] = bad ? NAN : lse;
+            for (int i = 0; i < 32; ++i)
+                o[c32 * 32 + i] = have_o ? (wA * __uint_as_float(ra[i]) + wB * __uint_as_float(rb[i])) * inv
+                                         : (bad ? NAN : 0.f);
         }
         tc_fence_before();
+        if (S == 1 && row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
+                                                  (((size_t)b * N + node) * a.Hq + head) * HD + X * 64);
+#pragma unroll
+            for (int q8 = 0; q8 < 8; ++q8) {
+                uint4 v;
+                v.x = pack_bf16(o[q8 * 8 + 0], o[q8 * 8 + 1]);
+                v.y = pack_bf16(o[q8 * 8 + 2], o[q8 * 8 + 3]);
+                v.z = pack_bf16(o[q8 * 8 + 4], o[q8 * 8 + 5]);
+                v.w = pack_bf16(o[q8 * 8 + 6], o[q8 * 8 + 7]);
+                dst[q8] = v;
+            }
+        }
     }
 
-    __syncthreads();
+    __syncthreads();  // every role finished; all TMEM reads completed
     if (warp == 2) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
     }
     if (S > 1) {
-        // ---- merge the splits of this row tile through distributed shared memory
-        cg::cluster_group cluster = cg::this_cluster();
-        cluster.sync();
-        const float* stage_o = reinterpret_cast<const float*>(base_ptr + SKV_OFF);
-        const int R = (TM + S - 1) / S;
-        const int r0 = split * R;
-        for (int item = tid; item < R * (HD / 4); item += TC_THREADS) {
-            const int r = r0 + item / (HD / 4), c4 = item % (HD / 4);
-            const int gr = tile * TM + r;
-            if (r >= TM || gr >= G * N) continue;
-            float mx = -INFINITY;
-            bool nan = false;
-            for (int s = 0; s < S; ++s) {
-                const float l = *cluster.map_shared_rank(&s_lse[r], s);
-                nan |= isnan(l);
-                mx = fmaxf(mx, l);
-            }
-            float den = 0.f;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int s = 0; s < S; ++s) {
-                const float l = *cluster.map_shared_rank(&s_lse[r], s);
-                if (l == -INFINITY || nan) continue;
-                const float w = ex2(l - mx);
-                const float4 v = *reinterpret_cast<const float4*>(
-                    cluster.map_shared_rank(stage_o + r * OPITCH + c4 * 4, s));
-                den += w;
-                acc.x = fmaf(w, v.x, acc.x);
-                acc.y = fmaf(w, v.y, acc.y);
-                acc.z = fmaf(w, v.z, acc.z);
-                acc.w = fmaf(w, v.w, acc.w);
-            }
-            const bool dead = nan || den == 0.f;
-            const float id = dead ? 0.f : 1.f / den;
-            const int node = gr / G, head = kvh * G + gr % G;
-            uint2 o;
-            o.x = pack_bf16(dead ? NAN : acc.x * id, dead ? NAN : acc.y * id);
-            o.y = pack_bf16(dead ? NAN : acc.z * id, dead ? NAN : acc.w * id);
-            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + (((size_t)b * N + node) * a.Hq + head) * HD +
-                                      c4 * 4) = o;
+        // ---- merge the KV splits of this row tile.  Each split stages its normalised
+        // partial rows and their log-sum-exp in shared memory, copies them to the
+        // workspace with coalesced stores, counts itself in, and once all S splits
+        // are in combines an equal share of the rows from all S partials.
+        const size_t group = ((size_t)b * a.Hkv + kvh) * a.row_tiles + tile;
+        float* part = a.o_part + group * (size_t)S * TM * RPITCH;  // [S][TM][RPITCH]
+        unsigned* arrive = a.counters + 2 * group;                  // [groups][2]: arrivals, departures
+        float* stage = reinterpret_cast<float*>(base_ptr + SK_OFF); // [TM][RPITCH]; the K ring is idle now
+        if (warp >= 4) {
+            float4* row = reinterpret_cast<float4*>(stage + r * RPITCH + X * 64);
+#pragma unroll
+            for (int q4 = 0; q4 < 16; ++q4) row[q4] = make_float4(o[q4 * 4], o[q4 * 4 + 1], o[q4 * 4 + 2], o[q4 * 4 + 3]);
+            if (X == 0) stage[r * RPITCH + HD] = lse;
         }
-        cluster.sync();  // peers may still read this CTA's shared memory until here
+        __syncthreads();
+        {
+            const float4* src = reinterpret_cast<const float4*>(stage);
+            float4* dst = reinterpret_cast<float4*>(part + (size_t)split * TM * RPITCH);
+            for (int i = tid; i < TM * RPITCH / 4; i += TC_THREADS) dst[i] = src[i];
+        }
+        __syncthreads();
+        __shared__ int s_all_in;
+        if (tid == 0) {
+            count_in(arrive);
+            s_all_in = wait_count(arrive, (unsigned)S, abort_flag) ? 1 : 0;
+        }
+        __syncthreads();
+        if (!s_all_in) {
+            // a peer never arrived: leave this CTA's share of the rows as NaN
+            const int R = (TM + S - 1) / S;
+            const int own = max(0, min(TM, (split + 1) * R) - split * R);
+            for (int item = tid; item < own * (HD / 4); item += TC_THREADS) {
+                const int rt = split * R + item / (HD / 4), gr = tile * TM + rt;
+                if (gr >= G * N) continue;
+                const int node = gr / G, head = kvh * G + gr % G;
+                uint2 ov;
+                ov.x = pack_bf16(NAN, NAN);
+                ov.y = ov.x;
+                *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) +
+                                          (((size_t)b * N + node) * a.Hq + head) * HD + (item % (HD / 4)) * 4) = ov;
+            }
+        } else
+        switch (S) {
+            case 2: merge_rows<2>(a, part, split, tile, b, kvh, tid); break;
+            case 3: merge_rows<3>(a, part, split, tile, b, kvh, tid); break;
+            case 4: merge_rows<4>(a, part, split, tile, b, kvh, tid); break;
+            case 5: merge_rows<5>(a, part, split, tile, b, kvh, tid); break;
+            case 6: merge_rows<6>(a, part, split, tile, b, kvh, tid); break;
+            case 7: merge_rows<7>(a, part, split, tile, b, kvh, tid); break;
+            case 8: merge_rows<8>(a, part, split, tile, b, kvh, tid); break;
+            case 9: merge_rows<9>(a, part, split, tile, b, kvh, tid); break;
+            case 10: merge_rows<10>(a, part, split, tile, b, kvh, tid); break;
+            case 11: merge_rows<11>(a, part, split, tile, b, kvh, tid); break;
+            case 12: merge_rows<12>(a, part, split, tile, b, kvh, tid); break;
+            case 13: merge_rows<13>(a, part, split, tile, b, kvh, tid); break;
+            case 14: merge_rows<14>(a, part, split, tile, b, kvh, tid); break;
+            case 15: merge_rows<15>(a, part, split, tile, b, kvh, tid); break;
+            default: merge_rows<16>(a, part, split, tile, b, kvh, tid); break;
+        }
+        __syncthreads();
+        if (tid == 0 && atomicAdd(arrive + 1, 1u) == (unsigned)(S - 1)) {
+            // the last split out: every peer has passed its wait, so both counters
+            // can return to zero for the next call
+            arrive[0] = 0u;
+            arrive[1] = 0u;
+            __threadfence();
+        }
     }
     if (tid == 0) {
         if (s_bad) report(a.status, s_bad);
@@ -632,31 +773,76 @@ bool make_kv_map(EncodeTiledFn fn, CUtensorMap* m, const void* ptr, int Hkv, int
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool tc_attrs_ready() {
+    static int state = -1;
+    if (state < 0) {
+        state = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) ==
+                cudaSuccess;
+        cudaGetLastError();
+    }
+    return state == 1;
+}
+
+// CTAs of this kernel the device holds at once (-1 if it cannot be queried)
+int tc_resident_ctas() {
+    static int cached = 0;
+    if (cached == 0) {
+        int n = -1, per_sm = 0, dev = 0, sms = 0;
+        if (tc_attrs_ready() && cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_tc_kernel, TC_THREADS, SMEM_BYTES) ==
+                cudaSuccess)
+            n = per_sm * sms;
+        cudaGetLastError();
+        cached = n;
+    }
+    return cached;
+}
+
 }  // namespace
 
 int tc_rows_per_tile() { return TM; }
-int tc_max_cluster() { return MAX_CLUSTER; }
+int tc_max_splits() { return MAX_SPLITS; }
+size_t tc_counter_offset(int64_t groups, int splits) {
+    return (size_t)groups * splits * TM * RPITCH * sizeof(float);
+}
+size_t tc_workspace_bytes(int64_t groups, int splits) {
+    if (splits <= 1) return 0;
+    return tc_counter_offset(groups, splits) + (((size_t)groups * 2 * sizeof(unsigned) + 255) & ~(size_t)255);
+}
+
+// KV splits per row tile: as many as keep the whole grid resident at once
+// (one wave, which the cooperative merge requires), at most 16, and at least
+// 256 tokens per split.
+int tc_pick_splits(int64_t groups, int64_t max_tokens, int sms) {
+    int cap = tc_resident_ctas();
+    if (cap <= 0) cap = sms;
+    if (groups * 2 > cap) return 1;
+    int64_t s = cap / groups;
+    if (s > MAX_SPLITS) s = MAX_SPLITS;
+    const int64_t by_len = max_tokens / 256;
+    if (s > by_len) s = by_len;
+    return s < 1 ? 1 : (int)s;
+}
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st, int* launches) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
-    if (a.D != HD || a.splits < 1 || a.splits > MAX_CLUSTER) return cudaErrorInvalidValue;
+    if (a.D != HD || a.splits < 1 || a.splits > MAX_SPLITS) return cudaErrorInvalidValue;
     CUtensorMap mk, mv;
     if (!make_kv_map(fn, &mk, a.k, a.Hkv, a.num_blocks) || !make_kv_map(fn, &mv, a.v, a.Hkv, a.num_blocks))
         return cudaErrorInvalidValue;
-    static cudaError_t attr =
-        cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    if (attr != cudaSuccess) return attr;
+    if (!tc_attrs_ready()) return cudaErrorInvalidDeviceFunction;
+    if (a.splits > 1 && (!a.o_part || !a.counters)) return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attrs[1];
     cfg.gridDim = dim3(a.splits, a.row_tiles, a.B * a.Hkv);
     cfg.blockDim = dim3(TC_THREADS, 1, 1);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = st;
-    attrs[0].id = cudaLaunchAttributeClusterDimension;
-    attrs[0].val.clusterDim.x = a.splits;
-    attrs[0].val.clusterDim.y = 1;
-    attrs[0].val.clusterDim.z = 1;
+    // the split merge waits on peers of the same launch: every CTA must be resident
+    attrs[0].id = cudaLaunchAttributeCooperative;
+    attrs[0].val.cooperative = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = a.splits > 1 ? 1 : 0;
     *launches = 1;

@@ -14,8 +14,10 @@ struct AttnArgs {
     const int32_t* prefix_lens;
     const int32_t* parent;
     void* out;
-    float* o_part;      // [splits][B][N][Hq][D] fp32 partial outputs (normalised)
+    float* o_part;      // CUDA-core path: [splits][B][N][Hq][D] fp32 partial outputs (normalised);
+                        // tensor-core path: [groups][splits][128][132] partial rows + lse
     float* lse_part;    // [splits][B][N][Hq] log2-domain log-sum-exp of each partial
+    unsigned* counters; // tensor-core path: [groups][2] arrival / departure counts, zero between calls
     int32_t* status;
     int B, N, Hq, Hkv, G, D, max_blocks, num_blocks, splits, row_tiles;
     float scale_log2;   // softmax_scale * log2(e)
@@ -28,7 +30,10 @@ int simt_rows_per_tile();
 // Tensor-core (tcgen05 / TMEM / TMA) bf16 kernel, head_dim 128.
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st, int* launches);
 int tc_rows_per_tile();
-int tc_max_cluster();
+int tc_max_splits();
+int tc_pick_splits(int64_t groups, int64_t max_tokens, int sms);
+size_t tc_workspace_bytes(int64_t groups, int splits);
+size_t tc_counter_offset(int64_t groups, int splits);
 
 struct SampleArgs {
     const float* p;
