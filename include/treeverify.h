@@ -123,6 +123,35 @@ TV_API tv_status tv_tree_attention(const tv_attn_desc *desc, const void *q, cons
                             void *stream);
 
 /*
+ * Tree attention without a caller-provided workspace.  (The pages describe
+ * no such call; it exists for callers of this library.)
+ *
+ * Same inputs, outputs, layouts and results as tv_tree_attention, for callers
+ * that cannot allocate device memory when they call: a process that hands all
+ * device memory to a fixed pool at start-up, a serving-runtime plugin whose
+ * hot path must not call the CUDA allocator (cudaMalloc may synchronise the
+ * device), or work recorded into a CUDA graph.  The scratch memory comes from
+ * a fixed device array of TV_STATIC_SCRATCH_BYTES inside the library, which
+ * every GPU that loads the library holds until the process exits; nothing is
+ * allocated or freed by this call.
+ *  - Returns TV_ERR_WORKSPACE, before launching anything, when the problem
+ *    needs more scratch than TV_STATIC_SCRATCH_BYTES (see
+ *    tv_tree_attention_workspace_size).
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - All calls share the one array per device, and it keeps the previous
+ *    call's contents (the call clears the parts that must start at zero):
+ *    calls that can overlap on the GPU, from any stream or thread, race on it
+ *    and must be serialised by the caller.
+ */
+#define TV_STATIC_SCRATCH_BYTES (12u << 20)
+
+TV_API tv_status tv_tree_attention_static(const tv_attn_desc *desc, const void *q, const void *paged_k,
+                                          const void *paged_v, const int32_t *block_table,
+                                          const int32_t *prefix_lens, const int32_t *parent_idx,
+                                          void *out, int32_t *dev_status, void *stream);
+
+/*
  * Acceptance walk problem.
  *   p, q         [batch][num_nodes][vocab] float32 probabilities:
  *                p[b][u] = target distribution after node u's path,

@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libtreeverify.so")
 TV_OK, TV_ERR_INVALID_ARG, TV_ERR_UNSUPPORTED, TV_ERR_TREE = 0, 1, 2, 3
 TV_ERR_BLOCK_TABLE, TV_ERR_WORKSPACE, TV_ERR_CUDA, TV_ERR_TIMEOUT = 4, 5, 6, 7
 TV_BF16, TV_F32 = 0, 1
+TV_STATIC_SCRATCH_BYTES = 12 << 20
 
 
 class TvAttnDesc(ctypes.Structure):
@@ -67,6 +68,7 @@ def lib() -> ctypes.CDLL:
         L.tv_tree_attention_workspace_size.argtypes = [ctypes.POINTER(TvAttnDesc)]
         L.tv_tree_attention_workspace_size.restype = sz
         L.tv_tree_attention.argtypes = [ctypes.POINTER(TvAttnDesc), P, P, P, P, P, P, P, P, sz, P, P]
+        L.tv_tree_attention_static.argtypes = [ctypes.POINTER(TvAttnDesc), P, P, P, P, P, P, P, P, P]
         L.tv_verify_sample_plan.argtypes = [ctypes.POINTER(TvSampleDesc), ctypes.POINTER(TvSamplePlan)]
         L.tv_verify_sample_workspace_size.argtypes = [ctypes.POINTER(TvSampleDesc)]
         L.tv_verify_sample_workspace_size.restype = sz
@@ -74,7 +76,8 @@ def lib() -> ctypes.CDLL:
         L.tv_status_string.argtypes = [ctypes.c_int32]
         L.tv_status_string.restype = ctypes.c_char_p
         L.tv_version.restype = ctypes.c_int32
-        for name in ("tv_tree_attention_plan", "tv_tree_attention", "tv_verify_sample_plan", "tv_verify_sample"):
+        for name in ("tv_tree_attention_plan", "tv_tree_attention", "tv_tree_attention_static",
+                     "tv_verify_sample_plan", "tv_verify_sample"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -124,6 +127,17 @@ def tv_tree_attention(desc, q, paged_k, paged_v, block_table, prefix_lens, paren
     return int(lib().tv_tree_attention(ctypes.byref(desc), _ptr(q), _ptr(paged_k), _ptr(paged_v), _ptr(block_table),
                                        _ptr(prefix_lens), _ptr(parent_idx), _ptr(out), _ptr(workspace),
                                        int(workspace_bytes), _ptr(dev_status), _stream(stream)))
+
+
+def tv_tree_attention_static(desc, q, paged_k, paged_v, block_table, prefix_lens, parent_idx, out,
+                             dev_status=None, stream=None) -> int:
+    """tv_tree_attention with the library's fixed scratch array instead of a
+    caller workspace, for callers that cannot allocate device memory when they
+    call.  The first call on a device must come before any stream capture;
+    overlapping calls race on the shared array."""
+    return int(lib().tv_tree_attention_static(ctypes.byref(desc), _ptr(q), _ptr(paged_k), _ptr(paged_v),
+                                              _ptr(block_table), _ptr(prefix_lens), _ptr(parent_idx), _ptr(out),
+                                              _ptr(dev_status), _stream(stream)))
 
 
 def tv_verify_sample_plan(desc: TvSampleDesc) -> TvSamplePlan:
