@@ -149,6 +149,23 @@ def sampler_bytes(wl, h) -> int:
     return rows * 8 * wl.vocab + tested * 12 + h["parent_idx"].size * 8
 
 
+# ------------------------------------------------------------------ multi-rank plumbing
+
+def reduce_max(values, world: int, device="cpu"):
+    """Element-wise maximum over ranks (timing is the slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_throughput(world: int, nodes_per_step: int, steps: int, max_ms: float) -> float:
+    """Whole-job nodes/s: every rank verifies its own sequences (weak scaling)."""
+    return world * nodes_per_step * steps / (max_ms / 1e3)
+
+
 # ------------------------------------------------------------------ our arm
 
 def run_ours(args, rank, world, local_rank):
@@ -277,17 +294,14 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = a0.elapsed_time(a1)
 
-    times = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = float(times[0]), float(times[1])
+    total_ms, e2e_ms = reduce_max([total_ms, e2e_ms], world, "cuda")
     if rank != 0:
         return None
 
     nodes = B * N
     ms_step = total_ms / K
-    value = world * nodes * K / (total_ms / 1e3)
-    e2e_value = world * nodes * K2 / (e2e_ms / 1e3)
+    value = job_throughput(world, nodes, K, total_ms)
+    e2e_value = job_throughput(world, nodes, K2, e2e_ms)
     peak, peak_kind, _ = load_peaks()
     a_bytes = attention_bytes(wl)
     s_bytes = sampler_bytes(wl, h)
