@@ -179,7 +179,7 @@ TV_API tv_status tv_tree_attention_static(const tv_attn_desc *desc, const void *
 typedef struct {
     int32_t batch;
     int32_t num_nodes;           /* 1..1024 */
-    int32_t vocab;               /* 1..(16 * 24576) */
+    int32_t vocab;               /* 1..221184 (16 CTAs x 13824 entries) */
 } tv_sample_desc;
 
 typedef struct {

@@ -88,7 +88,7 @@ def test_attention_plans():
     (dict(batch=0, num_nodes=4, vocab=10), tv.TV_ERR_INVALID_ARG),
     (dict(batch=1, num_nodes=0, vocab=10), tv.TV_ERR_INVALID_ARG),
     (dict(batch=1, num_nodes=1025, vocab=10), tv.TV_ERR_UNSUPPORTED),
-    (dict(batch=1, num_nodes=4, vocab=16 * 24576 + 1), tv.TV_ERR_UNSUPPORTED),
+    (dict(batch=1, num_nodes=4, vocab=16 * 13824 + 1), tv.TV_ERR_UNSUPPORTED),
 ])
 def test_sampler_rejects_bad_descriptors(kw, status):
     d = tv.TvSampleDesc(**kw)
@@ -101,5 +101,5 @@ def test_sampler_plan_covers_vocab():
         p = tv.tv_verify_sample_plan(tv.TvSampleDesc(1, 64, V))
         assert p.cluster_ctas * p.slice >= V and p.slice % 4 == 0
         assert 32 <= p.threads <= 512 and p.threads % 32 == 0
-        assert p.smem_bytes == 8 * p.slice
+        assert p.smem_bytes == 16 * p.slice
     assert tv.tv_verify_sample_workspace_size(tv.TvSampleDesc(1, 64, 1000)) == 0

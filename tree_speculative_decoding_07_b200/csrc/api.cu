@@ -78,13 +78,14 @@ tv_status check_sample_desc(const tv_sample_desc* d) {
     if (!d) return TV_ERR_INVALID_ARG;
     if (d->batch < 1 || d->num_nodes < 1 || d->vocab < 1) return TV_ERR_INVALID_ARG;
     if (d->num_nodes > 1024) return TV_ERR_UNSUPPORTED;
-    if (d->vocab > 16 * 24576) return TV_ERR_UNSUPPORTED;
+    if (d->vocab > 16 * 13824) return TV_ERR_UNSUPPORTED;
     if ((int64_t)d->batch * 16 > INT32_MAX) return TV_ERR_UNSUPPORTED;
     return TV_OK;
 }
 
 // One cluster per sequence; each CTA caches a slice of about 8K entries of
-// a row's p and q (64 KB) so a 128K-entry row spreads over 16 SMs.
+// two rows' p and q (two buffers: the current node's row and the next one's
+// prefetch, 16 bytes per entry) so a 128K-entry row spreads over 16 SMs.
 void make_sample_plan(const tv_sample_desc* d, tv_sample_plan* p) {
     const int max_c = tv::sample_max_cluster();
     int c = (d->vocab + 8191) / 8192;
@@ -98,7 +99,7 @@ void make_sample_plan(const tv_sample_desc* d, tv_sample_plan* p) {
     p->cluster_ctas = c;
     p->threads = threads;
     p->slice = slice;
-    p->smem_bytes = (int32_t)(2 * sizeof(float) * (size_t)slice);
+    p->smem_bytes = (int32_t)(4 * sizeof(float) * (size_t)slice);
     p->launches = 1;
 }
 

@@ -15,13 +15,17 @@
 // where max(0, p - c q) > 0, (p - c q)/Z - q = (p - (c + Z) q)/Z, and where it
 // is 0 both forms are <= 0.  A zero Z keeps (c, Z).
 //
-// Layout: one thread-block cluster of C CTAs per sequence.  CTA k holds the
-// vocabulary slice [k*S, (k+1)*S) of the current node's p and q rows in
-// shared memory, loaded once per node when first needed; every later sibling
-// pass and the final draw read the cached slice.  Each normaliser is an fp64
-// reduction (per thread, warp shuffle, CTA, then the C partials read through
-// distributed shared memory in rank order), so every CTA obtains the same
-// bits and takes the same branch without further communication.
+// Layout: one thread-block cluster of C CTAs per sequence; CTA k owns the
+// vocabulary slice [k*S, (k+1)*S).  When the walk arrives at a node every CTA
+// starts a bulk copy of its slice of that node's p and q rows into one of two
+// shared-memory buffers, so the row is usually resident by the time a
+// rejection needs it.  Each normaliser is an fp64 reduction: per lane over a
+// contiguous per-warp segment, warp shuffle, CTA, then every CTA pushes its
+// partial to all peers with st.async, which completes on the receiver's own
+// mbarrier; every CTA adds the C partials in rank order, so all obtain the
+// same bits and take the same branches.  The bonus draw reuses the per-CTA
+// and per-warp partials of the last pass: the owning CTA, warp and lane are
+// located from them, and one lane scans its few elements.
 #include <cooperative_groups.h>
 
 #include "tv_common.cuh"
@@ -35,21 +39,73 @@ namespace {
 constexpr int MAX_NODES = 1024;
 constexpr int MAX_THREADS = 512;
 constexpr int MAX_CLUSTER = 16;
+constexpr long long WAIT_LIMIT = 1ll << 32;  // clock cycles (~2 s)
 
 struct SampleShared {
-    int16_t parent[MAX_NODES];
-    int16_t child_start[MAX_NODES];
-    int16_t child_count[MAX_NODES];
-    int16_t child_list[MAX_NODES];
+    int32_t parent[MAX_NODES];
     int32_t token[MAX_NODES];
     double ch_p[32], ch_q[32], ch_u[32];
     int32_t ch_node[32];
+    int ch_n;      // children gathered in this batch
+    int ch_next;   // index where the scan for the next batch resumes (N when done)
     double warp_part[MAX_THREADS / 32];
-    double cta_part[2];           // this CTA's partial, double-buffered by pass parity
-    double all_part[MAX_CLUSTER]; // every CTA's partial of the latest pass
-    int bad;
+    double peer[2][MAX_CLUSTER];  // partials from every CTA of the cluster, by pass parity
+    unsigned long long peer_bar[2];
+    unsigned long long row_bar[2];
+    int timeout;
     int found;
+    int wsel;
+    double wbefore;
 };
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// bounded wait on one phase; false (and the timeout flag set) when it runs out
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* timeout) {
+    if (mbar_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (;;) {
+        if (mbar_try(bar, parity)) return true;
+        if (clock64() - t0 > WAIT_LIMIT) {
+            *timeout = 1;
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+// remote store of one double that completes 8 bytes on the receiver's mbarrier
+__device__ __forceinline__ void st_async_f64(uint32_t remote_addr, double v, uint32_t remote_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];" ::"r"(remote_addr),
+                 "l"(__double_as_longlong(v)), "r"(remote_bar)
+                 : "memory");
+}
+// bulk copy global -> this CTA's shared memory, completing on a local mbarrier
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
 
 __device__ __forceinline__ double warp_sum_d(double v) {
 #pragma unroll
@@ -65,70 +121,92 @@ __device__ __forceinline__ double resid(float p, float q, double c) {
 struct Walker {
     const SampleArgs& a;
     SampleShared& sh;
-    float* ps;
-    float* qs;
-    int rank, C, lo, n, tid, lane, warp, nwarps;
-    int pass;
+    float* buf;      // [2][2][slice]: buffer x holds p at buf + 2*x*slice, q right after
+    int b, rank, C, lo, n, tid, lane, warp, nwarps, segw;
+    bool bulk;
+    int passes;      // cluster passes so far
+    int row_uses[2];
+    bool row_pending[2];
 
-    // Sum over the whole row of resid(p, q, c); every CTA returns the same value.
-    __device__ double cluster_sum(double c) {
-        double acc = 0.0;
-        for (int i = tid; i < n; i += blockDim.x) acc += resid(ps[i], qs[i], c);
-        acc = warp_sum_d(acc);
-        if (lane == 0) sh.warp_part[warp] = acc;
+    __device__ float* ps(int x) const { return buf + (size_t)2 * x * a.slice; }
+    __device__ float* qs(int x) const { return ps(x) + a.slice; }
+    __device__ uint32_t row_bar(int x) const { return smem_u32(&sh.row_bar[x]); }
+
+    // Wait until buffer x holds its row (collective).
+    __device__ void wait_row(int x) {
+        if (!row_pending[x]) return;
+        mbar_wait(row_bar(x), row_uses[x] & 1, &sh.timeout);
+        ++row_uses[x];
+        row_pending[x] = false;
+    }
+
+    // Start loading this CTA's slice of node u's p and q rows into buffer x (collective).
+    __device__ void issue_row(int x, int u) {
+        wait_row(x);  // the buffer's previous copy must have landed before it is reused
+        const size_t base = ((size_t)b * a.N + u) * (size_t)a.V + lo;
+        if (bulk) {
+            if (tid == 0) {
+                mbar_expect_tx(row_bar(x), (uint32_t)(8 * n));
+                if (n > 0) {
+                    bulk_load(smem_u32(ps(x)), a.p + base, (uint32_t)(4 * n), row_bar(x));
+                    bulk_load(smem_u32(qs(x)), a.q + base, (uint32_t)(4 * n), row_bar(x));
+                }
+            }
+        } else {
+            float* pd = ps(x);
+            float* qd = qs(x);
+            for (int i = tid; i < n; i += blockDim.x) {
+                pd[i] = __ldg(a.p + base + i);
+                qd[i] = __ldg(a.q + base + i);
+            }
+            __syncthreads();
+            if (tid == 0) mbar_expect_tx(row_bar(x), 0);
+        }
+        row_pending[x] = true;
+    }
+
+    // Sum over the whole row of resid(p, q, c) from buffer x; every CTA returns
+    // the same value.  Leaves this CTA's per-warp partials in sh.warp_part and
+    // every CTA's partial in sh.peer[parity of the pass].
+    __device__ double cluster_pass(int x, double c) {
+        const float* p = ps(x);
+        const float* q = qs(x);
+        const int s0 = min(n, warp * segw), s1 = min(n, s0 + segw);
+        double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+        int i = s0 + lane;
+        for (; i + 96 < s1; i += 128) {
+            a0 += resid(p[i], q[i], c);
+            a1 += resid(p[i + 32], q[i + 32], c);
+            a2 += resid(p[i + 64], q[i + 64], c);
+            a3 += resid(p[i + 96], q[i + 96], c);
+        }
+        for (; i < s1; i += 32) a0 += resid(p[i], q[i], c);
+        const double wsum = warp_sum_d((a0 + a1) + (a2 + a3));
+        if (lane == 0) sh.warp_part[warp] = wsum;
         __syncthreads();
-        const int slot = pass & 1;
-        ++pass;
+        const int par = passes & 1;
+        const uint32_t use = (uint32_t)(passes >> 1);
+        ++passes;
         if (tid == 0) {
             double s = 0.0;
-            for (int w = 0; w < nwarps; ++w) s += sh.warp_part[w];
-            sh.cta_part[slot] = s;
+            for (int k = 0; k < nwarps; ++k) s += sh.warp_part[k];
+            if (C == 1) {
+                sh.peer[par][0] = s;
+            } else {
+                const uint32_t bar = smem_u32(&sh.peer_bar[par]);
+                mbar_expect_tx(bar, (uint32_t)(8 * C));
+                const uint32_t slot = smem_u32(&sh.peer[par][rank]);
+                for (int r = 0; r < C; ++r) st_async_f64(mapa(slot, r), s, mapa(bar, r));
+            }
         }
         if (C == 1) {
             __syncthreads();
-            if (tid == 0) sh.all_part[0] = sh.cta_part[slot];
-            __syncthreads();
-            return sh.all_part[0];
-        }
-        cg::cluster_group cluster = cg::this_cluster();
-        cluster.sync();  // every CTA's partial of this pass is written
-        if (tid < C) sh.all_part[tid] = *cluster.map_shared_rank(&sh.cta_part[slot], tid);
-        __syncthreads();
-        double total = 0.0;
-        for (int k = 0; k < C; ++k) total += sh.all_part[k];
-        // A later pass writes the other slot; the pass after that rewrites this
-        // slot only once every CTA has passed the next cluster.sync, i.e. after
-        // all remote reads of this pass.
-        return total;
-    }
-
-    __device__ void load_row(int u) {
-        const size_t base = ((size_t)(blockIdx.x / C) * a.N + u) * (size_t)a.V + lo;
-        const float* pr = a.p + base;
-        const float* qr = a.q + base;
-        if (a.vec4) {
-            const int n4 = n >> 2;
-            const float4* p4 = reinterpret_cast<const float4*>(pr);
-            const float4* q4 = reinterpret_cast<const float4*>(qr);
-            float4* ps4 = reinterpret_cast<float4*>(ps);
-            float4* qs4 = reinterpret_cast<float4*>(qs);
-#pragma unroll 4
-            for (int i = tid; i < n4; i += blockDim.x) {
-                ps4[i] = __ldg(p4 + i);
-                qs4[i] = __ldg(q4 + i);
-            }
-            for (int i = (n4 << 2) + tid; i < n; i += blockDim.x) {
-                ps[i] = __ldg(pr + i);
-                qs[i] = __ldg(qr + i);
-            }
         } else {
-#pragma unroll 4
-            for (int i = tid; i < n; i += blockDim.x) {
-                ps[i] = __ldg(pr + i);
-                qs[i] = __ldg(qr + i);
-            }
+            mbar_wait(smem_u32(&sh.peer_bar[par]), use & 1, &sh.timeout);
         }
-        __syncthreads();
+        double total = 0.0;
+        for (int r = 0; r < C; ++r) total += sh.peer[par][r];
+        return total;
     }
 };
 
@@ -142,45 +220,36 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
     const int N = a.N;
     const int lo = min(a.V, rank * a.slice);
     const int n = min(a.V, lo + a.slice) - lo;
-    float* ps = reinterpret_cast<float*>(sample_dyn);
-    float* qs = ps + a.slice;
 
-    // ---- tree: validate, child lists in ascending index order
-    if (tid == 0) sh.bad = 0;
+    if (tid == 0) {
+        sh.timeout = 0;
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(smem_u32(&sh.row_bar[x]), 1);
+            mbar_init(smem_u32(&sh.peer_bar[x]), 1);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (C > 1) cg::this_cluster().sync();  // every CTA's barriers exist before any peer pushes to them
+
+    Walker w{a, sh, reinterpret_cast<float*>(sample_dyn), b, rank, C, lo, n, tid, lane, warp, nwarps,
+             ((n + nwarps - 1) / nwarps + 31) / 32 * 32, a.vec4 != 0, 0, {0, 0}, {false, false}};
+    // the root's row is needed unless its first child is accepted: start it now
+    w.issue_row(0, 0);
+
+    // ---- tree and tokens; a malformed sequence gets -1 outputs
     for (int i = tid; i < N; i += blockDim.x) {
-        sh.parent[i] = (int16_t)max(-1, min(a.parent[(size_t)b * N + i], MAX_NODES - 1));
+        sh.parent[i] = a.parent[(size_t)b * N + i];
         sh.token[i] = a.tokens[(size_t)b * N + i];
-        sh.child_count[i] = 0;
     }
     __syncthreads();
+    bool bad_local = false;
     for (int i = tid; i < N; i += blockDim.x) {
-        const int p = a.parent[(size_t)b * N + i];
-        const bool ok = (i == 0) ? p == -1 : (p >= 0 && p < i && sh.token[i] >= 0 && sh.token[i] < a.V);
-        if (!ok) sh.bad = 1;
+        const int p = sh.parent[i];
+        bad_local |= (i == 0) ? p != -1 : (p < 0 || p >= i || sh.token[i] < 0 || sh.token[i] >= a.V);
     }
-    __syncthreads();
-    const bool bad = sh.bad != 0;
-    if (!bad) {
-        if (tid == 0) {
-            for (int c = 1; c < N; ++c) sh.child_count[sh.parent[c]]++;
-            int s = 0;
-            for (int v = 0; v < N; ++v) { sh.child_start[v] = (int16_t)s; s += sh.child_count[v]; }
-        }
-        __syncthreads();
-        // child c goes to slot start(parent) + (number of earlier siblings)
-        for (int c = 1 + tid; c < N; c += blockDim.x) {
-            const int p = sh.parent[c];
-            int r = 0;
-            for (int j = p + 1; j < c; ++j) r += sh.parent[j] == p;
-            sh.child_list[sh.child_start[p] + r] = (int16_t)c;
-        }
-        __syncthreads();
-    }
-
-    Walker w{a, sh, ps, qs, rank, C, lo, n, tid, lane, warp, nwarps, 0};
     int32_t* path_out = a.path + (size_t)b * N;
-
-    if (bad) {
+    if (__syncthreads_or(bad_local)) {
         if (rank == 0) {
             for (int i = tid; i < N; i += blockDim.x) path_out[i] = -1;
             if (tid == 0) {
@@ -189,66 +258,105 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
                 report(a.status, TV_ERR_TREE);
             }
         }
-        if (C > 1) cg::this_cluster().sync();
+        w.wait_row(0);
         return;
     }
 
     // ---- walk from the root
-    int u = 0, len = 0;
-    int loaded = -1;  // node whose row slice sits in ps/qs
+    int u = 0, len = 0, x = 0;
     double cur_c = 0.0, cur_z = 1.0;
+    int last_pass_node = -1;
+    double last_pass_c = -1.0;
     for (;;) {
         cur_c = 0.0;
         cur_z = 1.0;
         int accepted = -1;
-        const int cs = sh.child_start[u], cc = sh.child_count[u];
-        for (int g0 = 0; g0 < cc && accepted < 0; g0 += 32) {
-            // gather up to 32 children's scalars at once
-            __syncthreads();
-            if (warp == 0 && g0 + lane < cc) {
-                const int c = sh.child_list[cs + g0 + lane];
-                const int x = sh.token[c];
-                const size_t row = ((size_t)b * N + u) * (size_t)a.V;
-                sh.ch_node[lane] = c;
-                sh.ch_p[lane] = (double)__ldg(a.p + row + x);
-                sh.ch_q[lane] = (double)__ldg(a.q + row + x);
-                sh.ch_u[lane] = (double)__ldg(a.uniforms + (size_t)b * N + c);
+        int scan = u + 1;
+        while (accepted < 0 && scan < N) {
+            // warp 0 collects the next (up to 32) children of u in ascending order and
+            // gathers their draft tokens' p, q and acceptance draws
+            if (warp == 0) {
+                int found = 0, next = N;
+                for (int c0 = scan; c0 < N; c0 += 32) {
+                    const int c = c0 + lane;
+                    const bool kid = c < N && sh.parent[c] == u;
+                    const unsigned m = __ballot_sync(0xffffffffu, kid);
+                    const int pos = found + __popc(m & ((1u << lane) - 1u));
+                    if (kid && pos < 32) sh.ch_node[pos] = c;
+                    if (found + __popc(m) > 32) {
+                        // resume after the last child taken from this chunk
+                        unsigned mm = m;
+                        for (int t = 0; t < 32 - found; ++t) mm &= mm - 1u;
+                        next = c0 + __ffs(mm) - 1;
+                        found = 32;
+                        break;
+                    }
+                    found += __popc(m);
+                }
+                __syncwarp();
+                if (lane < found) {
+                    const int c = sh.ch_node[lane];
+                    const size_t row = ((size_t)b * N + u) * (size_t)a.V;
+                    sh.ch_p[lane] = (double)__ldg(a.p + row + sh.token[c]);
+                    sh.ch_q[lane] = (double)__ldg(a.q + row + sh.token[c]);
+                    sh.ch_u[lane] = (double)__ldg(a.uniforms + (size_t)b * N + c);
+                }
+                if (lane == 0) {
+                    sh.ch_n = found;
+                    sh.ch_next = next;
+                }
             }
             __syncthreads();
-            const int gn = min(32, cc - g0);
+            const int gn = sh.ch_n;
             for (int k = 0; k < gn; ++k) {
                 const double px = sh.ch_p[k], qx = sh.ch_q[k], r = sh.ch_u[k];
                 const double num = cur_c == 0.0 ? px : fmax(0.0, fma(-cur_c, qx, px));
                 const bool acc = qx > 0.0 ? (r < num / (cur_z * qx)) : (num > 0.0);
-                if (acc) { accepted = sh.ch_node[k]; break; }
-                if (loaded != u) { w.load_row(u); loaded = u; }
+                if (acc) {
+                    accepted = sh.ch_node[k];
+                    break;
+                }
+                w.wait_row(x);
                 const double c_new = cur_c + cur_z;
-                const double z_new = w.cluster_sum(c_new);
-                if (z_new > 0.0) { cur_c = c_new; cur_z = z_new; }
+                const double z_new = w.cluster_pass(x, c_new);
+                last_pass_node = u;
+                last_pass_c = c_new;
+                if (z_new > 0.0) {
+                    cur_c = c_new;
+                    cur_z = z_new;
+                }
             }
+            scan = sh.ch_next;
+            __syncthreads();  // ch_* are rewritten by the next batch
         }
-        if (accepted >= 0) {
-            if (rank == 0 && tid == 0) path_out[len] = accepted;
-            ++len;
-            u = accepted;
-            continue;
-        }
-        break;
+        if (accepted < 0) break;
+        if (rank == 0 && tid == 0) path_out[len] = accepted;
+        ++len;
+        u = accepted;
+        x ^= 1;
+        w.issue_row(x, u);  // prefetch the new node's row into the other buffer
     }
 
     // ---- bonus token: first index whose running residual mass exceeds u0 * total
-    if (loaded != u) { w.load_row(u); loaded = u; }
-    const double total = w.cluster_sum(cur_c);  // also leaves every CTA's partial in all_part
+    w.wait_row(x);
+    double total;
+    if (last_pass_node == u && last_pass_c == cur_c) {
+        total = cur_z;  // the last pass summed exactly this distribution; reuse its partials
+    } else {
+        total = w.cluster_pass(x, cur_c);
+    }
+    const int par = (w.passes - 1) & 1;
     const double target = (double)__ldg(a.uniforms + (size_t)b * N) * total;
-    // first CTA whose inclusive prefix exceeds the target; the last CTA with
-    // mass if rounding leaves none
     int owner = -1, last_pos_cta = -1;
     double before = 0.0, run = 0.0;
     for (int k = 0; k < C; ++k) {
-        const double pk = sh.all_part[k];
+        const double pk = sh.peer[par][k];
         if (pk > 0.0) last_pos_cta = k;
         if (owner < 0) {
-            if (run + pk > target) { owner = k; before = run; }
+            if (run + pk > target) {
+                owner = k;
+                before = run;
+            }
             run += pk;
         }
     }
@@ -256,54 +364,66 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
     if (fallback) owner = last_pos_cta;
 
     if (rank == owner) {
-        // warp segments of the slice, contiguous, 32-aligned
-        const int segw = ((n + nwarps - 1) / nwarps + 31) / 32 * 32;
-        const int s0 = min(n, warp * segw), s1 = min(n, s0 + segw);
-        double ws = 0.0;
-        for (int i = s0 + lane; i < s1; i += 32) ws += resid(ps[i], qs[i], cur_c);
-        ws = warp_sum_d(ws);
-        if (lane == 0) sh.warp_part[warp] = ws;
-        if (tid == 0) sh.found = -1;
-        __syncthreads();
-        __shared__ int s_warp;
-        __shared__ double s_before;
+        const float* p = w.ps(x);
+        const float* q = w.qs(x);
         if (tid == 0) {
+            // first warp segment whose running sum crosses the target; the last one
+            // with mass if rounding leaves none
             int wsel = -1, wlast = -1;
             double rb = before, rr = before;
             for (int k = 0; k < nwarps; ++k) {
                 if (sh.warp_part[k] > 0.0) wlast = k;
                 if (wsel < 0 && !fallback) {
-                    if (rr + sh.warp_part[k] > target) { wsel = k; rb = rr; }
+                    if (rr + sh.warp_part[k] > target) {
+                        wsel = k;
+                        rb = rr;
+                    }
                     rr += sh.warp_part[k];
                 }
             }
-            if (wsel < 0) { wsel = wlast; rb = -INFINITY; }  // rounding: last positive element
-            s_warp = wsel;
-            s_before = rb;
+            sh.wsel = wsel >= 0 ? wsel : wlast;
+            sh.wbefore = wsel >= 0 ? rb : -INFINITY;  // -inf: take the segment's last positive element
+            sh.found = -1;
         }
         __syncthreads();
-        if (warp == s_warp) {
-            const bool take_last = s_before == -INFINITY;
-            double rr = s_before;
-            int pick = -1, lastp = -1;
-            for (int i0 = s0; i0 < s1; i0 += 32) {
-                const int i = i0 + lane;
-                const double v = i < s1 ? resid(ps[i], qs[i], cur_c) : 0.0;
-                double sc = v;  // inclusive scan over the lanes
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const double t = __shfl_up_sync(0xffffffffu, sc, o);
-                    if (lane >= o) sc += t;
-                }
-                const unsigned pos = __ballot_sync(0xffffffffu, v > 0.0);
-                if (pos) lastp = i0 + 31 - __clz(pos);
-                if (!take_last) {
-                    const unsigned hit = __ballot_sync(0xffffffffu, rr + sc > target);
-                    if (hit) { pick = i0 + __ffs(hit) - 1; break; }
-                    rr += __shfl_sync(0xffffffffu, sc, 31);
-                }
+        if (warp == sh.wsel) {
+            const int s0 = min(n, warp * w.segw), s1 = min(n, s0 + w.segw);
+            const int per = (s1 - s0 + 31) / 32;
+            const int e0 = min(s1, s0 + lane * per), e1 = min(s1, e0 + per);
+            double mine = 0.0;
+            int mylast = -1;
+            for (int i = e0; i < e1; ++i) {
+                const double v = resid(p[i], q[i], cur_c);
+                mine += v;
+                if (v > 0.0) mylast = i;
             }
-            if (pick < 0) pick = lastp;  // rounding left no crossing inside the segment
+            double incl = mine;  // inclusive scan over the lanes
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const double t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            const bool take_last = sh.wbefore == -INFINITY;
+            const unsigned hit = take_last ? 0u : __ballot_sync(0xffffffffu, sh.wbefore + incl > target);
+            const unsigned pos = __ballot_sync(0xffffffffu, mylast >= 0);
+            int pick = -1;
+            if (hit) {
+                const int hl = __ffs(hit) - 1;
+                if (lane == hl) {
+                    double rsum = sh.wbefore + incl - mine;
+                    for (int i = e0; i < e1; ++i) {
+                        const double v = resid(p[i], q[i], cur_c);
+                        if (v > 0.0) pick = i;
+                        rsum += v;
+                        if (rsum > target && v > 0.0) break;
+                    }
+                }
+                pick = __shfl_sync(0xffffffffu, pick, hl);
+            } else if (pos) {
+                // rounding left no crossing: the segment's last positive element
+                const int ll = 31 - __clz(pos);
+                pick = __shfl_sync(0xffffffffu, mylast, ll);
+            }
             if (lane == 0) sh.found = pick;
         }
         __syncthreads();
@@ -313,11 +433,16 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
         }
         for (int i = len + tid; i < N; i += blockDim.x) path_out[i] = -1;
     } else if (owner < 0 && rank == 0) {
-        // no mass anywhere (all-zero distribution)
-        if (tid == 0) { a.bonus[b] = -1; a.len[b] = len; }
+        // no mass anywhere (an all-zero distribution)
+        if (tid == 0) {
+            a.bonus[b] = -1;
+            a.len[b] = len;
+        }
         for (int i = len + tid; i < N; i += blockDim.x) path_out[i] = -1;
     }
-    if (C > 1) cg::this_cluster().sync();  // keep shared memory alive for remote readers
+    // no copy may still be landing in this CTA's shared memory when it retires
+    w.wait_row(x ^ 1);
+    if (tid == 0 && sh.timeout) report(a.status, TV_ERR_TIMEOUT);
 }
 
 }  // namespace
@@ -326,19 +451,20 @@ int sample_max_cluster() {
     static int best = -1;
     if (best >= 0) return best;
     best = 8;
-    if (cudaFuncSetAttribute(verify_sample_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+    if (cudaFuncSetAttribute(verify_sample_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+        cudaFuncSetAttribute(verify_sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024) ==
+            cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
         cfg.gridDim = dim3(16, 1, 1);
         cfg.blockDim = dim3(MAX_THREADS, 1, 1);
-        cfg.dynamicSmemBytes = 96 * 1024;
+        cfg.dynamicSmemBytes = 160 * 1024;
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 16;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        cudaFuncSetAttribute(verify_sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
         int clusters = 0;
         if (cudaOccupancyMaxActiveClusters(&clusters, verify_sample_kernel, &cfg) == cudaSuccess && clusters > 0)
             best = 16;
