@@ -44,10 +44,18 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback", {}
 
 
-def kernel_source_hash() -> str:
+# the sources each kernel's code and launch configuration come from
+KERNEL_SOURCES = {
+    "attn_tc": ("api.cu", "attn_tc.cu", "kernels.h", "tv_common.cuh"),
+    "attn_simt": ("api.cu", "attn_simt.cu", "kernels.h", "tv_common.cuh"),
+    "verify_sample": ("api.cu", "sample.cu", "kernels.h", "tv_common.cuh"),
+}
+
+
+def kernel_source_hash(kernel_key: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "tree_speculative_decoding_07_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel_key]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -62,7 +70,7 @@ def ncu_traffic(kernel_key: str, workload: str):
         with open(path) as f:
             d = json.load(f)
         e = d[kernel_key][workload]
-        if e.get("source_hash") != kernel_source_hash():
+        if e.get("source_hash") != kernel_source_hash(kernel_key):
             return None
         return float(e["dram_bytes_per_launch"])
     except Exception:
@@ -210,29 +218,32 @@ def run_ours(args, rank, world, local_rank):
         if s2:
             raise tv.TreeVerifyError(s2, "tv_verify_sample")
 
-    def step(mid):
+    def step():
         attn_call(stream)
-        mid.record(stream)
         sample_call(stream)
 
-    # ---- device-resident timing (L2 flushed before every step).  Each call is
-    # replayed from a CUDA graph so host launch work stays out of the events.
+    # ---- device-resident timing (L2 flushed before every step).  The step is
+    # replayed from one CUDA graph (attention, then the walk, launched with a
+    # programmatic dependency so the walk's set-up overlaps attention's tail), so
+    # host launch work stays out of the events.  Each kernel is then timed alone
+    # from its own graph for the per-kernel figures and the roofline.
     W, K = args.warmup, args.steps
     for _ in range(2):
-        step(torch.cuda.Event())
+        step()
     torch.cuda.synchronize()
-    g_attn, g_samp = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    g_step, g_attn, g_samp = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        attn_call(torch.cuda.current_stream())
+        sample_call(torch.cuda.current_stream())
     with torch.cuda.graph(g_attn):
         attn_call(torch.cuda.current_stream())
     with torch.cuda.graph(g_samp):
         sample_call(torch.cuda.current_stream())
     torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     for _ in range(W):
         flush.zero_()
-        g_attn.replay()
-        g_samp.replay()
+        g_step.replay()
     torch.cuda.synchronize()
     clocks = ClockSampler(local_rank)
     if world > 1:
@@ -242,20 +253,31 @@ def run_ours(args, rank, world, local_rank):
     t_wall = time.perf_counter()
     for k in range(K):
         flush.zero_()
-        e0, mid, e1 = ev[k]
+        e0, e1 = ev[k]
         e0.record(stream)
-        g_attn.replay()
-        mid.record(stream)
-        g_samp.replay()
+        g_step.replay()
         e1.record(stream)
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
-    attn_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
-    samp_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
-    step_ms = [ev[k][0].elapsed_time(ev[k][2]) for k in range(K)]
+    step_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
+
+    def kernel_ms(graph):
+        for _ in range(W):
+            flush.zero_()
+            graph.replay()
+        for k in range(K):
+            flush.zero_()
+            ev[k][0].record(stream)
+            graph.replay()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        return [e0.elapsed_time(e1) for e0, e1 in ev]
+
+    attn_ms = kernel_ms(g_attn)
+    samp_ms = kernel_ms(g_samp)
     total_ms = float(sum(step_ms))
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())}")
@@ -275,7 +297,7 @@ def run_ours(args, rank, world, local_rank):
         for key, t in pin.items():
             dst = d[key]
             (dst.view(torch.int16) if dst.dtype == torch.bfloat16 else dst).copy_(t, non_blocking=True)
-        step(torch.cuda.Event())
+        step()
         out_h.copy_(out, non_blocking=True)
         path_h.copy_(path, non_blocking=True)
         alen_h.copy_(alen, non_blocking=True)
@@ -330,6 +352,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": f"flushed before every step ({L2_FLUSH_BYTES >> 20} MB write, outside the step events)"},
         "attention_us": attn_avg_s * 1e6,
         "sample_us": (sum(samp_ms) / K) * 1e3,
+        "per_kernel_timing": "each kernel replayed alone from its own graph, L2 flushed before each launch",
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": ncu_traffic(kernel_key, args.workload), "kernel": kernel_key,
                      "algorithmic_bytes": a_bytes, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"

@@ -402,6 +402,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     };
     int ids = (warp == 0 || warp == 3) ? load_id(lane >> 3) : 0;
     __syncthreads();
+    // a kernel launched after this one with programmatic stream serialisation may
+    // start its set-up now; it waits for this grid before reading anything
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     tc_fence_after();
     const uint32_t tmem = s_tmem;
 

@@ -231,6 +231,10 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
     }
     __syncthreads();
     if (C > 1) cg::this_cluster().sync();  // every CTA's barriers exist before any peer pushes to them
+    // the kernel may have been launched while the previous one on the stream was still
+    // running (programmatic dependent launch): its inputs are read only after that
+    // kernel has completed and its memory is visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     Walker w{a, sh, reinterpret_cast<float*>(sample_dyn), b, rank, C, lo, n, tid, lane, warp, nwarps,
              ((n + nwarps - 1) / nwarps + 31) / 32 * 32, a.vec4 != 0, 0, {0, 0}, {false, false}};
@@ -482,17 +486,21 @@ cudaError_t launch_verify_sample(const SampleArgs& a, cudaStream_t st, int* laun
         if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     cfg.gridDim = dim3((unsigned)a.cluster * (unsigned)a.B, 1, 1);
     cfg.blockDim = dim3(a.threads, 1, 1);
     cfg.dynamicSmemBytes = a.smem_bytes;
     cfg.stream = st;
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = a.cluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    // launch set-up may overlap the previous kernel's tail; the kernel waits for that
+    // kernel (griddepcontrol.wait) before reading any input
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = a.cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = a.cluster > 1 ? 1 : 0;
+    cfg.numAttrs = a.cluster > 1 ? 2 : 1;
     *launches = 1;
     return cudaLaunchKernelEx(&cfg, verify_sample_kernel, a);
 }
