@@ -57,6 +57,8 @@ constexpr int BLK_PER_TILE = TN / TV_BLOCK;
 constexpr int KST = 3;           // K ring depth
 constexpr int VST = 3;           // V ring depth
 constexpr int MAX_SPLITS = 16;
+constexpr int ID_RING = 8;       // tiles of block ids held per producer
+constexpr int ID_AHEAD = 6;      // tiles between an id copy's issue and its use
 constexpr uint32_t SQ_OFF = 0;             // Q: 2 x [128 rows][128 B], swizzled
 constexpr uint32_t SK_OFF = 32768;         // K ring: KST x 32 KB
 constexpr uint32_t SV_OFF = SK_OFF + KST * 32768u;  // V ring: VST x 32 KB
@@ -76,10 +78,12 @@ constexpr int BAR_V_EMPTY = BAR_V_FULL + VST;    // VST: P V done with the V slo
 constexpr int BAR_S_FULL = BAR_V_EMPTY + VST;    // 2: S buffer written
 constexpr int BAR_P_FULL = BAR_S_FULL + 2;       // 2: group's P written (and O rescaled)
 constexpr int BAR_O_DONE = BAR_P_FULL + 2;       // 2: group's P V done
-constexpr int BAR_Q_READY = BAR_O_DONE + 2;      // Q staged
-constexpr int BAR_DRAIN = BAR_Q_READY + 1;       // all MMAs of the CTA done
-constexpr int BAR_COUNT = BAR_DRAIN + 1;
-static_assert(BAR_COUNT == 2 * KST + 2 * VST + 8, "barrier slots overlap");
+constexpr int BAR_PV_DONE = BAR_O_DONE + 2;      // 2: P V of the tile in an S buffer done (buffer free)
+constexpr int BAR_Q_READY = BAR_PV_DONE + 2;     // Q staged
+constexpr int BAR_DRAIN_QK = BAR_Q_READY + 1;    // all S = Q K^T MMAs done
+constexpr int BAR_DRAIN_PV = BAR_DRAIN_QK + 1;   // all P V MMAs done
+constexpr int BAR_COUNT = BAR_DRAIN_PV + 1;
+static_assert(BAR_COUNT == 2 * KST + 2 * VST + 11, "barrier slots overlap");
 
 // instruction descriptor, kind::f16: D fp32, A/B bf16, A K-major,
 // B K-major (S = Q K^T) or MN-major (O += P V), M = 128, N = 128
@@ -143,6 +147,15 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// 4-byte asynchronous global -> shared copy (no register holds the value)
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -320,6 +333,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort, s_bad;
     __shared__ int32_t s_par[TV_MAX_NODES_ATTN];
+    __shared__ __align__(16) int32_t s_ids[2][ID_RING * BLK_PER_TILE];  // block ids, per producer
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int split = blockIdx.x, tile = blockIdx.y;
@@ -339,7 +353,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     auto s_full = [&](int s) { return bar0 + 8u * (BAR_S_FULL + s); };
     auto p_full = [&](int x) { return bar0 + 8u * (BAR_P_FULL + x); };
     auto o_done = [&](int x) { return bar0 + 8u * (BAR_O_DONE + x); };
-    const uint32_t q_ready = bar0 + 8u * BAR_Q_READY, mma_drain = bar0 + 8u * BAR_DRAIN;
+    auto pv_done = [&](int sb) { return bar0 + 8u * (BAR_PV_DONE + sb); };
+    const uint32_t q_ready = bar0 + 8u * BAR_Q_READY;
+    const uint32_t drain_qk = bar0 + 8u * BAR_DRAIN_QK, drain_pv = bar0 + 8u * BAR_DRAIN_PV;
     volatile int* abort_flag = &s_abort;
     // results of the softmax groups, consumed by the split merge after the role blocks
     float o[64];
@@ -364,9 +380,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             mbar_init(s_full(s), 1);
             mbar_init(p_full(s), 128);
             mbar_init(o_done(s), 1);
+            mbar_init(pv_done(s), 1);
         }
         mbar_init(q_ready, 256);
-        mbar_init(mma_drain, 1);
+        mbar_init(drain_qk, 1);
+        mbar_init(drain_pv, 1);
         fence_barrier_init();
     }
     if (warp == 2) {
@@ -384,23 +402,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     split_range(bad_len ? 0 : total, S, split, t0, t1);
     const int ntiles = (t1 - t0 + TN - 1) / TN;
     const int last_blk = (t1 - 1) / TV_BLOCK;
-    // the producer's first block ids are fetched before the barrier so the
-    // loads overlap barrier set-up and TMEM allocation
+    // Block ids reach the producers through a shared-memory ring that cp.async
+    // fills ID_AHEAD tiles ahead of use, so no tile's copies wait on a
+    // block-table load (a register loaded one tile earlier would stall every
+    // iteration for one global-memory latency).  The first copies start before
+    // the barrier, overlapping barrier set-up and TMEM allocation.
     const int32_t* bt = a.block_table + (size_t)b * a.max_blocks;
-    // producer lane l holds the block id of block l % 8 of tile j + l / 8: four tiles of lookahead
-    bool bad_id = false;
-    auto load_id = [&](int jt) {
-        if (jt >= ntiles) return 0;
-        int bi = (t0 + jt * TN) / TV_BLOCK + (lane & 7);
-        if (bi > last_blk) bi = last_blk;
-        int id = bt[bi];
-        if (id < 0 || id >= a.num_blocks) {
-            bad_id = true;
-            id = 0;
+    const int prod = warp == 0 ? 0 : 1;
+    auto prefetch_ids = [&](int jt) {
+        if (jt < ntiles && lane < BLK_PER_TILE) {
+            int bi = (t0 + jt * TN) / TV_BLOCK + lane;
+            if (bi > last_blk) bi = last_blk;
+            cp_async_4(smem_u32(&s_ids[prod][(jt % ID_RING) * BLK_PER_TILE + lane]), bt + bi);
         }
-        return id;
+        cp_async_commit();  // one group per tile on every lane, empty or not
     };
-    int ids = (warp == 0 || warp == 3) ? load_id(lane >> 3) : 0;
+    if (warp == 0 || warp == 3)
+        for (int jt = 0; jt < ID_AHEAD; ++jt) prefetch_ids(jt);
     __syncthreads();
     // a kernel launched after this one with programmatic stream serialisation may
     // start its set-up now; it waits for this grid before reading anything
@@ -414,13 +432,26 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const CUtensorMap* map = is_k ? &tmk : &tmv;
         const int depth = is_k ? KST : VST;
         int issued = 0;
+        bool bad_id = false;
         for (int j = 0; j < ntiles; ++j) {
             const int s = j % depth;
             if (j >= depth && !warp_wait(is_k ? k_empty(s) : v_empty(s), ((j - depth) / depth) & 1, abort_flag)) break;
-            int cur[BLK_PER_TILE];
-#pragma unroll
-            for (int k = 0; k < BLK_PER_TILE; ++k) cur[k] = __shfl_sync(0xffffffffu, ids, k);
+            // this lane's id copies for tile j are complete; the warp barrier makes
+            // every lane's copies visible to lane 0
+            cp_async_wait<ID_AHEAD - 1>();
+            __syncwarp();
             if (lane == 0) {
+                int cur[BLK_PER_TILE];
+                const int32_t* ring = &s_ids[prod][(j % ID_RING) * BLK_PER_TILE];
+#pragma unroll
+                for (int k = 0; k < BLK_PER_TILE; ++k) {
+                    int id = ring[k];
+                    if (id < 0 || id >= a.num_blocks) {
+                        bad_id = true;
+                        id = 0;
+                    }
+                    cur[k] = id;
+                }
                 const uint32_t full = is_k ? k_full(s) : v_full(s);
                 const uint32_t dst = is_k ? sK(s) : sV(s);
                 mbar_expect_tx(full, TILE_BYTES);
@@ -430,15 +461,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     for (int h = 0; h < 2; ++h)
                         tma_load_4d(dst + h * HALF_BYTES + k * 2048u, map, full, 0, kvh * 2 + h, 0, cur[k]);
             }
+            __syncwarp();
+            // the slot refilled here last held tile j + ID_AHEAD - ID_RING, read before
+            prefetch_ids(j + ID_AHEAD);
             ++issued;
             // let the first tile land before streaming the rest, so it does not queue
             // behind every other tile of the launch
             if (j == 0 && ntiles > 1 && !warp_wait(is_k ? k_full(0) : v_full(0), 0, abort_flag)) break;
-            // slide the lookahead window by one tile
-            const int nxt = __shfl_down_sync(0xffffffffu, ids, 8);
-            ids = lane < 24 ? nxt : load_id(j + 4);
-            __syncwarp();
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");  // no id copy lands after the ring is abandoned
         if (bad_id) s_bad = TV_ERR_BLOCK_TABLE;
         if (*abort_flag && lane == 0) {
             // let copies already in flight land before the CTA retires
@@ -451,15 +482,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer (one thread)
+        // ---------------- S = Q K^T issuer (one thread).  The two MMA streams are issued
+        // from warps on different SM sub-partitions: a thread issuing tcgen05.mma shares
+        // its sub-partition's issue slots with two softmax warps, and one thread issuing
+        // all sixteen MMAs of a tile was slower than the tile's softmax.
         if (ntiles > 0 && lane == 0) {
             bool ok = mbar_wait(q_ready, 0, abort_flag);
             bool issued_any = false;
-            // S = Q K^T of tile j into S buffer j % 2
-            auto issue_qk = [&](int j) {
+            for (int j = 0; ok && j < ntiles; ++j) {
                 const int ks = j % KST, sb = j & 1;
-                if (!mbar_wait(k_full(ks), (j / KST) & 1, abort_flag)) return false;
-                // S buffer j % 2 held P of tile j - 2, whose P V was issued before this call
+                // S buffer j % 2 holds P of tile j - 2 until that tile's P V has finished;
+                // the buffer's barrier cannot run two phases ahead of this wait, because
+                // P V of tile j needs the S tile issued here
+                if (j >= 2) ok = mbar_wait(pv_done(sb), ((j - 2) >> 1) & 1, abort_flag);
+                if (ok) ok = mbar_wait(k_full(ks), (j / KST) & 1, abort_flag);
+                if (!ok) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k) {
@@ -470,10 +507,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 mma_commit(s_full(sb));
                 mma_commit(k_empty(ks));
                 issued_any = true;
-                return true;
-            };
-            // the S tiles run two ahead of P V, so the softmax groups never wait for S
-            for (int j = 0; ok && j < 2 && j < ntiles; ++j) ok = issue_qk(j);
+            }
+            if (issued_any) {
+                // every MMA issued by this thread has finished before TMEM is released
+                mma_commit(drain_qk);
+                const long long c0 = clock64();
+                while (!mbar_try(drain_qk, 0) && clock64() - c0 < WAIT_LIMIT) {
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ---------------- O += P V issuer (one thread)
+        if (ntiles > 0 && lane == 0) {
+            bool ok = true, issued_any = false;
             for (int t = 0; ok && t < ntiles; ++t) {
                 const int vs = t % VST;
                 ok = mbar_wait(v_full(vs), (t / VST) & 1, abort_flag);
@@ -487,16 +534,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                     sdesc(sV(vs) + (x * 4 + k) * 2048u, HALF_BYTES, 1024), IDESC_PV,
                                     (t > 0 || k > 0) ? 1u : 0u);
                     mma_commit(o_done(x));
+                    issued_any = true;
                 }
                 if (!ok) break;
                 mma_commit(v_empty(vs));
-                if (t + 2 < ntiles) ok = issue_qk(t + 2);
+                mma_commit(pv_done(t & 1));
             }
             if (issued_any) {
-                // every MMA issued by this thread has finished before TMEM is released
-                mma_commit(mma_drain);
+                mma_commit(drain_pv);
                 const long long c0 = clock64();
-                while (!mbar_try(mma_drain, 0) && clock64() - c0 < WAIT_LIMIT) {
+                while (!mbar_try(drain_pv, 0) && clock64() - c0 < WAIT_LIMIT) {
                 }
             }
         }
