@@ -46,7 +46,7 @@ def load_peaks():
 
 # the sources each kernel's code and launch configuration come from
 KERNEL_SOURCES = {
-    "attn_tc": ("api.cu", "attn_tc.cu", "kernels.h", "tv_common.cuh"),
+    "attn_tc": ("api.cu", "attn_tc.cu", "kernels.h", "tc_device.cuh", "tv_common.cuh"),
     "attn_simt": ("api.cu", "attn_simt.cu", "kernels.h", "tv_common.cuh"),
     "verify_sample": ("api.cu", "sample.cu", "kernels.h", "tv_common.cuh"),
 }
