@@ -143,7 +143,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
         tc_fence_before();
     }
-    for (int i = tid; i < N; i += TC_THREADS) s_par[i] = a.parent[(size_t)b * N + i];
+    // the prefix length decides the split range and so the first block ids: it is
+    // loaded first, and the tree's parent array only after the id copies are issued
     const int L = a.prefix_lens[b];
     const int total = L + N;
     const bool bad_len = L < 0 || (total + TV_BLOCK - 1) / TV_BLOCK > a.max_blocks;
@@ -168,6 +169,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     };
     if (warp == 0 || warp == 3)
         for (int jt = 0; jt < ID_AHEAD; ++jt) prefetch_ids(jt);
+    for (int i = tid; i < N; i += TC_THREADS) s_par[i] = a.parent[(size_t)b * N + i];
     __syncthreads();
     // a kernel launched after this one with programmatic stream serialisation may
     // start its set-up now; it waits for this grid before reading anything

@@ -208,23 +208,29 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
 // Combine rows [split * R, split * R + R) of one ROWS-row tile from the S
 // partials in the workspace (layout [S][ROWS][RPITCH]: 128 outputs, lse):
 // out = sum_s 2^(lse_s - m) o_s / sum_s 2^(lse_s - m), m = max_s lse_s.
+// Each item is CW columns of one row; with up to 9 splits an item takes 8
+// columns, so every thread issues all its loads in one round.
 template <int ROWS, int THREADS, int S_>
 __device__ __forceinline__ void merge_rows(const AttnArgs& a, const float* part, int split, int tile, int b, int kvh,
                                            int tid) {
     constexpr int R = (ROWS + S_ - 1) / S_;
+    constexpr int CW = S_ <= 9 ? 8 : 4;  // columns per item
+    constexpr int NQ = CW / 4;           // float4 per split and item
+    constexpr int NC = HD / CW;
     const int own = max(0, min(ROWS, (split + 1) * R) - split * R);
-    for (int item = tid; item < own * (HD / 4); item += THREADS) {
-        const int rr = item / (HD / 4), c4 = item % (HD / 4);
+    for (int item = tid; item < own * NC; item += THREADS) {
+        const int rr = item / NC, cc = item % NC;
         const int rt = split * R + rr;
         const int gr = tile * ROWS + rt;
         if (gr >= a.G * a.N) continue;
         float ls[S_];
-        float4 v[S_];
+        float4 v[S_][NQ];
 #pragma unroll
         for (int k = 0; k < S_; ++k) {
             const float* prow = part + ((size_t)k * ROWS + rt) * RPITCH;
             ls[k] = prow[HD];
-            v[k] = reinterpret_cast<const float4*>(prow)[c4];
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) v[k][q] = reinterpret_cast<const float4*>(prow)[cc * NQ + q];
         }
         float mx = -INFINITY;
         bool nan = false;
@@ -234,24 +240,33 @@ __device__ __forceinline__ void merge_rows(const AttnArgs& a, const float* part,
             mx = fmaxf(mx, ls[k]);
         }
         float den = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float acc[CW];
+#pragma unroll
+        for (int e = 0; e < CW; ++e) acc[e] = 0.f;
 #pragma unroll
         for (int k = 0; k < S_; ++k) {
             const float w = ls[k] == -INFINITY ? 0.f : ex2(ls[k] - mx);
             den += w;
-            acc.x = fmaf(w, v[k].x, acc.x);
-            acc.y = fmaf(w, v[k].y, acc.y);
-            acc.z = fmaf(w, v[k].z, acc.z);
-            acc.w = fmaf(w, v[k].w, acc.w);
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                acc[4 * q + 0] = fmaf(w, v[k][q].x, acc[4 * q + 0]);
+                acc[4 * q + 1] = fmaf(w, v[k][q].y, acc[4 * q + 1]);
+                acc[4 * q + 2] = fmaf(w, v[k][q].z, acc[4 * q + 2]);
+                acc[4 * q + 3] = fmaf(w, v[k][q].w, acc[4 * q + 3]);
+            }
         }
         const bool dead = nan || !(den > 0.f);
         const float id = dead ? 0.f : 1.f / den;
         const int node = gr / a.G, head = kvh * a.G + gr % a.G;
-        uint2 ov;
-        ov.x = pack_bf16(dead ? NAN : acc.x * id, dead ? NAN : acc.y * id);
-        ov.y = pack_bf16(dead ? NAN : acc.z * id, dead ? NAN : acc.w * id);
-        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + (((size_t)b * a.N + node) * a.Hq + head) * HD +
-                                  c4 * 4) = ov;
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + (((size_t)b * a.N + node) * a.Hq + head) * HD + cc * CW;
+        uint32_t pk[CW / 2];
+#pragma unroll
+        for (int e = 0; e < CW / 2; ++e)
+            pk[e] = pack_bf16(dead ? NAN : acc[2 * e] * id, dead ? NAN : acc[2 * e + 1] * id);
+        if constexpr (CW == 8)
+            *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        else
+            *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
     }
 }
 
