@@ -113,9 +113,13 @@ __device__ __forceinline__ double warp_sum_d(double v) {
     return v;
 }
 
+// max(0, d) for the residual terms: the sign is read from the high word, because
+// the fp64 max instruction runs at an eighth of the fp64 add / fma rate
+__device__ __forceinline__ double pos_part(double d) { return __double2hiint(d) >= 0 ? d : 0.0; }
+
 // residual mass of one element: p itself while c == 0, else max(0, p - c q)
 __device__ __forceinline__ double resid(float p, float q, double c) {
-    return c == 0.0 ? (double)p : fmax(0.0, fma(-c, (double)q, (double)p));
+    return c == 0.0 ? (double)p : pos_part(fma(-c, (double)q, (double)p));
 }
 
 struct Walker {
@@ -173,30 +177,45 @@ struct Walker {
         const float* q = qs(x);
         const int s0 = min(n, warp * segw), s1 = min(n, s0 + segw);
         double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-        int i = s0 + lane;
-        for (; i + 96 < s1; i += 128) {
-            a0 += resid(p[i], q[i], c);
-            a1 += resid(p[i + 32], q[i + 32], c);
-            a2 += resid(p[i + 64], q[i + 64], c);
-            a3 += resid(p[i + 96], q[i + 96], c);
+        // four consecutive elements per lane and step (16-byte shared loads; segw is a
+        // multiple of 128 and the slices start 16-byte aligned); a lane's last,
+        // incomplete step at the end of the row is done element by element
+        int i = s0 + 4 * lane;
+        if (c == 0.0) {
+            for (; i + 3 < s1; i += 128) {
+                const float4 pv = *reinterpret_cast<const float4*>(p + i);
+                a0 += (double)pv.x;
+                a1 += (double)pv.y;
+                a2 += (double)pv.z;
+                a3 += (double)pv.w;
+            }
+        } else {
+            for (; i + 3 < s1; i += 128) {
+                const float4 pv = *reinterpret_cast<const float4*>(p + i);
+                const float4 qv = *reinterpret_cast<const float4*>(q + i);
+                a0 += pos_part(fma(-c, (double)qv.x, (double)pv.x));
+                a1 += pos_part(fma(-c, (double)qv.y, (double)pv.y));
+                a2 += pos_part(fma(-c, (double)qv.z, (double)pv.z));
+                a3 += pos_part(fma(-c, (double)qv.w, (double)pv.w));
+            }
         }
-        for (; i < s1; i += 32) a0 += resid(p[i], q[i], c);
+        for (int e = i; e < s1 && e < i + 4; ++e) a0 += resid(p[e], q[e], c);
         const double wsum = warp_sum_d((a0 + a1) + (a2 + a3));
         if (lane == 0) sh.warp_part[warp] = wsum;
         __syncthreads();
         const int par = passes & 1;
         const uint32_t use = (uint32_t)(passes >> 1);
         ++passes;
-        if (tid == 0) {
-            double s = 0.0;
-            for (int k = 0; k < nwarps; ++k) s += sh.warp_part[k];
+        if (warp == 0) {
+            // this CTA's partial (a fixed shuffle tree over its warps), sent to every
+            // CTA of the cluster, one lane per receiver
+            const double s = warp_sum_d(lane < nwarps ? sh.warp_part[lane] : 0.0);
             if (C == 1) {
-                sh.peer[par][0] = s;
+                if (lane == 0) sh.peer[par][0] = s;
             } else {
                 const uint32_t bar = smem_u32(&sh.peer_bar[par]);
-                mbar_expect_tx(bar, (uint32_t)(8 * C));
-                const uint32_t slot = smem_u32(&sh.peer[par][rank]);
-                for (int r = 0; r < C; ++r) st_async_f64(mapa(slot, r), s, mapa(bar, r));
+                if (lane == 0) mbar_expect_tx(bar, (uint32_t)(8 * C));
+                if (lane < C) st_async_f64(mapa(smem_u32(&sh.peer[par][rank]), lane), s, mapa(bar, lane));
             }
         }
         if (C == 1) {
@@ -204,9 +223,9 @@ struct Walker {
         } else {
             mbar_wait(smem_u32(&sh.peer_bar[par]), use & 1, &sh.timeout);
         }
-        double total = 0.0;
-        for (int r = 0; r < C; ++r) total += sh.peer[par][r];
-        return total;
+        // every warp adds the C partials with the same shuffle tree, so all CTAs (and
+        // all warps) obtain the same bits and take the same branches
+        return warp_sum_d(lane < C ? sh.peer[par][lane] : 0.0);
     }
 };
 
@@ -237,7 +256,7 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
     Walker w{a, sh, reinterpret_cast<float*>(sample_dyn), b, rank, C, lo, n, tid, lane, warp, nwarps,
-             ((n + nwarps - 1) / nwarps + 31) / 32 * 32, a.vec4 != 0, 0, {0, 0}, {false, false}};
+             ((n + nwarps - 1) / nwarps + 127) / 128 * 128, a.vec4 != 0, 0, {0, 0}, {false, false}};
     // the root's row is needed unless its first child is accepted: start it now
     w.issue_row(0, 0);
 
@@ -314,8 +333,9 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
             const int gn = sh.ch_n;
             for (int k = 0; k < gn; ++k) {
                 const double px = sh.ch_p[k], qx = sh.ch_q[k], r = sh.ch_u[k];
-                const double num = cur_c == 0.0 ? px : fmax(0.0, fma(-cur_c, qx, px));
-                const bool acc = qx > 0.0 ? (r < num / (cur_z * qx)) : (num > 0.0);
+                // r < num / (Z q(x)), compared without the fp64 division
+                const double num = cur_c == 0.0 ? px : pos_part(fma(-cur_c, qx, px));
+                const bool acc = qx > 0.0 ? (r * (cur_z * qx) < num) : (num > 0.0);
                 if (acc) {
                     accepted = sh.ch_node[k];
                     break;
