@@ -367,21 +367,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 m_run = mt;
             }
             const float mu = m_run == -INFINITY ? 0.f : m_run;
+            // exponentials, packed as bf16 pairs (token 2i in the low half of column i) as
+            // they are made, over the first 32 of this group's S columns of the tile,
+            // whose scores were read above
             float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int i = 0; i < HALF_N; ++i) {
-                x[i] = ex2(fmaf(x[i], sl, -mu));
-                s4[i & 3] += x[i];
-            }
-            l_run = l_run * f + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
-            // P as bf16 pairs (token 2i in the low half of column i) over the first 32 of
-            // this group's S columns of the tile, whose scores were read above
             {
                 uint32_t pk[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(x[2 * i], x[2 * i + 1]);
+                for (int i = 0; i < 32; ++i) {
+                    const float e0 = ex2(fmaf(x[2 * i], sl, -mu));
+                    const float e1 = ex2(fmaf(x[2 * i + 1], sl, -mu));
+                    s4[(2 * i) & 3] += e0;
+                    s4[(2 * i + 1) & 3] += e1;
+                    pk[i] = pack_bf16(e0, e1);
+                }
                 tmem_st_x32(tmem + lane_base + sb * TN + X * HALF_N, pk);
             }
+            l_run = l_run * f + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
             if (lim < TN) {
                 // value rows past the split end may hold stale data: clear this group's ones
                 const int tok = X * HALF_N + (r & 63);

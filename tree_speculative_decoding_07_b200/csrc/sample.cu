@@ -249,7 +249,6 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
-    if (C > 1) cg::this_cluster().sync();  // every CTA's barriers exist before any peer pushes to them
     // the kernel may have been launched while the previous one on the stream was still
     // running (programmatic dependent launch): its inputs are read only after that
     // kernel has completed and its memory is visible
@@ -265,7 +264,12 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
         sh.parent[i] = a.parent[(size_t)b * N + i];
         sh.token[i] = a.tokens[(size_t)b * N + i];
     }
-    __syncthreads();
+    // every CTA's barriers must exist before a peer pushes to them (the first pass);
+    // the cluster barrier sits here so the loads above are already in flight
+    if (C > 1)
+        cg::this_cluster().sync();
+    else
+        __syncthreads();
     bool bad_local = false;
     for (int i = tid; i < N; i += blockDim.x) {
         const int p = sh.parent[i];
