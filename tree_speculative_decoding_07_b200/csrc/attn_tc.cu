@@ -449,6 +449,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                          : (bad ? NAN : 0.f);
         }
         tc_fence_before();
+        if (S > 1) {
+            // this split's partial row straight to the workspace: the group's 64
+            // outputs as bf16, and (group A) the row's log-sum-exp
+            const size_t group = ((size_t)b * a.Hkv + kvh) * a.row_tiles + tile;
+            uint8_t* prow = reinterpret_cast<uint8_t*>(a.o_part) + ((group * S + split) * TM + r) * PROW_BYTES;
+            uint4* dst = reinterpret_cast<uint4*>(prow + X * HD);
+#pragma unroll
+            for (int q8 = 0; q8 < 8; ++q8)
+                dst[q8] = make_uint4(pack_bf16(o[q8 * 8 + 0], o[q8 * 8 + 1]), pack_bf16(o[q8 * 8 + 2], o[q8 * 8 + 3]),
+                                     pack_bf16(o[q8 * 8 + 4], o[q8 * 8 + 5]), pack_bf16(o[q8 * 8 + 6], o[q8 * 8 + 7]));
+            if (X == 0) *reinterpret_cast<float*>(prow + 2 * HD) = lse;
+        }
         if (S == 1 && row_ok) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
                                                   (((size_t)b * N + node) * a.Hq + head) * HD + X * 64);
@@ -470,27 +482,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
     }
     if (S > 1) {
-        // ---- merge the KV splits of this row tile.  Each split stages its normalised
-        // partial rows and their log-sum-exp in shared memory, copies them to the
-        // workspace with coalesced stores, counts itself in, and once all S splits
-        // are in combines an equal share of the rows from all S partials.
+        // ---- merge the KV splits of this row tile.  Each split has written its
+        // normalised partial rows (bf16) and their log-sum-exp to the workspace; it
+        // counts itself in, and once all S splits are in combines an equal share of
+        // the rows from all S partials.
         const size_t group = ((size_t)b * a.Hkv + kvh) * a.row_tiles + tile;
-        float* part = a.o_part + group * (size_t)S * TM * RPITCH;  // [S][TM][RPITCH]
-        unsigned* arrive = a.counters + 2 * group;                  // [groups][2]: arrivals, departures
-        float* stage = reinterpret_cast<float*>(base_ptr + SK_OFF); // [TM][RPITCH]; the K ring is idle now
-        if (warp >= 4) {
-            float4* row = reinterpret_cast<float4*>(stage + r * RPITCH + X * 64);
-#pragma unroll
-            for (int q4 = 0; q4 < 16; ++q4) row[q4] = make_float4(o[q4 * 4], o[q4 * 4 + 1], o[q4 * 4 + 2], o[q4 * 4 + 3]);
-            if (X == 0) stage[r * RPITCH + HD] = lse;
-        }
-        __syncthreads();
-        {
-            const float4* src = reinterpret_cast<const float4*>(stage);
-            float4* dst = reinterpret_cast<float4*>(part + (size_t)split * TM * RPITCH);
-            for (int i = tid; i < TM * RPITCH / 4; i += TC_THREADS) dst[i] = src[i];
-        }
-        __syncthreads();
+        const uint8_t* part = reinterpret_cast<const uint8_t*>(a.o_part) + group * (size_t)S * TM * PROW_BYTES;
+        unsigned* arrive = a.counters + 2 * group;  // [groups][2]: arrivals, departures
         __shared__ int s_all_in;
         if (tid == 0) {
             count_in(arrive);
@@ -575,7 +573,7 @@ int tc_resident_ctas() {
 int tc_rows_per_tile() { return TM; }
 int tc_max_splits() { return MAX_SPLITS; }
 size_t tc_counter_offset(int64_t groups, int splits) {
-    return (size_t)groups * splits * TM * RPITCH * sizeof(float);
+    return (size_t)groups * splits * TM * PROW_BYTES;
 }
 size_t tc_workspace_bytes(int64_t groups, int splits) {
     if (splits <= 1) return 0;

@@ -15,7 +15,8 @@ struct AttnArgs {
     const int32_t* parent;
     void* out;
     float* o_part;      // CUDA-core path: [splits][B][N][Hq][D] fp32 partial outputs (normalised);
-                        // tensor-core path: [groups][splits][128][132] partial rows + lse
+                        // tensor-core path: [groups][splits][128] partial rows of 272 bytes
+                        // (128 bf16 outputs, fp32 log-sum-exp, padding)
     float* lse_part;    // [splits][B][N][Hq] log2-domain log-sum-exp of each partial
     unsigned* counters; // tensor-core path: [groups][2] arrival / departure counts, zero between calls
     int32_t* status;

@@ -21,7 +21,9 @@ constexpr int ID_RING = 8;       // tiles of block ids held per producer
 constexpr int ID_AHEAD = 6;      // tiles between an id copy's issue and its use
 constexpr uint32_t TILE_BYTES = 32768;     // one K or V tile: 2 halves x 128 rows x 128 B
 constexpr uint32_t HALF_BYTES = 16384;
-constexpr int RPITCH = HD + 4;             // floats per workspace partial row: 128 outputs, lse, padding
+// one split's partial row in the workspace: 128 normalised outputs as bf16, the
+// row's log-sum-exp as fp32 at byte 256, padding to a 16-byte multiple
+constexpr int PROW_BYTES = 272;
 constexpr long long WAIT_LIMIT = 1ll << 32;  // clock cycles (~2 s)
 
 // instruction descriptor, kind::f16: D fp32, A/B bf16, A K-major,
@@ -206,17 +208,14 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 // Combine rows [split * R, split * R + R) of one ROWS-row tile from the S
-// partials in the workspace (layout [S][ROWS][RPITCH]: 128 outputs, lse):
+// partials in the workspace (layout [S][ROWS] rows of PROW_BYTES):
 // out = sum_s 2^(lse_s - m) o_s / sum_s 2^(lse_s - m), m = max_s lse_s.
-// Each item is CW columns of one row; with up to 9 splits an item takes 8
-// columns, so every thread issues all its loads in one round.
+// Each item is 8 columns of one row, so a thread issues all its loads at once.
 template <int ROWS, int THREADS, int S_>
-__device__ __forceinline__ void merge_rows(const AttnArgs& a, const float* part, int split, int tile, int b, int kvh,
+__device__ __forceinline__ void merge_rows(const AttnArgs& a, const uint8_t* part, int split, int tile, int b, int kvh,
                                            int tid) {
     constexpr int R = (ROWS + S_ - 1) / S_;
-    constexpr int CW = S_ <= 9 ? 8 : 4;  // columns per item
-    constexpr int NQ = CW / 4;           // float4 per split and item
-    constexpr int NC = HD / CW;
+    constexpr int NC = HD / 8;
     const int own = max(0, min(ROWS, (split + 1) * R) - split * R);
     for (int item = tid; item < own * NC; item += THREADS) {
         const int rr = item / NC, cc = item % NC;
@@ -224,13 +223,12 @@ __device__ __forceinline__ void merge_rows(const AttnArgs& a, const float* part,
         const int gr = tile * ROWS + rt;
         if (gr >= a.G * a.N) continue;
         float ls[S_];
-        float4 v[S_][NQ];
+        uint4 v[S_];
 #pragma unroll
         for (int k = 0; k < S_; ++k) {
-            const float* prow = part + ((size_t)k * ROWS + rt) * RPITCH;
-            ls[k] = prow[HD];
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) v[k][q] = reinterpret_cast<const float4*>(prow)[cc * NQ + q];
+            const uint8_t* prow = part + ((size_t)k * ROWS + rt) * PROW_BYTES;
+            ls[k] = *reinterpret_cast<const float*>(prow + 2 * HD);
+            v[k] = reinterpret_cast<const uint4*>(prow)[cc];
         }
         float mx = -INFINITY;
         bool nan = false;
@@ -240,33 +238,28 @@ __device__ __forceinline__ void merge_rows(const AttnArgs& a, const float* part,
             mx = fmaxf(mx, ls[k]);
         }
         float den = 0.f;
-        float acc[CW];
+        float acc[8];
 #pragma unroll
-        for (int e = 0; e < CW; ++e) acc[e] = 0.f;
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
         for (int k = 0; k < S_; ++k) {
             const float w = ls[k] == -INFINITY ? 0.f : ex2(ls[k] - mx);
             den += w;
+            const uint32_t wd[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
 #pragma unroll
-            for (int q = 0; q < NQ; ++q) {
-                acc[4 * q + 0] = fmaf(w, v[k][q].x, acc[4 * q + 0]);
-                acc[4 * q + 1] = fmaf(w, v[k][q].y, acc[4 * q + 1]);
-                acc[4 * q + 2] = fmaf(w, v[k][q].z, acc[4 * q + 2]);
-                acc[4 * q + 3] = fmaf(w, v[k][q].w, acc[4 * q + 3]);
+            for (int e = 0; e < 4; ++e) {
+                acc[2 * e] = fmaf(w, __uint_as_float(wd[e] << 16), acc[2 * e]);
+                acc[2 * e + 1] = fmaf(w, __uint_as_float(wd[e] & 0xFFFF0000u), acc[2 * e + 1]);
             }
         }
         const bool dead = nan || !(den > 0.f);
         const float id = dead ? 0.f : 1.f / den;
         const int node = gr / a.G, head = kvh * a.G + gr % a.G;
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + (((size_t)b * a.N + node) * a.Hq + head) * HD + cc * CW;
-        uint32_t pk[CW / 2];
+        uint32_t pk[4];
 #pragma unroll
-        for (int e = 0; e < CW / 2; ++e)
-            pk[e] = pack_bf16(dead ? NAN : acc[2 * e] * id, dead ? NAN : acc[2 * e + 1] * id);
-        if constexpr (CW == 8)
-            *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        else
-            *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+        for (int e = 0; e < 4; ++e) pk[e] = pack_bf16(dead ? NAN : acc[2 * e] * id, dead ? NAN : acc[2 * e + 1] * id);
+        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + (((size_t)b * a.N + node) * a.Hq + head) * HD +
+                                  cc * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
 }
 
