@@ -176,6 +176,17 @@ def job_throughput(world: int, nodes_per_step: int, steps: int, max_ms: float) -
 
 # ------------------------------------------------------------------ our arm
 
+def workload_config(name: str, wl, world: int) -> dict:
+    """The workload both arms of the bench report (same dict for each)."""
+    N = wl.num_nodes
+    return {"workload": f"{name}: batch {wl.batch}, prefix {int(wl.prefix_lens[0])}, "
+                        f"Hq {wl.num_q_heads}/Hkv {wl.num_kv_heads}, D {wl.head_dim}, {wl.dtype}, "
+                        f"{N}-node tree, vocab {wl.vocab}",
+            "global_batch": world * wl.batch, "tree_nodes": N, "seq_len": int(wl.prefix_lens.max()) + N,
+            "parallelism": f"replicas x{world} (independent sequences per GPU)",
+            "l2": f"flushed before every step ({L2_FLUSH_BYTES >> 20} MB write, outside the step events)"}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -344,12 +355,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": wl.dtype,
         "data": "synthetic (Philox4x32-10 seeded; no dataset)",
-        "config": {"workload": f"{args.workload}: batch {wl.batch}, prefix {int(wl.prefix_lens[0])}, "
-                               f"Hq {wl.num_q_heads}/Hkv {wl.num_kv_heads}, D {wl.head_dim}, {wl.dtype}, "
-                               f"{N}-node tree, vocab {wl.vocab}",
-                   "global_batch": world * B, "tree_nodes": N, "seq_len": int(wl.prefix_lens.max()) + N,
-                   "parallelism": f"replicas x{world} (independent sequences per GPU)",
-                   "l2": f"flushed before every step ({L2_FLUSH_BYTES >> 20} MB write, outside the step events)"},
+        "config": workload_config(args.workload, wl, world),
         "attention_us": attn_avg_s * 1e6,
         "sample_us": (sum(samp_ms) / K) * 1e3,
         "per_kernel_timing": "each kernel replayed alone from its own graph, L2 flushed before each launch",
@@ -437,7 +443,7 @@ def run_reference(args, rank, world):
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "nodes/s", "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (Philox4x32-10 seeded; no dataset)",
-            "config": {"workload": args.workload}, "cpu_baseline": {"value": value, "unit": "nodes/s",
+            "config": workload_config(args.workload, wl, world), "cpu_baseline": {"value": value, "unit": "nodes/s",
                                                                   "cores": cores, "kind": "oracle",
                                                                   "sample": sample},
             "e2e": {"value": value, "unit": "nodes/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
