@@ -51,6 +51,7 @@ def _bind(path):
     L.or_tree_mask.argtypes = [i32, P, P]
     L.or_tree_attention.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, dbl, i64, P, P]
     L.or_verify_sample.argtypes = [i32, i32, i64, P, P, P, P, P, dbl, P, P, P, P, P]
+    L.or_commit_path.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P]
     L.or_set_threads.argtypes = [ctypes.c_int]
     L.or_max_threads.restype = ctypes.c_int
     return L
@@ -152,3 +153,24 @@ def verify_sample(p, q, tree_tokens, parent_idx, uniforms, eps: float = 1e-6, L=
     rc = (L or lib()).or_verify_sample(B, N, V, _p(pp), _p(qq), _p(tt), _p(pa), _p(uu), float(eps),
                                        _p(path), _p(alen), _p(bonus), _p(near), _p(rows))
     return {"accepted_path": path, "accepted_len": alen, "bonus_token": bonus, "near": near, "rows": rows, "rc": rc}
+
+
+def commit_path(k_cache, v_cache, block_table, prefix_lens, accepted_path, accepted_len, L=None):
+    """Move each sequence's accepted path into the cached prefix, in place on
+    copies of the caches (oracle.c or_commit_path).  Caches [nb][16][Hkv][D]
+    of any dtype (rows are moved as bytes).  Returns (k, v, new_prefix_lens,
+    status)."""
+    L = L or lib()
+    k = np.ascontiguousarray(k_cache).copy()
+    v = np.ascontiguousarray(v_cache).copy()
+    bt = np.ascontiguousarray(block_table, np.int32)
+    pl = np.ascontiguousarray(prefix_lens, np.int32)
+    path = np.ascontiguousarray(accepted_path, np.int32)
+    ln = np.ascontiguousarray(accepted_len, np.int32)
+    nb, bs, hkv, d = k.shape
+    assert bs == 16 and v.shape == k.shape
+    B, N = path.shape
+    new_pl = np.zeros(B, np.int32)
+    st = L.or_commit_path(B, N, hkv, d, bt.shape[1], nb, k.dtype.itemsize, _p(k), _p(v), _p(bt), _p(pl), _p(path),
+                          _p(ln), _p(new_pl))
+    return k, v, new_pl, int(st)

@@ -279,3 +279,77 @@ int or_verify_sample(int32_t B, int32_t N, int64_t V, const float *p, const floa
     }
     return err;
 }
+
+/*
+ * or_commit_path -- the step after verification: the accepted path joins the
+ * cached prefix and every other tree entry is released.
+ *
+ * Sources: blog "Speculative decoding x tree attention", section "KV cache
+ * management and prefix sharing" (rejected tokens' KV must be freed or rolled
+ * back at once; paged engines do it through block-table operations), and
+ * glossary "Tree-based speculative decoding", section "KV cache management
+ * challenges" (each tree node has a KV entry; after verification every entry
+ * off the accepted path is pruned; page-based management avoids fragmentation).
+ *
+ * Readings (listed in the design notes): tree node j of sequence b sits at
+ * logical position L_b + j; the root (node 0) stays at L_b; accepted node
+ * path[k] (k = 0 .. len-1) moves to position L_b + 1 + k, for every KV head and
+ * both K and V; the new prefix length is L_b + 1 + len.  Positions at or past
+ * the new length are free (the caller's allocator may reclaim whole blocks past
+ * it); nothing else in the cache changes.  A sequence with len < 0 (the walk
+ * flagged its tree) keeps its length and cache.  A path that is not strictly
+ * increasing inside [1, N), a length over N - 1, or a prefix / block id out of
+ * range leaves the sequence untouched and returns an error code.
+ *
+ * Layout: cache [num_blocks][16][Hkv][D] elements of elem_size bytes; logical
+ * position t of sequence b lives in block bt[b][t / 16], slot t % 16.
+ * Rows are moved as bytes, so any element type works.
+ */
+int or_commit_path(int32_t B, int32_t N, int32_t Hkv, int32_t D, int32_t max_blocks, int32_t num_blocks,
+                   int32_t elem_size, void *k_cache, void *v_cache, const int32_t *block_table,
+                   const int32_t *prefix_lens, const int32_t *path, const int32_t *len, int32_t *new_prefix_lens) {
+    const int64_t row = (int64_t)D * elem_size;  /* bytes of one (position, head) row */
+    int err = OR_OK;
+    for (int32_t b = 0; b < B; ++b) {
+        const int32_t L = prefix_lens[b];
+        const int32_t n = len[b];
+        new_prefix_lens[b] = L;
+        if (n < 0) continue;
+        if (L < 0 || n > N - 1 || (int64_t)L + N > (int64_t)max_blocks * 16) { err = OR_ERR_ARG; continue; }
+        const int32_t *pb = path + (int64_t)b * N;
+        int ok = 1;
+        for (int32_t k = 0; k < n; ++k) {
+            const int32_t prev = k == 0 ? 0 : pb[k - 1];
+            if (pb[k] <= prev || pb[k] >= N) ok = 0;
+        }
+        if (!ok) { err = OR_ERR_TREE; continue; }
+        const int32_t *bt = block_table + (int64_t)b * max_blocks;
+        for (int32_t t = L; t < L + N; ++t) {
+            const int32_t id = bt[t / 16];
+            if (id < 0 || id >= num_blocks) ok = 0;
+        }
+        if (!ok) { err = OR_ERR_BLOCK; continue; }
+        /* read every source row first, then write: a destination may be another row's source */
+        const int64_t per_pos = (int64_t)Hkv * row;
+        unsigned char *tmp = (unsigned char *)malloc((size_t)(2 * (int64_t)n * per_pos + 1));
+        for (int c = 0; c < 2; ++c) {
+            unsigned char *cache = (unsigned char *)(c == 0 ? k_cache : v_cache);
+            for (int32_t k = 0; k < n; ++k) {
+                const int32_t t = L + pb[k];
+                memcpy(tmp + ((int64_t)c * n + k) * per_pos,
+                       cache + ((int64_t)bt[t / 16] * 16 + t % 16) * per_pos, (size_t)per_pos);
+            }
+        }
+        for (int c = 0; c < 2; ++c) {
+            unsigned char *cache = (unsigned char *)(c == 0 ? k_cache : v_cache);
+            for (int32_t k = 0; k < n; ++k) {
+                const int32_t t = L + 1 + k;
+                memcpy(cache + ((int64_t)bt[t / 16] * 16 + t % 16) * per_pos,
+                       tmp + ((int64_t)c * n + k) * per_pos, (size_t)per_pos);
+            }
+        }
+        free(tmp);
+        new_prefix_lens[b] = L + 1 + n;
+    }
+    return err;
+}

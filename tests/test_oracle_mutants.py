@@ -16,6 +16,7 @@ SRC = os.path.join(ROOT, "oracle", "oracle.c")
 
 ATTN = ["tests/test_oracle_mask.py", "tests/test_oracle_attention.py"]
 SAMP = ["tests/test_oracle_sampler.py"]
+COMMIT = ["tests/test_oracle_commit.py"]
 
 MUTANTS = [
     # (name, original text, planted text, pin files)
@@ -35,6 +36,11 @@ MUTANTS = [
      "(void)pc;", SAMP),
     ("siblings_descending", "for (int32_t c = u + 1; c < N; ++c) {", "for (int32_t c = N - 1; c > u; --c) {", SAMP),
     ("cdf_non_strict", "if (run > target) { k = x; break; }", "if (run >= target) { k = x; break; }", SAMP),
+    ("commit_dest_off_by_one", "const int32_t t = L + 1 + k;", "const int32_t t = L + k;", COMMIT),
+    ("commit_length_without_root", "new_prefix_lens[b] = L + 1 + n;", "new_prefix_lens[b] = L + n;", COMMIT),
+    ("commit_path_reversed", "const int32_t t = L + pb[k];", "const int32_t t = L + pb[n - 1 - k];", COMMIT),
+    ("commit_accepts_non_increasing", "if (pb[k] <= prev || pb[k] >= N) ok = 0;", "if (pb[k] >= N) ok = 0;",
+     COMMIT),
 ]
 
 
