@@ -188,6 +188,57 @@ def workload_config(name: str, wl, world: int) -> dict:
             "l2": f"flushed before every step ({L2_FLUSH_BYTES >> 20} MB write, outside the step events)"}
 
 
+def deepest_paths(parent_idx: np.ndarray):
+    """Each tree's deepest root-to-leaf path (root excluded), as a walk that
+    accepts every node on it would return it."""
+    B, N = parent_idx.shape
+    path = np.full((B, N), -1, np.int32)
+    plen = np.zeros(B, np.int32)
+    for b in range(B):
+        depth = np.zeros(N, np.int64)
+        for i in range(1, N):
+            depth[i] = depth[parent_idx[b, i]] + 1
+        node, nodes = int(np.argmax(depth)), []
+        while node > 0:
+            nodes.append(node)
+            node = int(parent_idx[b, node])
+        nodes.reverse()
+        path[b, :len(nodes)] = nodes
+        plen[b] = len(nodes)
+    return path, plen
+
+
+def time_commit(tv, wl, d, flush, stream, W, K):
+    """tv_commit_path (the step after verification) on copies of the caches,
+    every tree's deepest path accepted; CUDA events, L2 flushed per call."""
+    import torch
+    path, plen = deepest_paths(wl.parent_idx)
+    kc, vc = d["k"].clone(), d["v"].clone()
+    dpath = torch.from_numpy(path).cuda()
+    dlen = torch.from_numpy(plen).cuda()
+    new_pl = torch.empty_like(d["prefix_lens"])
+    call = lambda: tv.commit_path(kc, vc, d["block_table"], d["prefix_lens"], dpath, dlen, new_pl, stream=stream)
+    for _ in range(W):
+        flush.zero_()
+        call()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    us = float(np.mean([e0.elapsed_time(e1) for e0, e1 in evs])) * 1e3
+    moved = int(sum(sum(1 for k in range(plen[b]) if path[b, k] != k + 1) for b in range(wl.batch)))
+    row_bytes = wl.head_dim * (2 if wl.dtype == "bf16" else 4)
+    nbytes = moved * wl.num_kv_heads * row_bytes * 2 * 2  # K and V, read and written
+    del kc, vc
+    return {"us": us, "accepted_nodes": int(plen.sum()), "moved_rows": moved, "bytes": nbytes,
+            "achieved_gbs": nbytes / (us * 1e-6) / 1e9 if us > 0 else None,
+            "note": "tv_commit_path, the step after verification (not part of the step timed above): every tree's "
+                    "deepest root-to-leaf path accepted; mean over calls, L2 flushed before each"}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -290,6 +341,7 @@ def run_ours(args, rank, world, local_rank):
 
     attn_ms = kernel_ms(g_attn)
     samp_ms = kernel_ms(g_samp)
+    commit = time_commit(tv, wl, d, flush, stream, W, min(K, 200))
     total_ms = float(sum(step_ms))
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())}")
@@ -371,6 +423,7 @@ def run_ours(args, rank, world, local_rank):
                           "sampler_bytes_literal": 2 * 4 * B * N * wl.vocab,
                           "note": "sampler bytes: rows the walk reads (algorithmic); literal = all of p and q"},
         "median_us_per_step": float(np.median(step_ms)) * 1e3,
+        "commit": commit,
         "e2e": {"value": e2e_value, "unit": "nodes/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": K2},
         "gpu_launches": K * (aplan.launches + splan.launches),

@@ -201,6 +201,46 @@ TV_API tv_status tv_verify_sample(const tv_sample_desc *desc, const float *p, co
                            int32_t *dev_status, void *stream);
 
 /* Static string for a status code. */
+/*
+ * Commit the accepted path into the KV cache: the step after verification.
+ * Blog "Speculative decoding x tree attention", section "KV cache management and
+ * prefix sharing", and glossary "Tree-based speculative decoding", section "KV
+ * cache management challenges": once the tree is verified, every tree entry off
+ * the accepted path is dropped, which paged caches do through block-table
+ * operations rather than by compacting memory.
+ *
+ * For each sequence b, tree node j sits at logical position prefix_lens[b] + j
+ * (the layout tv_tree_attention reads).  With n = accepted_len[b] >= 0 and the
+ * node indices accepted_path[b][0 .. n) (root excluded, strictly increasing, as
+ * tv_verify_sample writes them), the K and V rows of node accepted_path[b][k]
+ * move to position prefix_lens[b] + 1 + k for every KV head; the root stays at
+ * prefix_lens[b]; new_prefix_lens[b] = prefix_lens[b] + 1 + n.  Positions from
+ * the new length on hold nothing live: blocks wholly past it may be returned
+ * to the caller's allocator (the block table is not changed).  accepted_len[b]
+ * < 0 (a sequence the walk flagged) leaves the sequence unchanged.
+ *
+ * Arguments: desc as for tv_tree_attention (batch, num_nodes, num_kv_heads,
+ * head_dim, block_size 16, max_blocks_per_seq, num_blocks and dtype are used;
+ * num_q_heads and softmax_scale are only validated).  paged_k / paged_v: device
+ * caches [num_blocks][16][Hkv][D], 16-byte aligned, updated in place; the
+ * blocks holding a sequence's tree span must belong to that sequence alone.
+ * block_table [B][max_blocks_per_seq], prefix_lens [B], accepted_path [B][N],
+ * accepted_len [B]: device int32, read.  new_prefix_lens [B]: device int32,
+ * written; must not be prefix_lens (it is read while written).  dev_status: a
+ * device int32 or NULL.  One launch on `stream`; no workspace; nothing is
+ * allocated.
+ * Errors: a bad descriptor, a null or misaligned pointer, or new_prefix_lens ==
+ * prefix_lens return before launching.  A path that is not strictly increasing
+ * inside [1, N), a length over N - 1, a prefix too long for the table, or a
+ * block id out of range in the tree's span leaves that sequence unchanged
+ * (new length = old) and writes TV_ERR_TREE, TV_ERR_INVALID_ARG or
+ * TV_ERR_BLOCK_TABLE to *dev_status.
+ */
+TV_API tv_status tv_commit_path(const tv_attn_desc *desc, void *paged_k, void *paged_v,
+                                const int32_t *block_table, const int32_t *prefix_lens,
+                                const int32_t *accepted_path, const int32_t *accepted_len,
+                                int32_t *new_prefix_lens, int32_t *dev_status, void *stream);
+
 TV_API const char *tv_status_string(int32_t status);
 
 /* Library version: major * 10000 + minor * 100 + patch. */

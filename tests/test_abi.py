@@ -103,3 +103,16 @@ def test_sampler_plan_covers_vocab():
         assert 32 <= p.threads <= 512 and p.threads % 32 == 0
         assert p.smem_bytes == 16 * p.slice
     assert tv.tv_verify_sample_workspace_size(tv.TvSampleDesc(1, 64, 1000)) == 0
+
+
+def test_commit_rejects_bad_arguments_before_launch():
+    d = _desc(num_nodes=8, num_q_heads=4, num_kv_heads=2, head_dim=64, max_blocks_per_seq=4, num_blocks=8)
+    a = 256  # a non-null, 16-byte aligned dummy address: nothing is launched on these paths
+    assert tv.tv_commit_path(d, None, a, a, a, a, a, a + 64, stream=0) == tv.TV_ERR_INVALID_ARG
+    assert tv.tv_commit_path(d, a, a, a, a, a, a, None, stream=0) == tv.TV_ERR_INVALID_ARG
+    # the new lengths may not overwrite the lengths still being read
+    assert tv.tv_commit_path(d, a, a, a, 512, a, a, 512, stream=0) == tv.TV_ERR_INVALID_ARG
+    # rows move as 16-byte pieces
+    assert tv.tv_commit_path(d, a + 8, a, a, a, a, a, a + 64, stream=0) == tv.TV_ERR_INVALID_ARG
+    bad = _desc(head_dim=96)
+    assert tv.tv_commit_path(bad, a, a, a, a, a, a, a + 64, stream=0) == tv.TV_ERR_UNSUPPORTED

@@ -73,11 +73,12 @@ def lib() -> ctypes.CDLL:
         L.tv_verify_sample_workspace_size.argtypes = [ctypes.POINTER(TvSampleDesc)]
         L.tv_verify_sample_workspace_size.restype = sz
         L.tv_verify_sample.argtypes = [ctypes.POINTER(TvSampleDesc), P, P, P, P, P, P, P, P, P, sz, P, P]
+        L.tv_commit_path.argtypes = [ctypes.POINTER(TvAttnDesc), P, P, P, P, P, P, P, P, P]
         L.tv_status_string.argtypes = [ctypes.c_int32]
         L.tv_status_string.restype = ctypes.c_char_p
         L.tv_version.restype = ctypes.c_int32
         for name in ("tv_tree_attention_plan", "tv_tree_attention", "tv_tree_attention_static",
-                     "tv_verify_sample_plan", "tv_verify_sample"):
+                     "tv_verify_sample_plan", "tv_verify_sample", "tv_commit_path"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -159,6 +160,13 @@ def tv_verify_sample(desc, p, q, tree_tokens, parent_idx, uniforms, accepted_pat
                                       _ptr(workspace), int(workspace_bytes), _ptr(dev_status), _stream(stream)))
 
 
+def tv_commit_path(desc, paged_k, paged_v, block_table, prefix_lens, accepted_path, accepted_len, new_prefix_lens,
+                   dev_status=None, stream=None) -> int:
+    return int(lib().tv_commit_path(ctypes.byref(desc), _ptr(paged_k), _ptr(paged_v), _ptr(block_table),
+                                    _ptr(prefix_lens), _ptr(accepted_path), _ptr(accepted_len),
+                                    _ptr(new_prefix_lens), _ptr(dev_status), _stream(stream)))
+
+
 # ------------------------------------------------------------ torch conveniences
 
 def attn_desc(q, k_cache, block_table, softmax_scale: float = 0.0) -> TvAttnDesc:
@@ -225,3 +233,28 @@ def verify_sample(p, q, tree_tokens, parent_idx, uniforms, accepted_path=None, a
     if s != TV_OK:
         raise TreeVerifyError(s, "tv_verify_sample")
     return accepted_path, accepted_len, bonus_token
+
+
+def commit_path(k_cache, v_cache, block_table, prefix_lens, accepted_path, accepted_len, new_prefix_lens=None,
+                dev_status=None, stream=None):
+    """Run tv_commit_path on the caches in place; returns new_prefix_lens."""
+    import torch
+    _check_cuda(k_cache, v_cache, block_table, prefix_lens, accepted_path, accepted_len, new_prefix_lens, dev_status)
+    for t in (block_table, prefix_lens, accepted_path, accepted_len):
+        if t.dtype != torch.int32:
+            raise TypeError("block_table, prefix_lens, accepted_path and accepted_len must be int32")
+    if v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype:
+        raise TypeError("k_cache and v_cache must match")
+    nb, bs, hkv, d = k_cache.shape
+    B, N = accepted_path.shape
+    dt = {torch.bfloat16: TV_BF16, torch.float32: TV_F32}.get(k_cache.dtype)
+    if dt is None:
+        raise TypeError(f"unsupported dtype {k_cache.dtype}")
+    desc = TvAttnDesc(B, N, hkv, hkv, d, bs, block_table.shape[1], nb, dt, 0.0)
+    if new_prefix_lens is None:
+        new_prefix_lens = torch.empty_like(prefix_lens)
+    s = tv_commit_path(desc, k_cache, v_cache, block_table, prefix_lens, accepted_path, accepted_len,
+                       new_prefix_lens, dev_status, stream)
+    if s != TV_OK:
+        raise TreeVerifyError(s, "tv_commit_path")
+    return new_prefix_lens

@@ -198,6 +198,26 @@ size_t tv_verify_sample_workspace_size(const tv_sample_desc* desc) {
     return 0;
 }
 
+tv_status tv_commit_path(const tv_attn_desc* desc, void* paged_k, void* paged_v, const int32_t* block_table,
+                         const int32_t* prefix_lens, const int32_t* accepted_path, const int32_t* accepted_len,
+                         int32_t* new_prefix_lens, int32_t* dev_status, void* stream) {
+    tv_status s = check_attn_desc(desc);
+    if (s != TV_OK) return s;
+    if (!paged_k || !paged_v || !block_table || !prefix_lens || !accepted_path || !accepted_len || !new_prefix_lens)
+        return TV_ERR_INVALID_ARG;
+    // other CTAs still read a sequence's prefix length while its new length is written
+    if (static_cast<const void*>(new_prefix_lens) == static_cast<const void*>(prefix_lens)) return TV_ERR_INVALID_ARG;
+    // rows move as 16-byte pieces
+    if ((reinterpret_cast<uintptr_t>(paged_k) | reinterpret_cast<uintptr_t>(paged_v)) & 15) return TV_ERR_INVALID_ARG;
+    tv::CommitArgs a = {};
+    a.k = paged_k; a.v = paged_v; a.block_table = block_table; a.prefix_lens = prefix_lens;
+    a.path = accepted_path; a.len = accepted_len; a.new_prefix_lens = new_prefix_lens; a.status = dev_status;
+    a.B = desc->batch; a.N = desc->num_nodes; a.Hkv = desc->num_kv_heads;
+    a.row_bytes = desc->head_dim * (desc->dtype == TV_BF16 ? 2 : 4);
+    a.max_blocks = desc->max_blocks_per_seq; a.num_blocks = desc->num_blocks;
+    return tv::launch_commit(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? TV_OK : TV_ERR_CUDA;
+}
+
 tv_status tv_verify_sample(const tv_sample_desc* desc, const float* p, const float* q, const int32_t* tree_tokens,
                            const int32_t* parent_idx, const float* uniforms, int32_t* accepted_path,
                            int32_t* accepted_len, int32_t* bonus_token, void* workspace, size_t workspace_bytes,

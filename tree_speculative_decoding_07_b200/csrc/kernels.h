@@ -52,6 +52,21 @@ struct SampleArgs {
 };
 
 cudaError_t launch_verify_sample(const SampleArgs& a, cudaStream_t st, int* launches);
+
+// KV commit of the accepted path (one launch).
+struct CommitArgs {
+    void* k;
+    void* v;
+    const int32_t* block_table;
+    const int32_t* prefix_lens;
+    const int32_t* path;   // [B][N] accepted node indices, root excluded
+    const int32_t* len;    // [B] accepted lengths (< 0: flagged, no commit)
+    int32_t* new_prefix_lens;
+    int32_t* status;
+    int B, N, Hkv, row_bytes, max_blocks, num_blocks;
+};
+cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st);
+size_t commit_smem_bytes(int N, int row_bytes);
 int sample_max_cluster();
 
 }  // namespace tv
