@@ -174,3 +174,21 @@ def commit_path(k_cache, v_cache, block_table, prefix_lens, accepted_path, accep
     st = L.or_commit_path(B, N, hkv, d, bt.shape[1], nb, k.dtype.itemsize, _p(k), _p(v), _p(bt), _p(pl), _p(path),
                           _p(ln), _p(new_pl))
     return k, v, new_pl, int(st)
+
+
+def softmax_rows(logits) -> np.ndarray:
+    """Plain softmax over the last axis in fp64 (max-shifted), rounded to fp32:
+    the distributions a verifier that takes logits works from."""
+    x = np.asarray(logits, dtype=np.float64)
+    e = np.exp(x - x.max(axis=-1, keepdims=True))
+    return (e / e.sum(axis=-1, keepdims=True)).astype(np.float32)
+
+
+def verify_sample_logits(target_logits, draft_logits, tree_tokens, parent_idx, uniforms, eps: float = 1e-6,
+                         L=None):
+    """The acceptance walk on p = softmax(target_logits), q =
+    softmax(draft_logits) (row-wise, temperature 1): the fused-logits form of
+    the step (the glossary's and the blog's p and q are the two models' output
+    distributions).  Same outputs as verify_sample."""
+    return verify_sample(softmax_rows(target_logits), softmax_rows(draft_logits), tree_tokens, parent_idx, uniforms,
+                         eps=eps, L=L)
