@@ -79,49 +79,99 @@ def ncu_traffic(kernel_key: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """SM clock and throttle-reason samples during the timed region, read
+    through NVML (a polling thread every few ms, plus sample_now(), which the
+    timing loop calls while the GPU still works through the queued steps, so a
+    region of a few ms still gets samples).  Falls back to nvidia-smi."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    BITS = (0x8, 0x40, 0x20, 0x4)  # NVML clocks-event reason bits, in NAMES order
 
     def __init__(self, index: int):
         self.index = index
+        self.handle = None
+        self.nvml = None
+        self.samples = []   # (sm_mhz, reason mask)
+        self.smax = None
+        self.thread = None
+        self.stop_flag = None
         self.proc = None
 
-    def start(self):
+    def _open(self):
+        import pynvml
+        pynvml.nvmlInit()
+        h = None
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.index).uuid)
+            h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
         except Exception:
-            self.proc = None
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+        self.nvml, self.handle = pynvml, h
+        self.smax = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+
+    def sample_now(self):
+        if self.handle is None:
+            return
+        n = self.nvml
+        try:
+            self.samples.append((float(n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)),
+                                 int(n.nvmlDeviceGetCurrentClocksEventReasons(self.handle))))
+        except Exception:
+            pass
+
+    def start(self):
+        import threading
+        try:
+            self._open()
+        except Exception:
+            self.handle = None
+        if self.handle is None:
+            try:
+                fields = ("index,clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                          "clocks_event_reasons.sw_power_cap")
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", str(self.index), f"--query-gpu={fields}", "--format=csv,noheader,nounits",
+                     "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except Exception:
+                self.proc = None
+            return
+        self.stop_flag = threading.Event()
+
+        def poll():
+            while not self.stop_flag.is_set():
+                self.sample_now()
+                self.stop_flag.wait(0.002)
+
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except Exception:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, smax, reasons = [], None, set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for line in out.strip().splitlines():
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join()
+        elif self.proc is not None:
+            self.proc.terminate()
             try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            for line in out.strip().splitlines():
+                parts = [x.strip() for x in line.split(",")]
+                try:
+                    mask = sum(b for b, v in zip(self.BITS, parts[3:7]) if v.lower().startswith("active"))
+                    self.samples.append((float(parts[1]), mask))
+                    self.smax = float(parts[2])
+                except (ValueError, IndexError):
+                    continue
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock readout unavailable"], "samples": 0}
+        reasons = sorted({n for _, m in self.samples for n, b in zip(self.NAMES, self.BITS) if m & b})
+        sm = [c for c, _ in self.samples]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.smax, "reasons": reasons,
+                "samples": len(sm), "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
 # ------------------------------------------------------------------ inputs
@@ -147,13 +197,32 @@ def attention_bytes(wl) -> int:
     return kv + qo
 
 
-def sampler_bytes(wl, h) -> int:
-    """Algorithmic bytes of the acceptance walk: 8 bytes (p and q) per tested
-    child plus both rows of every node whose row the walk reads in full
-    (as logged by the oracle), plus tree metadata."""
-    import oracle
-    r = oracle.verify_sample(h["p"], h["q"], h["tokens"], h["parent_idx"], h["uniforms"])
-    rows = int(r["rows"].sum())
+def walk_rows(parent_idx, path, alen, every_visited: bool = False) -> int:
+    """Vocabulary rows an acceptance walk reads in full, from its result: at a
+    visited node the walk reads the whole row once a child is rejected (the
+    residual), and the last visited node's row for the bonus draw.  Children
+    are tested in ascending index order, so a rejection happened at node u iff
+    u has a child below the accepted one.  With every_visited, each visited
+    node's row counts (the logits walk needs every visited row's softmax)."""
+    rows = 0
+    for b in range(parent_idx.shape[0]):
+        n = int(alen[b])
+        if n < 0:
+            continue
+        nodes = [0] + [int(x) for x in path[b, :n]]
+        for k in range(n):
+            u, c = nodes[k], nodes[k + 1]
+            if every_visited or bool((parent_idx[b, 1:c] == u).any()):
+                rows += 1
+        rows += 1
+    return rows
+
+
+def sampler_bytes(wl, h, path, alen, every_visited: bool = False) -> int:
+    """Algorithmic bytes of the acceptance walk: both rows (p and q, 4 bytes
+    each) of every row it reads in full, 12 bytes per tested child (p(x),
+    q(x), its uniform) and the tree metadata (token, parent)."""
+    rows = walk_rows(h["parent_idx"], path, alen, every_visited)
     tested = int((h["parent_idx"] >= 0).sum())
     return rows * 8 * wl.vocab + tested * 12 + h["parent_idx"].size * 8
 
@@ -239,6 +308,55 @@ def time_commit(tv, wl, d, flush, stream, W, K):
                     "deepest root-to-leaf path accepted; mean over calls, L2 flushed before each"}
 
 
+def time_logits_walk(tv, wl, d, flush, stream, W, K, ref):
+    """tv_verify_sample_logits (the walk on the two models' logits) timed alone
+    from its own graph, L2 flushed before each launch; also how many sequences
+    end exactly as the walk on p, q (ref) does."""
+    import torch
+    lp, lq = wl.logits()
+    dlp, dlq = torch.from_numpy(lp).cuda(), torch.from_numpy(lq).cuda()
+    B, N = wl.batch, wl.num_nodes
+    path = torch.empty((B, N), dtype=torch.int32, device="cuda")
+    alen = torch.empty((B,), dtype=torch.int32, device="cuda")
+    bonus = torch.empty((B,), dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sdesc = tv.TvSampleDesc(B, N, wl.vocab)
+
+    def call(st):
+        s = tv.tv_verify_sample_logits(sdesc, dlp, dlq, d["tokens"], d["parent_idx"], d["uniforms"], path, alen,
+                                       bonus, None, 0, status, st)
+        if s:
+            raise tv.TreeVerifyError(s, "tv_verify_sample_logits")
+
+    call(stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call(torch.cuda.current_stream())
+    for _ in range(W):
+        flush.zero_()
+        g.replay()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} from the logits walk")
+    us = float(np.mean([e0.elapsed_time(e1) for e0, e1 in evs])) * 1e3
+    p_np, a_np, b_np = path.cpu().numpy(), alen.cpu().numpy(), bonus.cpu().numpy()
+    nbytes = sampler_bytes(wl, {"parent_idx": wl.parent_idx}, p_np, a_np, every_visited=True)
+    same = ((a_np == ref["alen"]) & (b_np == ref["bonus"]) & (p_np == ref["path"]).all(axis=1))
+    del g, dlp, dlq
+    return {"us": us, "bytes": nbytes, "achieved_gbs": nbytes / (us * 1e-6) / 1e9 if us > 0 else None,
+            "same_as_pq_walk": int(same.sum()), "sequences": B,
+            "note": "tv_verify_sample_logits on fp32 logits (softmax formed per visited row inside the walk); bytes: "
+                    "both logit rows of every visited node plus per-child gathers; mean over launches, L2 flushed "
+                    "before each"}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -320,6 +438,7 @@ def run_ours(args, rank, world, local_rank):
         e0.record(stream)
         g_step.replay()
         e1.record(stream)
+    clocks.sample_now()  # the queued steps are still running
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall
     clk = clocks.stop()
@@ -341,7 +460,9 @@ def run_ours(args, rank, world, local_rank):
 
     attn_ms = kernel_ms(g_attn)
     samp_ms = kernel_ms(g_samp)
+    walk = {"path": path.cpu().numpy(), "alen": alen.cpu().numpy(), "bonus": bonus.cpu().numpy()}
     commit = time_commit(tv, wl, d, flush, stream, W, min(K, 200))
+    logits_walk = time_logits_walk(tv, wl, d, flush, stream, W, min(K, 200), walk)
     total_ms = float(sum(step_ms))
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())}")
@@ -390,7 +511,7 @@ def run_ours(args, rank, world, local_rank):
     e2e_value = job_throughput(world, nodes, K2, e2e_ms)
     peak, peak_kind, _ = load_peaks()
     a_bytes = attention_bytes(wl)
-    s_bytes = sampler_bytes(wl, h)
+    s_bytes = sampler_bytes(wl, h, walk["path"], walk["alen"])
     attn_avg_s = (sum(attn_ms) / K) / 1e3
     achieved = a_bytes / attn_avg_s / 1e9
     kernel_key = "attn_tc" if aplan.kernel == 0 else "attn_simt"
@@ -424,6 +545,7 @@ def run_ours(args, rank, world, local_rank):
                           "note": "sampler bytes: rows the walk reads (algorithmic); literal = all of p and q"},
         "median_us_per_step": float(np.median(step_ms)) * 1e3,
         "commit": commit,
+        "sample_logits": logits_walk,
         "e2e": {"value": e2e_value, "unit": "nodes/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": K2},
         "gpu_launches": K * (aplan.launches + splan.launches),

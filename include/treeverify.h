@@ -202,6 +202,33 @@ TV_API tv_status tv_verify_sample(const tv_sample_desc *desc, const float *p, co
 
 /* Static string for a status code. */
 /*
+ * The acceptance walk on the two models' logits instead of their
+ * distributions (the fused-logits form of tv_verify_sample).  Blog
+ * "Speculative decoding x tree attention", section 2, and glossary
+ * "Tree-based speculative decoding", section "SpecInfer": p and q are the
+ * target and draft models' output distributions, i.e. the row softmax of
+ * their logits.
+ *
+ * Same descriptor, tree, uniforms, outputs, errors and stream behaviour as
+ * tv_verify_sample; target_logits and draft_logits are fp32 [B][N][V] device
+ * arrays (row u: the logits after node u's path), and p = softmax(target row),
+ * q = softmax(draft row) at temperature 1.  Each row the walk visits is read
+ * once and turned into its softmax in shared memory (row max, fp64 sum of
+ * exp(l - max), both cluster-wide); p and q are never written to memory.  The
+ * exponentials are fp32, so a decision can differ from an exact-arithmetic walk
+ * only when its uniform lies within about 1e-6 of the threshold.  A logit of
+ * -inf (a masked token) has probability 0; every row the walk visits needs at
+ * least one finite logit (an all -inf row has no softmax and its result is
+ * undefined).
+ */
+TV_API tv_status tv_verify_sample_logits(const tv_sample_desc *desc, const float *target_logits,
+                                         const float *draft_logits, const int32_t *tree_tokens,
+                                         const int32_t *parent_idx, const float *uniforms,
+                                         int32_t *accepted_path, int32_t *accepted_len, int32_t *bonus_token,
+                                         void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                                         void *stream);
+
+/*
  * Commit the accepted path into the KV cache: the step after verification.
  * Blog "Speculative decoding x tree attention", section "KV cache management and
  * prefix sharing", and glossary "Tree-based speculative decoding", section "KV

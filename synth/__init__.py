@@ -78,6 +78,7 @@ def lib():
         L.sy_normal_bf16.argtypes = [P, i64, u64, u32, i64, dbl]
         L.sy_paged_cache.argtypes = [P, ctypes.c_int, i32, i32, i32, i32, i32, P, P, i64, u64, u32, dbl]
         L.sy_pq_rows.argtypes = [P, P, i64, P, i64, u64, u32, u32, ctypes.c_int, dbl, dbl]
+        L.sy_logit_rows.argtypes = [P, P, i64, P, i64, u64, u32, u32, ctypes.c_int, dbl, dbl]
         L.sy_categorical.argtypes = [P, i64, dbl]
         L.sy_categorical.restype = i64
         _lib = L
@@ -133,6 +134,17 @@ def pq_rows(row_ids, V: int, seed: int, mode: int, sp: float, sn: float):
     if R:
         lib().sy_pq_rows(_ptr(p), _ptr(q), R, _ptr(row_ids), V, seed, STREAM_LOGIT, STREAM_NOISE, mode, sp, sn)
     return p, q
+
+
+def logit_rows(row_ids, V: int, seed: int, mode: int, sp: float, sn: float):
+    """The logits whose row softmaxes pq_rows returns (target, draft), float32."""
+    row_ids = np.ascontiguousarray(np.asarray(row_ids, dtype=np.int64))
+    R = row_ids.shape[0]
+    la = np.empty((R, V), dtype=np.float32)
+    lb = np.empty((R, V), dtype=np.float32)
+    if R:
+        lib().sy_logit_rows(_ptr(la), _ptr(lb), R, _ptr(row_ids), V, seed, STREAM_LOGIT, STREAM_NOISE, mode, sp, sn)
+    return la, lb
 
 
 def categorical(w: np.ndarray, u: float) -> int:
@@ -286,6 +298,14 @@ class Workload:
             shape = (self.batch, self.num_nodes, self.vocab)
             self.extra["pq"] = (p.reshape(shape), q.reshape(shape))
         return self.extra["pq"]
+
+    def logits(self):
+        """(target, draft) logits float32 [B][N][V] whose row softmaxes are pq()."""
+        if "logits" not in self.extra:
+            la, lb = logit_rows(self.row_keys.reshape(-1), self.vocab, self.seed, self.pq_mode, self.pq_sp, self.pq_sn)
+            shape = (self.batch, self.num_nodes, self.vocab)
+            self.extra["logits"] = (la.reshape(shape), lb.reshape(shape))
+        return self.extra["logits"]
 
     def uniforms(self) -> np.ndarray:
         return uniforms(self.batch * self.num_nodes, self.seed, STREAM_UNIFORM).reshape(self.batch, self.num_nodes)

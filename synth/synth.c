@@ -197,6 +197,25 @@ void sy_pq_rows(float *p, float *q, int64_t rows, const int64_t *row_ids, int64_
 }
 
 /*
+ * The same rows' logits, before any softmax: la = sp * n_a and lb = sp * n_b
+ * (mode 0) or la + sn * n_b (mode 1), each rounded to float.  The inputs of a
+ * verifier that takes the two models' logits.
+ */
+void sy_logit_rows(float *la, float *lb, int64_t rows, const int64_t *row_ids, int64_t V, uint64_t seed,
+                   uint32_t stream_a, uint32_t stream_b, int mode, double sp, double sn) {
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t r = 0; r < rows; ++r) {
+        uint64_t base = (uint64_t)row_ids[r] * (uint64_t)V;
+        for (int64_t x = 0; x < V; ++x) {
+            double a = sp * normal_at(seed, stream_a, base + x);
+            double nb = normal_at(seed, stream_b, base + x);
+            la[r * V + x] = (float)a;
+            lb[r * V + x] = (float)((mode == 0) ? sp * nb : a + sn * nb);
+        }
+    }
+}
+
+/*
  * Draw one index from the (not necessarily normalised) weights w[0..V) with
  * a uniform u in [0,1): the first index whose running double sum exceeds
  * u * total; the last positive index if rounding leaves none.  Used only to

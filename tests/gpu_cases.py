@@ -118,10 +118,11 @@ def random_attn(seed, B, N, Hq, Hkv, D, prefix_lens, dtype="bf16", permute=True,
     return Attn(q, k, v, bt, prefix_lens, parents, dtype, Hkv)
 
 
-def run_sampler_gpu(p, q, tokens, parent, uniforms, status=None):
+def run_sampler_gpu(p, q, tokens, parent, uniforms, status=None, logits=False):
+    """The walk on the GPU; with logits=True p and q are the two models' logits."""
     path, alen, bonus = tv.verify_sample(dev(np.asarray(p, np.float32)), dev(np.asarray(q, np.float32)),
                                          dev(np.asarray(tokens, np.int32)), dev(np.asarray(parent, np.int32)),
-                                         dev(np.asarray(uniforms, np.float32)), dev_status=status)
+                                         dev(np.asarray(uniforms, np.float32)), dev_status=status, logits=logits)
     torch.cuda.synchronize()
     return {"accepted_path": path.cpu().numpy(), "accepted_len": alen.cpu().numpy(),
             "bonus_token": bonus.cpu().numpy()}

@@ -94,6 +94,16 @@ def test_sampler_rejects_bad_descriptors(kw, status):
     d = tv.TvSampleDesc(**kw)
     dummy = 256
     assert tv.tv_verify_sample(d, *([dummy] * 8), stream=0) == status
+    assert tv.tv_verify_sample_logits(d, *([dummy] * 8), stream=0) == status
+
+
+def test_sampler_rejects_null_pointers():
+    d = tv.TvSampleDesc(2, 8, 1000)
+    for i in range(8):
+        args = [256] * 8
+        args[i] = 0
+        assert tv.tv_verify_sample(d, *args, stream=0) == tv.TV_ERR_INVALID_ARG
+        assert tv.tv_verify_sample_logits(d, *args, stream=0) == tv.TV_ERR_INVALID_ARG
 
 
 def test_sampler_plan_covers_vocab():

@@ -1,0 +1,31 @@
+"""Host-side bookkeeping of bench.py: the count of vocabulary rows an
+acceptance walk reads in full, which the roofline's algorithmic bytes use,
+matches the count the oracle logs while it walks."""
+import numpy as np
+
+import bench
+import oracle
+import synth
+
+
+def test_walk_rows_matches_the_oracle_log():
+    rng = np.random.default_rng(4)
+    B, N, V = 300, 12, 64
+    parent = np.array([[-1] + [int(rng.integers(0, i)) for i in range(1, N)] for _ in range(B)], np.int32)
+    lp = rng.normal(0, 2, (B, N, V))
+    p = oracle.softmax_rows(lp)
+    q = oracle.softmax_rows(lp + rng.normal(0, 1.5, (B, N, V)))
+    tok = rng.integers(0, V, (B, N)).astype(np.int32)
+    u = rng.random((B, N)).astype(np.float32)
+    r = oracle.verify_sample(p, q, tok, parent, u)
+    assert bench.walk_rows(parent, r["accepted_path"], r["accepted_len"]) == int(r["rows"].sum())
+    # every visited row: one per accepted node plus the last one
+    assert bench.walk_rows(parent, r["accepted_path"], r["accepted_len"], every_visited=True) == \
+        int((r["accepted_len"] + 1).sum())
+
+
+def test_walk_rows_on_the_small_workload():
+    wl = synth.make("tiny")
+    p, q = wl.pq()
+    r = oracle.verify_sample(p, q, wl.tree_tokens, wl.parent_idx, wl.uniforms())
+    assert bench.walk_rows(wl.parent_idx, r["accepted_path"], r["accepted_len"]) == int(r["rows"].sum())

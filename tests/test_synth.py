@@ -59,3 +59,16 @@ def test_bf16_cache_is_rounded_normal():
     # logical position 0, head 0 equals element 0 of the K stream
     ref = synth.normals(4, wl.seed, synth.STREAM_K)[0]
     assert k[bt[0], 0, 0, 0] == ref
+
+
+def test_logits_are_the_distributions_before_softmax():
+    # the row softmax of the generated logits is the generated p, q
+    for name in ("tiny", "l8b"):
+        wl = synth.make(name)
+        p, q = wl.pq()
+        lp, lq = wl.logits()
+        assert lp.shape == p.shape and lp.dtype == np.float32
+        for l, d in ((lp, p), (lq, q)):
+            x = l[0, :3].astype(np.float64)
+            e = np.exp(x - x.max(axis=-1, keepdims=True))
+            np.testing.assert_allclose(e / e.sum(axis=-1, keepdims=True), d[0, :3], rtol=2e-6, atol=1e-30)

@@ -74,11 +74,12 @@ def lib() -> ctypes.CDLL:
         L.tv_verify_sample_workspace_size.restype = sz
         L.tv_verify_sample.argtypes = [ctypes.POINTER(TvSampleDesc), P, P, P, P, P, P, P, P, P, sz, P, P]
         L.tv_commit_path.argtypes = [ctypes.POINTER(TvAttnDesc), P, P, P, P, P, P, P, P, P]
+        L.tv_verify_sample_logits.argtypes = [ctypes.POINTER(TvSampleDesc), P, P, P, P, P, P, P, P, P, sz, P, P]
         L.tv_status_string.argtypes = [ctypes.c_int32]
         L.tv_status_string.restype = ctypes.c_char_p
         L.tv_version.restype = ctypes.c_int32
         for name in ("tv_tree_attention_plan", "tv_tree_attention", "tv_tree_attention_static",
-                     "tv_verify_sample_plan", "tv_verify_sample", "tv_commit_path"):
+                     "tv_verify_sample_plan", "tv_verify_sample", "tv_commit_path", "tv_verify_sample_logits"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -160,6 +161,16 @@ def tv_verify_sample(desc, p, q, tree_tokens, parent_idx, uniforms, accepted_pat
                                       _ptr(workspace), int(workspace_bytes), _ptr(dev_status), _stream(stream)))
 
 
+def tv_verify_sample_logits(desc, target_logits, draft_logits, tree_tokens, parent_idx, uniforms, accepted_path,
+                            accepted_len, bonus_token, workspace=None, workspace_bytes: int = 0, dev_status=None,
+                            stream=None) -> int:
+    return int(lib().tv_verify_sample_logits(ctypes.byref(desc), _ptr(target_logits), _ptr(draft_logits),
+                                             _ptr(tree_tokens), _ptr(parent_idx), _ptr(uniforms),
+                                             _ptr(accepted_path), _ptr(accepted_len), _ptr(bonus_token),
+                                             _ptr(workspace), int(workspace_bytes), _ptr(dev_status),
+                                             _stream(stream)))
+
+
 def tv_commit_path(desc, paged_k, paged_v, block_table, prefix_lens, accepted_path, accepted_len, new_prefix_lens,
                    dev_status=None, stream=None) -> int:
     return int(lib().tv_commit_path(ctypes.byref(desc), _ptr(paged_k), _ptr(paged_v), _ptr(block_table),
@@ -213,8 +224,9 @@ def tree_attention(q, k_cache, v_cache, block_table, prefix_lens, parent_idx, so
 
 
 def verify_sample(p, q, tree_tokens, parent_idx, uniforms, accepted_path=None, accepted_len=None,
-                  bonus_token=None, dev_status=None, stream=None):
-    """Run tv_verify_sample; returns (accepted_path, accepted_len, bonus_token)."""
+                  bonus_token=None, dev_status=None, stream=None, logits: bool = False):
+    """Run tv_verify_sample (or, with logits=True, tv_verify_sample_logits on the
+    two models' logits); returns (accepted_path, accepted_len, bonus_token)."""
     import torch
     _check_cuda(p, q, tree_tokens, parent_idx, uniforms, dev_status)
     if p.dtype != torch.float32 or q.dtype != torch.float32 or uniforms.dtype != torch.float32:
@@ -228,10 +240,11 @@ def verify_sample(p, q, tree_tokens, parent_idx, uniforms, accepted_path=None, a
     if bonus_token is None:
         bonus_token = torch.empty((B,), dtype=torch.int32, device=dev)
     desc = TvSampleDesc(B, N, V)
-    s = tv_verify_sample(desc, p, q, tree_tokens, parent_idx, uniforms, accepted_path, accepted_len, bonus_token,
-                         None, 0, dev_status, stream)
+    call = tv_verify_sample_logits if logits else tv_verify_sample
+    s = call(desc, p, q, tree_tokens, parent_idx, uniforms, accepted_path, accepted_len, bonus_token, None, 0,
+             dev_status, stream)
     if s != TV_OK:
-        raise TreeVerifyError(s, "tv_verify_sample")
+        raise TreeVerifyError(s, call.__name__)
     return accepted_path, accepted_len, bonus_token
 
 

@@ -105,6 +105,30 @@ void make_sample_plan(const tv_sample_desc* d, tv_sample_plan* p) {
 
 }  // namespace
 
+namespace {
+tv_status verify_sample_common(const tv_sample_desc* desc, const float* p, const float* q, const int32_t* tree_tokens,
+                               const int32_t* parent_idx, const float* uniforms, int32_t* accepted_path,
+                               int32_t* accepted_len, int32_t* bonus_token, int32_t* dev_status, void* stream,
+                               bool logits) {
+    tv_status s = check_sample_desc(desc);
+    if (s != TV_OK) return s;
+    if (!p || !q || !tree_tokens || !parent_idx || !uniforms || !accepted_path || !accepted_len || !bonus_token)
+        return TV_ERR_INVALID_ARG;
+    tv_sample_plan plan;
+    make_sample_plan(desc, &plan);
+    tv::SampleArgs a = {};
+    a.p = p; a.q = q; a.tokens = tree_tokens; a.parent = parent_idx; a.uniforms = uniforms;
+    a.path = accepted_path; a.len = accepted_len; a.bonus = bonus_token; a.status = dev_status;
+    a.B = desc->batch; a.N = desc->num_nodes; a.V = desc->vocab;
+    a.cluster = plan.cluster_ctas; a.threads = plan.threads; a.slice = plan.slice; a.smem_bytes = plan.smem_bytes;
+    a.vec4 = (desc->vocab % 4 == 0) && !(reinterpret_cast<uintptr_t>(p) & 15) && !(reinterpret_cast<uintptr_t>(q) & 15);
+    a.logits = logits ? 1 : 0;
+    int launches = 0;
+    cudaError_t e = tv::launch_verify_sample(a, static_cast<cudaStream_t>(stream), &launches);
+    return e == cudaSuccess ? TV_OK : TV_ERR_CUDA;
+}
+}  // namespace
+
 extern "C" {
 
 int32_t tv_version(void) { return 100; }
@@ -218,27 +242,25 @@ tv_status tv_commit_path(const tv_attn_desc* desc, void* paged_k, void* paged_v,
     return tv::launch_commit(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? TV_OK : TV_ERR_CUDA;
 }
 
+
 tv_status tv_verify_sample(const tv_sample_desc* desc, const float* p, const float* q, const int32_t* tree_tokens,
                            const int32_t* parent_idx, const float* uniforms, int32_t* accepted_path,
                            int32_t* accepted_len, int32_t* bonus_token, void* workspace, size_t workspace_bytes,
                            int32_t* dev_status, void* stream) {
     (void)workspace;
     (void)workspace_bytes;
-    tv_status s = check_sample_desc(desc);
-    if (s != TV_OK) return s;
-    if (!p || !q || !tree_tokens || !parent_idx || !uniforms || !accepted_path || !accepted_len || !bonus_token)
-        return TV_ERR_INVALID_ARG;
-    tv_sample_plan plan;
-    make_sample_plan(desc, &plan);
-    tv::SampleArgs a = {};
-    a.p = p; a.q = q; a.tokens = tree_tokens; a.parent = parent_idx; a.uniforms = uniforms;
-    a.path = accepted_path; a.len = accepted_len; a.bonus = bonus_token; a.status = dev_status;
-    a.B = desc->batch; a.N = desc->num_nodes; a.V = desc->vocab;
-    a.cluster = plan.cluster_ctas; a.threads = plan.threads; a.slice = plan.slice; a.smem_bytes = plan.smem_bytes;
-    a.vec4 = (desc->vocab % 4 == 0) && !(reinterpret_cast<uintptr_t>(p) & 15) && !(reinterpret_cast<uintptr_t>(q) & 15);
-    int launches = 0;
-    cudaError_t e = tv::launch_verify_sample(a, static_cast<cudaStream_t>(stream), &launches);
-    return e == cudaSuccess ? TV_OK : TV_ERR_CUDA;
+    return verify_sample_common(desc, p, q, tree_tokens, parent_idx, uniforms, accepted_path, accepted_len,
+                                bonus_token, dev_status, stream, false);
+}
+
+tv_status tv_verify_sample_logits(const tv_sample_desc* desc, const float* target_logits, const float* draft_logits,
+                                  const int32_t* tree_tokens, const int32_t* parent_idx, const float* uniforms,
+                                  int32_t* accepted_path, int32_t* accepted_len, int32_t* bonus_token,
+                                  void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    (void)workspace;
+    (void)workspace_bytes;
+    return verify_sample_common(desc, target_logits, draft_logits, tree_tokens, parent_idx, uniforms, accepted_path,
+                                accepted_len, bonus_token, dev_status, stream, true);
 }
 
 }  // extern "C"

@@ -49,6 +49,7 @@ struct SampleArgs {
     int B, N, V;
     int cluster, threads, slice, smem_bytes;
     int vec4;           // rows start 16-byte aligned and V % 4 == 0
+    int logits;         // p and q hold the two models' logits: the walk applies the row softmax
 };
 
 cudaError_t launch_verify_sample(const SampleArgs& a, cudaStream_t st, int* launches);

@@ -49,7 +49,9 @@ struct SampleShared {
     int ch_n;      // children gathered in this batch
     int ch_next;   // index where the scan for the next batch resumes (N when done)
     double warp_part[MAX_THREADS / 32];
-    double peer[2][MAX_CLUSTER];  // partials from every CTA of the cluster, by pass parity
+    double warp_part2[MAX_THREADS / 32];
+    double peer[2][MAX_CLUSTER];   // values from every CTA of the cluster, by exchange parity
+    double peer2[2][MAX_CLUSTER];  // second values of two-value exchanges
     unsigned long long peer_bar[2];
     unsigned long long row_bar[2];
     int timeout;
@@ -112,6 +114,16 @@ __device__ __forceinline__ double warp_sum_d(double v) {
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
+__device__ __forceinline__ double warp_max_d(double v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_max_f(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
 
 // max(0, d) for the residual terms: the sign is read from the high word, because
 // the fp64 max instruction runs at an eighth of the fp64 add / fma rate
@@ -128,9 +140,12 @@ struct Walker {
     float* buf;      // [2][2][slice]: buffer x holds p at buf + 2*x*slice, q right after
     int b, rank, C, lo, n, tid, lane, warp, nwarps, segw;
     bool bulk;
-    int passes;      // cluster passes so far
+    int passes;      // cluster exchanges so far
     int row_uses[2];
     bool row_pending[2];
+    // logits mode: the softmax of the row in buffer x is p = exp(l - mp) * zp_inv
+    float row_mp[2], row_mq[2];
+    double row_zp_inv[2], row_zq_inv[2];
 
     __device__ float* ps(int x) const { return buf + (size_t)2 * x * a.slice; }
     __device__ float* qs(int x) const { return ps(x) + a.slice; }
@@ -203,19 +218,36 @@ struct Walker {
         const double wsum = warp_sum_d((a0 + a1) + (a2 + a3));
         if (lane == 0) sh.warp_part[warp] = wsum;
         __syncthreads();
+        // this CTA's partial: a fixed shuffle tree over its warps (warp 0's value is sent)
+        const double s = warp == 0 ? warp_sum_d(lane < nwarps ? sh.warp_part[lane] : 0.0) : 0.0;
+        double total, unused;
+        exchange(1, s, 0.0, false, total, unused);
+        return total;
+    }
+
+    // One cluster-wide exchange of nv (1 or 2) values: warp 0 holds this CTA's values
+    // v0, v1 and sends them to every CTA of the cluster (one lane per receiver, by
+    // st.async completing on the receiver's own mbarrier); every warp then combines
+    // the C values with the same shuffle tree -- sums, or maxima when take_max -- so
+    // all CTAs and all warps obtain the same bits and take the same branches.  The
+    // per-CTA values stay in sh.peer / sh.peer2 at the parity of the exchange.
+    __device__ void exchange(int nv, double v0, double v1, bool take_max, double& r0, double& r1) {
         const int par = passes & 1;
         const uint32_t use = (uint32_t)(passes >> 1);
         ++passes;
         if (warp == 0) {
-            // this CTA's partial (a fixed shuffle tree over its warps), sent to every
-            // CTA of the cluster, one lane per receiver
-            const double s = warp_sum_d(lane < nwarps ? sh.warp_part[lane] : 0.0);
             if (C == 1) {
-                if (lane == 0) sh.peer[par][0] = s;
+                if (lane == 0) {
+                    sh.peer[par][0] = v0;
+                    sh.peer2[par][0] = v1;
+                }
             } else {
                 const uint32_t bar = smem_u32(&sh.peer_bar[par]);
-                if (lane == 0) mbar_expect_tx(bar, (uint32_t)(8 * C));
-                if (lane < C) st_async_f64(mapa(smem_u32(&sh.peer[par][rank]), lane), s, mapa(bar, lane));
+                if (lane == 0) mbar_expect_tx(bar, (uint32_t)(8 * nv * C));
+                if (lane < C) {
+                    st_async_f64(mapa(smem_u32(&sh.peer[par][rank]), lane), v0, mapa(bar, lane));
+                    if (nv == 2) st_async_f64(mapa(smem_u32(&sh.peer2[par][rank]), lane), v1, mapa(bar, lane));
+                }
             }
         }
         if (C == 1) {
@@ -223,12 +255,80 @@ struct Walker {
         } else {
             mbar_wait(smem_u32(&sh.peer_bar[par]), use & 1, &sh.timeout);
         }
-        // every warp adds the C partials with the same shuffle tree, so all CTAs (and
-        // all warps) obtain the same bits and take the same branches
-        return warp_sum_d(lane < C ? sh.peer[par][lane] : 0.0);
+        const double id = take_max ? -INFINITY : 0.0;
+        const double x0 = lane < C ? sh.peer[par][lane] : id;
+        r0 = take_max ? warp_max_d(x0) : warp_sum_d(x0);
+        if (nv == 2) {
+            const double x1 = lane < C ? sh.peer2[par][lane] : id;
+            r1 = take_max ? warp_max_d(x1) : warp_sum_d(x1);
+        } else {
+            r1 = 0.0;
+        }
+    }
+
+    // Logits mode: buffer x holds this CTA's slice of one node's target and draft
+    // logits.  Turn them in place into the row softmax: e = exp(l - M) in fp32 with M
+    // the row max, Z the fp64 sum of e over the whole row (both cluster-wide), and
+    // p = (float)(e * (1 / Z)); keep M and 1 / Z for the children's p(x), q(x), which
+    // the gather computes with the same expression so they equal the converted row.
+    __device__ void prep_row(int x) {
+        float* pl = ps(x);
+        float* ql = qs(x);
+        float mp = -INFINITY, mq = -INFINITY;
+        for (int i = tid; i < n; i += blockDim.x) {
+            mp = fmaxf(mp, pl[i]);
+            mq = fmaxf(mq, ql[i]);
+        }
+        mp = warp_max_f(mp);
+        mq = warp_max_f(mq);
+        if (lane == 0) {
+            sh.warp_part[warp] = (double)mp;
+            sh.warp_part2[warp] = (double)mq;
+        }
+        __syncthreads();
+        double Mp, Mq;
+        {
+            const double v0 = warp == 0 ? warp_max_d(lane < nwarps ? sh.warp_part[lane] : -INFINITY) : 0.0;
+            const double v1 = warp == 0 ? warp_max_d(lane < nwarps ? sh.warp_part2[lane] : -INFINITY) : 0.0;
+            exchange(2, v0, v1, true, Mp, Mq);
+        }
+        const float mpf = (float)Mp, mqf = (float)Mq;
+        double sp = 0.0, sq = 0.0;
+        for (int i = tid; i < n; i += blockDim.x) {
+            const float ep = expf(pl[i] - mpf), eq = expf(ql[i] - mqf);
+            pl[i] = ep;
+            ql[i] = eq;
+            sp += (double)ep;
+            sq += (double)eq;
+        }
+        sp = warp_sum_d(sp);
+        sq = warp_sum_d(sq);
+        __syncthreads();  // warp 0 has read the max partials before its exchange
+        if (lane == 0) {
+            sh.warp_part[warp] = sp;
+            sh.warp_part2[warp] = sq;
+        }
+        __syncthreads();
+        double Zp, Zq;
+        {
+            const double v0 = warp == 0 ? warp_sum_d(lane < nwarps ? sh.warp_part[lane] : 0.0) : 0.0;
+            const double v1 = warp == 0 ? warp_sum_d(lane < nwarps ? sh.warp_part2[lane] : 0.0) : 0.0;
+            exchange(2, v0, v1, false, Zp, Zq);
+        }
+        const double zpi = Zp > 0.0 ? 1.0 / Zp : 0.0, zqi = Zq > 0.0 ? 1.0 / Zq : 0.0;
+        for (int i = tid; i < n; i += blockDim.x) {
+            pl[i] = (float)((double)pl[i] * zpi);
+            ql[i] = (float)((double)ql[i] * zqi);
+        }
+        __syncthreads();
+        row_mp[x] = mpf;
+        row_mq[x] = mqf;
+        row_zp_inv[x] = zpi;
+        row_zq_inv[x] = zqi;
     }
 };
 
+template <bool LOGITS>
 __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a) {
     extern __shared__ float4 sample_dyn[];
     __shared__ SampleShared sh;
@@ -255,7 +355,8 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
     Walker w{a, sh, reinterpret_cast<float*>(sample_dyn), b, rank, C, lo, n, tid, lane, warp, nwarps,
-             ((n + nwarps - 1) / nwarps + 127) / 128 * 128, a.vec4 != 0, 0, {0, 0}, {false, false}};
+             ((n + nwarps - 1) / nwarps + 127) / 128 * 128, a.vec4 != 0, 0, {0, 0}, {false, false},
+             {0.f, 0.f}, {0.f, 0.f}, {0.0, 0.0}, {0.0, 0.0}};
     // the root's row is needed unless its first child is accepted: start it now
     w.issue_row(0, 0);
 
@@ -299,6 +400,11 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
         cur_z = 1.0;
         int accepted = -1;
         int scan = u + 1;
+        if (LOGITS) {
+            // even the first child's test needs the row's softmax normalisers
+            w.wait_row(x);
+            w.prep_row(x);
+        }
         while (accepted < 0 && scan < N) {
             // warp 0 collects the next (up to 32) children of u in ascending order and
             // gathers their draft tokens' p, q and acceptance draws
@@ -324,8 +430,15 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
                 if (lane < found) {
                     const int c = sh.ch_node[lane];
                     const size_t row = ((size_t)b * N + u) * (size_t)a.V;
-                    sh.ch_p[lane] = (double)__ldg(a.p + row + sh.token[c]);
-                    sh.ch_q[lane] = (double)__ldg(a.q + row + sh.token[c]);
+                    if (LOGITS) {
+                        const float ep = expf(__ldg(a.p + row + sh.token[c]) - w.row_mp[x]);
+                        const float eq = expf(__ldg(a.q + row + sh.token[c]) - w.row_mq[x]);
+                        sh.ch_p[lane] = (double)(float)((double)ep * w.row_zp_inv[x]);
+                        sh.ch_q[lane] = (double)(float)((double)eq * w.row_zq_inv[x]);
+                    } else {
+                        sh.ch_p[lane] = (double)__ldg(a.p + row + sh.token[c]);
+                        sh.ch_q[lane] = (double)__ldg(a.q + row + sh.token[c]);
+                    }
                     sh.ch_u[lane] = (double)__ldg(a.uniforms + (size_t)b * N + c);
                 }
                 if (lane == 0) {
@@ -479,8 +592,9 @@ int sample_max_cluster() {
     static int best = -1;
     if (best >= 0) return best;
     best = 8;
-    if (cudaFuncSetAttribute(verify_sample_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
-        cudaFuncSetAttribute(verify_sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024) ==
+    if (cudaFuncSetAttribute(verify_sample_kernel<false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+            cudaSuccess &&
+        cudaFuncSetAttribute(verify_sample_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024) ==
             cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
@@ -494,7 +608,7 @@ int sample_max_cluster() {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, verify_sample_kernel, &cfg) == cudaSuccess && clusters > 0)
+        if (cudaOccupancyMaxActiveClusters(&clusters, verify_sample_kernel<false>, &cfg) == cudaSuccess && clusters > 0)
             best = 16;
     }
     cudaGetLastError();
@@ -502,11 +616,11 @@ int sample_max_cluster() {
 }
 
 cudaError_t launch_verify_sample(const SampleArgs& a, cudaStream_t st, int* launches) {
-    cudaError_t e = cudaFuncSetAttribute(verify_sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         a.smem_bytes);
+    void (*kern)(SampleArgs) = a.logits ? verify_sample_kernel<true> : verify_sample_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, a.smem_bytes);
     if (e != cudaSuccess) return e;
     if (a.cluster > 8) {
-        e = cudaFuncSetAttribute(verify_sample_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg = {};
@@ -526,7 +640,7 @@ cudaError_t launch_verify_sample(const SampleArgs& a, cudaStream_t st, int* laun
     cfg.attrs = attr;
     cfg.numAttrs = a.cluster > 1 ? 2 : 1;
     *launches = 1;
-    return cudaLaunchKernelEx(&cfg, verify_sample_kernel, a);
+    return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 }  // namespace tv
