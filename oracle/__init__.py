@@ -176,6 +176,84 @@ def commit_path(k_cache, v_cache, block_table, prefix_lens, accepted_path, accep
     return k, v, new_pl, int(st)
 
 
+def chain_parents(B: int, N: int) -> np.ndarray:
+    """Parent arrays of B chains of N nodes (linear speculation: node i's parent
+    is i - 1), the tree a NULL parent array stands for in the library."""
+    return np.tile(np.arange(-1, N - 1, dtype=np.int32), (B, 1))
+
+
+def _seq_parent(parent_idx, b: int, n: int) -> np.ndarray:
+    return chain_parents(1, n) if parent_idx is None else np.asarray(parent_idx, np.int32)[b:b + 1, :n]
+
+
+def tree_attention_ragged(query, k_cache, v_cache, block_table, prefix_lens, parent_idx, node_counts, num_kv_heads,
+                          dtype: str, scale: float | None = None) -> np.ndarray:
+    """Ragged trees in one batch: sequence b's tree is its first node_counts[b]
+    nodes, and by the definition of tree attention (glossary, "Tree attention")
+    each sequence is its own problem, so this is :func:`tree_attention` on each
+    sequence's slice.  parent_idx None means chains.  Rows of padding nodes are
+    NaN (not defined)."""
+    B, N, Hq, D = query.shape
+    out = np.full((B, N, Hq, D), np.nan)
+    for b in range(B):
+        n = int(node_counts[b])
+        if n == 0:
+            continue
+        out[b, :n] = tree_attention(query[b:b + 1, :n], k_cache, v_cache, np.asarray(block_table)[b:b + 1],
+                                    np.asarray(prefix_lens)[b:b + 1], _seq_parent(parent_idx, b, n), num_kv_heads,
+                                    dtype, scale)[0]
+    return out
+
+
+def verify_sample_ragged(p, q, tree_tokens, parent_idx, uniforms, node_counts, eps: float = 1e-6,
+                         logits: bool = False):
+    """The walk on ragged trees: sequence b's tree is its first node_counts[b]
+    nodes (children past it do not exist); each sequence walks on its own
+    slice with :func:`verify_sample` (or :func:`verify_sample_logits`).  A
+    sequence with no nodes accepts nothing and draws no token (length 0,
+    bonus -1).  parent_idx None means chains."""
+    B, N = np.asarray(tree_tokens).shape
+    res = {"accepted_path": np.full((B, N), -1, np.int32), "accepted_len": np.zeros(B, np.int32),
+           "bonus_token": np.full(B, -1, np.int32), "near": np.zeros(B, np.int32), "rows": np.zeros(B, np.int32),
+           "rc": 0}
+    walk = verify_sample_logits if logits else verify_sample
+    for b in range(B):
+        n = int(node_counts[b])
+        if n == 0:
+            continue
+        r = walk(np.asarray(p)[b:b + 1, :n], np.asarray(q)[b:b + 1, :n], np.asarray(tree_tokens)[b:b + 1, :n],
+                 _seq_parent(parent_idx, b, n), np.asarray(uniforms)[b:b + 1, :n], eps=eps)
+        res["accepted_path"][b, :n] = r["accepted_path"][0]
+        for key in ("accepted_len", "bonus_token", "near", "rows"):
+            res[key][b] = r[key][0]
+        res["rc"] = res["rc"] or r["rc"]
+    return res
+
+
+def commit_path_ragged(k_cache, v_cache, block_table, prefix_lens, accepted_path, accepted_len, node_counts):
+    """The KV commit on ragged trees: each sequence is committed on its own
+    with :func:`commit_path` over its node_counts[b]-node tree (its blocks are
+    its own, so the order does not matter).  Returns (k, v, new_prefix_lens,
+    status)."""
+    k = np.ascontiguousarray(k_cache).copy()
+    v = np.ascontiguousarray(v_cache).copy()
+    pl = np.asarray(prefix_lens, np.int32)
+    path = np.asarray(accepted_path, np.int32)
+    alen = np.asarray(accepted_len, np.int32)
+    B = path.shape[0]
+    new_pl = pl.copy()
+    st = 0
+    for b in range(B):
+        n = int(node_counts[b])
+        if n == 0 or alen[b] < 0:
+            continue
+        k, v, npl, s = commit_path(k, v, np.asarray(block_table)[b:b + 1], pl[b:b + 1], path[b:b + 1, :n],
+                                   alen[b:b + 1])
+        new_pl[b] = npl[0]
+        st = st or s
+    return k, v, new_pl, st
+
+
 def softmax_rows(logits) -> np.ndarray:
     """Plain softmax over the last axis in fp64 (max-shifted), rounded to fp32:
     the distributions a verifier that takes logits works from."""
