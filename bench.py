@@ -184,6 +184,7 @@ def make_inputs(workload: str, seed: int):
         "query": wl.query(), "k": wl.k_cache(), "v": wl.v_cache(), "block_table": wl.block_table,
         "prefix_lens": wl.prefix_lens, "parent_idx": wl.parent_idx, "p": p, "q": q,
         "tokens": wl.tree_tokens, "uniforms": wl.uniforms(),
+        **({} if wl.node_counts is None else {"node_counts": wl.node_counts}),
     }
 
 
@@ -192,8 +193,8 @@ def attention_bytes(wl) -> int:
     row the call must read (prefix plus tree block, per KV head), the queries
     and the outputs."""
     el = 2 if wl.dtype == "bf16" else 4
-    kv = 2 * int((wl.prefix_lens.astype(np.int64) + wl.num_nodes).sum()) * wl.num_kv_heads * wl.head_dim * el
-    qo = 2 * wl.batch * wl.num_nodes * wl.num_q_heads * wl.head_dim * el
+    kv = 2 * int((wl.prefix_lens.astype(np.int64) + wl.counts).sum()) * wl.num_kv_heads * wl.head_dim * el
+    qo = 2 * int(wl.counts.sum()) * wl.num_q_heads * wl.head_dim * el
     return kv + qo
 
 
@@ -223,8 +224,9 @@ def sampler_bytes(wl, h, path, alen, every_visited: bool = False) -> int:
     each) of every row it reads in full, 12 bytes per tested child (p(x),
     q(x), its uniform) and the tree metadata (token, parent)."""
     rows = walk_rows(h["parent_idx"], path, alen, every_visited)
-    tested = int((h["parent_idx"] >= 0).sum())
-    return rows * 8 * wl.vocab + tested * 12 + h["parent_idx"].size * 8
+    counts = wl.counts
+    tested = int((counts - 1).clip(min=0).sum())  # every node but the roots is a child
+    return rows * 8 * wl.vocab + tested * 12 + int(counts.sum()) * 8
 
 
 # ------------------------------------------------------------------ multi-rank plumbing
@@ -249,23 +251,27 @@ def job_throughput(world: int, nodes_per_step: int, steps: int, max_ms: float) -
 def workload_config(name: str, wl, world: int) -> dict:
     """The workload both arms of the bench report (same dict for each)."""
     N = wl.num_nodes
+    tree = (f"{N}-node tree" if wl.node_counts is None else
+            f"ragged trees of 1..{N} nodes ({int(wl.counts.sum())} in all; every fourth a chain)")
     return {"workload": f"{name}: batch {wl.batch}, prefix {int(wl.prefix_lens[0])}, "
                         f"Hq {wl.num_q_heads}/Hkv {wl.num_kv_heads}, D {wl.head_dim}, {wl.dtype}, "
-                        f"{N}-node tree, vocab {wl.vocab}",
+                        f"{tree}, vocab {wl.vocab}",
             "global_batch": world * wl.batch, "tree_nodes": N, "seq_len": int(wl.prefix_lens.max()) + N,
             "parallelism": f"replicas x{world} (independent sequences per GPU)",
             "l2": f"flushed before every step ({L2_FLUSH_BYTES >> 20} MB write, outside the step events)"}
 
 
-def deepest_paths(parent_idx: np.ndarray):
+def deepest_paths(parent_idx: np.ndarray, counts=None):
     """Each tree's deepest root-to-leaf path (root excluded), as a walk that
-    accepts every node on it would return it."""
+    accepts every node on it would return it; counts[b] limits sequence b's
+    tree to its first counts[b] nodes."""
     B, N = parent_idx.shape
     path = np.full((B, N), -1, np.int32)
     plen = np.zeros(B, np.int32)
     for b in range(B):
+        n = N if counts is None else int(counts[b])
         depth = np.zeros(N, np.int64)
-        for i in range(1, N):
+        for i in range(1, n):
             depth[i] = depth[parent_idx[b, i]] + 1
         node, nodes = int(np.argmax(depth)), []
         while node > 0:
@@ -281,12 +287,13 @@ def time_commit(tv, wl, d, flush, stream, W, K):
     """tv_commit_path (the step after verification) on copies of the caches,
     every tree's deepest path accepted; CUDA events, L2 flushed per call."""
     import torch
-    path, plen = deepest_paths(wl.parent_idx)
+    path, plen = deepest_paths(wl.parent_idx, wl.node_counts)
     kc, vc = d["k"].clone(), d["v"].clone()
     dpath = torch.from_numpy(path).cuda()
     dlen = torch.from_numpy(plen).cuda()
     new_pl = torch.empty_like(d["prefix_lens"])
-    call = lambda: tv.commit_path(kc, vc, d["block_table"], d["prefix_lens"], dpath, dlen, new_pl, stream=stream)
+    call = lambda: tv.commit_path(kc, vc, d["block_table"], d["prefix_lens"], dpath, dlen, new_pl, stream=stream,
+                                  node_counts=d.get("node_counts"))
     for _ in range(W):
         flush.zero_()
         call()
@@ -320,7 +327,7 @@ def time_logits_walk(tv, wl, d, flush, stream, W, K, ref):
     alen = torch.empty((B,), dtype=torch.int32, device="cuda")
     bonus = torch.empty((B,), dtype=torch.int32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    sdesc = tv.TvSampleDesc(B, N, wl.vocab)
+    sdesc = tv.TvSampleDesc(B, N, wl.vocab, tv._ptr(d.get("node_counts")))
 
     def call(st):
         s = tv.tv_verify_sample_logits(sdesc, dlp, dlq, d["tokens"], d["parent_idx"], d["uniforms"], path, alen,
@@ -378,11 +385,11 @@ def run_ours(args, rank, world, local_rank):
     alen = torch.empty((B,), dtype=torch.int32, device="cuda")
     bonus = torch.empty((B,), dtype=torch.int32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    adesc = tv.attn_desc(d["query"], d["k"], d["block_table"])
+    adesc = tv.attn_desc(d["query"], d["k"], d["block_table"], node_counts=d.get("node_counts"))
     aplan = tv.tv_tree_attention_plan(adesc)
     ws_bytes = aplan.workspace_bytes
     ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
-    sdesc = tv.TvSampleDesc(B, N, wl.vocab)
+    sdesc = tv.TvSampleDesc(B, N, wl.vocab, tv._ptr(d.get("node_counts")))
     splan = tv.tv_verify_sample_plan(sdesc)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
@@ -505,7 +512,7 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return None
 
-    nodes = B * N
+    nodes = int(wl.counts.sum())
     ms_step = total_ms / K
     value = job_throughput(world, nodes, K, total_ms)
     e2e_value = job_throughput(world, nodes, K2, e2e_ms)
@@ -564,6 +571,24 @@ def oracle_step_times(wl, h, rows_frac: float):
     the query rows (extrapolated to all rows) plus the full acceptance walk."""
     import oracle
     B, N, Hq = wl.batch, wl.num_nodes, wl.num_q_heads
+    if wl.node_counts is not None:
+        # ragged trees: each sequence is its own oracle problem over its own nodes
+        total_rows = int(wl.counts.sum()) * Hq
+        done = 0
+        t0 = time.perf_counter()
+        for b in range(B):
+            nb = int(wl.counts[b])
+            m = max(1, int(round(nb * Hq * rows_frac)))
+            sel = np.linspace(0, nb * Hq - 1, m).astype(np.int64)
+            rows = np.stack([np.zeros_like(sel), sel // Hq, sel % Hq], axis=1).astype(np.int32)
+            oracle.tree_attention(h["query"][b:b + 1, :nb], h["k"], h["v"], h["block_table"][b:b + 1],
+                                  h["prefix_lens"][b:b + 1], h["parent_idx"][b:b + 1, :nb], wl.num_kv_heads,
+                                  wl.dtype, rows=rows)
+            done += m
+        t_attn = (time.perf_counter() - t0) * total_rows / done
+        t0 = time.perf_counter()
+        oracle.verify_sample_ragged(h["p"], h["q"], h["tokens"], h["parent_idx"], h["uniforms"], wl.counts)
+        return t_attn + time.perf_counter() - t0, done, total_rows
     total_rows = B * N * Hq
     n = max(1, int(round(total_rows * rows_frac)))
     sel = np.linspace(0, total_rows - 1, n).astype(np.int64)
@@ -594,7 +619,7 @@ def cpu_baseline(wl, h, budget_s: float = 20.0):
         if frac >= 1.0 and time.perf_counter() - t_start > budget_s / 2:
             break
     per_step = t_sum / steps
-    return {"value": wl.batch * wl.num_nodes / per_step, "unit": "nodes/s", "cores": cores, "kind": "oracle",
+    return {"value": int(wl.counts.sum()) / per_step, "unit": "nodes/s", "cores": cores, "kind": "oracle",
             "sample": f"{steps} oracle step(s): attention on {rows_done // steps} of {total} query rows "
                       f"(time scaled to all rows) plus the full fp64 acceptance walk; "
                       f"{per_step * 1e3:.1f} ms per full step"}
@@ -617,7 +642,7 @@ def run_reference(args, rank, world):
         t, n_rows, total = oracle_step_times(wl, h, frac)
         times.append(t)
     per_step = sum(times) / K
-    value = wl.batch * wl.num_nodes / per_step
+    value = int(wl.counts.sum()) / per_step
     cores = oracle.max_threads()
     sample = (f"each step: oracle attention on {n_rows} of {total} query rows (time scaled to all rows) "
               f"plus the full fp64 acceptance walk")
@@ -636,7 +661,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default="l8b", choices=("tiny", "l8b", "l70b", "mix", "long"))
+    ap.add_argument("--workload", default="l8b", choices=("tiny", "l8b", "l70b", "mix", "long", "ragged"))
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -73,7 +73,17 @@ typedef enum { TV_BF16 = 0, TV_F32 = 1 } tv_dtype;
  *               sequence b lives in physical block block_table[b][j]
  *   prefix_lens [batch] int32: L_b, committed tokens before the tree
  *   parent_idx  [batch][num_nodes] int32: parent_idx[b][0] = -1 (the root,
- *               i.e. the last committed token), 0 <= parent_idx[b][i] < i
+ *               i.e. the last committed token), 0 <= parent_idx[b][i] < i;
+ *               NULL means every tree is a chain (parent of node i is i - 1:
+ *               linear speculation, whose mask is plain causal)
+ *   node_counts (descriptor field) [batch] int32 device array, or NULL: the
+ *               number n_b of tree nodes of sequence b, 0 <= n_b <= num_nodes
+ *               (ragged trees in one call; num_nodes is the capacity and the
+ *               row stride).  Nodes n_b .. num_nodes-1 are padding: their
+ *               parent_idx entries are ignored and their `out` rows are not
+ *               written; n_b = 0 leaves the sequence out of this step.  A count
+ *               outside [0, num_nodes] gives the sequence NaN rows and
+ *               TV_ERR_INVALID_ARG in *dev_status.  NULL = num_nodes for all b.
  * Node i's key/value sit at logical position L_b + i of the paged cache;
  * the caller writes them before the call.  Query head h reads KV head
  * h / (num_q_heads / num_kv_heads).  Row (b, i, h) of `out` is softmax
@@ -95,6 +105,7 @@ typedef struct {
     int32_t num_blocks;          /* physical blocks in paged_k / paged_v */
     int32_t dtype;               /* tv_dtype of q, paged_k, paged_v and out */
     float softmax_scale;         /* 0 => 1/sqrt(head_dim) */
+    const int32_t *node_counts;  /* device [batch] nodes per sequence, or NULL (= num_nodes each) */
 } tv_attn_desc;
 
 /* How a call will run (host-side query; launches nothing). */
@@ -158,7 +169,11 @@ TV_API tv_status tv_tree_attention_static(const tv_attn_desc *desc, const void *
  *                q[b][u] = draft distribution node u's children were drawn from
  *   tree_tokens  [batch][num_nodes] int32 draft token of each node (the
  *                root's entry is ignored)
- *   parent_idx   [batch][num_nodes] int32 as for tv_tree_attention
+ *   parent_idx   [batch][num_nodes] int32 as for tv_tree_attention (NULL:
+ *                chains)
+ *   node_counts  (descriptor field) as for tv_tree_attention: children at or
+ *                past n_b do not exist; n_b = 0 gives accepted_len 0, bonus
+ *                -1 and an all -1 path (no tree this step)
  *   uniforms     [batch][num_nodes] float32 in [0,1): uniforms[b][c] (c >= 1)
  *                is node c's acceptance draw, uniforms[b][0] the bonus draw
  * Walk: from the root, children of the current node u are tried in
@@ -174,12 +189,14 @@ TV_API tv_status tv_tree_attention_static(const tv_attn_desc *desc, const void *
  *                 excluded, in walk order, padded with -1
  *   accepted_len  [batch] int32, bonus_token [batch] int32
  * A malformed tree or token gives accepted_len = -1, bonus = -1 and
- * TV_ERR_TREE in *dev_status.
+ * TV_ERR_TREE in *dev_status (a node count outside [0, num_nodes]:
+ * TV_ERR_INVALID_ARG).
  */
 typedef struct {
     int32_t batch;
     int32_t num_nodes;           /* 1..1024 */
     int32_t vocab;               /* 1..221184 (16 CTAs x 13824 entries) */
+    const int32_t *node_counts;  /* device [batch] nodes per sequence, or NULL (= num_nodes each) */
 } tv_sample_desc;
 
 typedef struct {
@@ -200,7 +217,6 @@ TV_API tv_status tv_verify_sample(const tv_sample_desc *desc, const float *p, co
                            int32_t *bonus_token, void *workspace, size_t workspace_bytes,
                            int32_t *dev_status, void *stream);
 
-/* Static string for a status code. */
 /*
  * The acceptance walk on the two models' logits instead of their
  * distributions (the fused-logits form of tv_verify_sample).  Blog
@@ -244,7 +260,10 @@ TV_API tv_status tv_verify_sample_logits(const tv_sample_desc *desc, const float
  * prefix_lens[b]; new_prefix_lens[b] = prefix_lens[b] + 1 + n.  Positions from
  * the new length on hold nothing live: blocks wholly past it may be returned
  * to the caller's allocator (the block table is not changed).  accepted_len[b]
- * < 0 (a sequence the walk flagged) leaves the sequence unchanged.
+ * < 0 (a sequence the walk flagged) leaves the sequence unchanged.  With
+ * desc->node_counts, the tree of sequence b has n_b nodes: path entries must
+ * lie in [1, n_b), the span checked is L_b .. L_b + n_b - 1, and n_b = 0 with
+ * accepted_len 0 commits nothing.
  *
  * Arguments: desc as for tv_tree_attention (batch, num_nodes, num_kv_heads,
  * head_dim, block_size 16, max_blocks_per_seq, num_blocks and dtype are used;
@@ -268,6 +287,7 @@ TV_API tv_status tv_commit_path(const tv_attn_desc *desc, void *paged_k, void *p
                                 const int32_t *accepted_path, const int32_t *accepted_len,
                                 int32_t *new_prefix_lens, int32_t *dev_status, void *stream);
 
+/* Static string for a status code. */
 TV_API const char *tv_status_string(int32_t status);
 
 /* Library version: major * 10000 + minor * 100 + patch. */

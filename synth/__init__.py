@@ -24,6 +24,17 @@ mix   batch 64, prefix ~ U{512..32768}, Hq 32 / Hkv 8, D 128, bf16, paged,
 long  batch 1, prefix 131072, Hq 64 / Hkv 8, D 128, bf16, paged, 128-node
       greedy budget tree (depth <= 6, <= 4 children), vocab 128256, p/q as l8b
 ====  =====================================================================
+
+One more shape, outside the five (``RAGGED_NAMES``): mixed serving with trees
+of different sizes in one call.
+
+======  ===================================================================
+ragged  batch 32, prefix ~ U{512..32768}, Hq 32 / Hkv 8, D 128, bf16, paged,
+        capacity 32 nodes, n_b ~ U{1..32} nodes per sequence; every fourth
+        sequence a chain (linear speculation), the rest DFS trees of depth
+        U{2..6}; padding slots hold parent -1 and token -1; vocab 151936,
+        p/q as mix
+======  ===================================================================
 """
 from __future__ import annotations
 
@@ -258,14 +269,22 @@ class Workload:
     paged: bool
     row_keys: np.ndarray           # int64 [B][N]: generator row key of each node's p/q
     extra: dict = field(default_factory=dict)
+    node_counts: np.ndarray | None = None  # int32 [B] nodes per sequence (ragged workloads)
 
     @property
     def max_blocks(self) -> int:
         return int(self.block_table.shape[1])
 
     @property
+    def counts(self) -> np.ndarray:
+        """Nodes per sequence (num_nodes for every sequence unless ragged)."""
+        if self.node_counts is None:
+            return np.full(self.batch, self.num_nodes, dtype=np.int32)
+        return self.node_counts
+
+    @property
     def seq_tokens(self) -> np.ndarray:
-        return (self.prefix_lens + self.num_nodes).astype(np.int32)
+        return (self.prefix_lens + self.counts).astype(np.int32)
 
     # ---- attention inputs
     def query(self) -> np.ndarray:
@@ -312,8 +331,10 @@ class Workload:
 
 
 def _block_table(prefix_lens, n_nodes, permute, seed):
+    """n_nodes: one tree size for all sequences, or one per sequence."""
     B = len(prefix_lens)
-    nblk = [(int(L) + n_nodes + BLOCK_SIZE - 1) // BLOCK_SIZE for L in prefix_lens]
+    nn = np.broadcast_to(np.asarray(n_nodes), (B,))
+    nblk = [(int(L) + int(n) + BLOCK_SIZE - 1) // BLOCK_SIZE for L, n in zip(prefix_lens, nn)]
     total = sum(nblk)
     ids = np.arange(total, dtype=np.int64)
     if permute:  # Fisher-Yates driven by the PERM stream
@@ -331,6 +352,7 @@ def _block_table(prefix_lens, n_nodes, permute, seed):
 
 
 CONFIG_NAMES = ("tiny", "l8b", "l70b", "mix", "long")
+RAGGED_NAMES = ("ragged",)
 
 
 def make(name: str, seed: int | None = None, need_tokens: bool = True) -> Workload:
@@ -339,8 +361,10 @@ def make(name: str, seed: int | None = None, need_tokens: bool = True) -> Worklo
     Heavy tensors (KV cache, p/q) are produced on demand by the Workload
     methods so callers only pay for what they use.  ``seed`` defaults to the
     workload's index + 1."""
+    if name in RAGGED_NAMES:
+        return _make_ragged(name, 10 + RAGGED_NAMES.index(name) if seed is None else seed, need_tokens)
     if name not in CONFIG_NAMES:
-        raise ValueError(f"unknown workload {name!r}; choose from {CONFIG_NAMES}")
+        raise ValueError(f"unknown workload {name!r}; choose from {CONFIG_NAMES + RAGGED_NAMES}")
     if seed is None:
         seed = CONFIG_NAMES.index(name) + 1
     if name == "tiny":
@@ -408,6 +432,35 @@ def make(name: str, seed: int | None = None, need_tokens: bool = True) -> Worklo
                 for c in range(1, N):
                     toks[b, c] = categorical(q[b, parents[b, c]], float(u[b, c]))
         wl.tree_tokens = toks
+    return wl
+
+
+def _make_ragged(name: str, seed: int, need_tokens: bool) -> Workload:
+    B, N, Hq, Hkv, D, dt, V = 32, 32, 32, 8, 128, "bf16", 151936
+    u = uniforms(2 * B, seed, STREAM_LEN)
+    prefix = (512 + np.minimum((u[:B] * (32768 - 512 + 1)).astype(np.int64), 32768 - 512)).astype(np.int32)
+    counts = (1 + np.minimum((u[B:] * N).astype(np.int64), N - 1)).astype(np.int32)
+    parents = np.full((B, N), -1, dtype=np.int32)
+    for b in range(B):
+        n = int(counts[b])
+        if b % 4 == 3:
+            parents[b, :n] = np.arange(-1, n - 1)
+        else:
+            dr = _Draws(seed, STREAM_TREE, b << 20)
+            parents[b, :n] = dfs_tree(dr, n, dr.randint(2, 6))
+    row_keys = np.arange(B, dtype=np.int64)[:, None] * N + np.arange(N, dtype=np.int64)[None, :]
+    bt, nb = _block_table(prefix, counts, True, seed)
+    wl = Workload(name, B, N, Hq, Hkv, D, dt, V, prefix, bt, nb, parents, None, seed, float(1.0 / np.sqrt(128.0)),
+                  1, 4.0, 1.5, True, row_keys, {}, counts)
+    toks = np.full((B, N), -1, dtype=np.int32)
+    toks[:, 0] = 0
+    if need_tokens:
+        p, q = wl.pq()
+        ut = uniforms(B * N, seed, STREAM_TOKEN).reshape(B, N)
+        for b in range(B):
+            for c in range(1, int(counts[b])):
+                toks[b, c] = categorical(q[b, parents[b, c]], float(ut[b, c]))
+    wl.tree_tokens = toks
     return wl
 
 

@@ -99,7 +99,7 @@ def test_sampler_rejects_bad_descriptors(kw, status):
 
 def test_sampler_rejects_null_pointers():
     d = tv.TvSampleDesc(2, 8, 1000)
-    for i in range(8):
+    for i in (0, 1, 2, 4, 5, 6, 7):  # parent_idx (3) may be NULL: chains
         args = [256] * 8
         args[i] = 0
         assert tv.tv_verify_sample(d, *args, stream=0) == tv.TV_ERR_INVALID_ARG

@@ -29,3 +29,11 @@ def test_walk_rows_on_the_small_workload():
     p, q = wl.pq()
     r = oracle.verify_sample(p, q, wl.tree_tokens, wl.parent_idx, wl.uniforms())
     assert bench.walk_rows(wl.parent_idx, r["accepted_path"], r["accepted_len"]) == int(r["rows"].sum())
+
+
+def test_deepest_paths_respect_node_counts():
+    par = np.array([[-1, 0, 1, 2, -1, -1], [-1, 0, 0, 2, 3, 4]], np.int32)
+    path, plen = bench.deepest_paths(par, np.array([4, 3]))
+    # sequence 1 keeps nodes 0, 1 <- 0, 2 <- 0: depth 1 at best, first deepest node 1
+    assert plen.tolist() == [3, 1]
+    assert path[0, :3].tolist() == [1, 2, 3] and path[1, :1].tolist() == [1]

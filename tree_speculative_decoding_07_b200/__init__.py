@@ -29,7 +29,7 @@ class TvAttnDesc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("num_nodes", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("block_size", ctypes.c_int32),
                 ("max_blocks_per_seq", ctypes.c_int32), ("num_blocks", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("softmax_scale", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("node_counts", ctypes.c_void_p)]
 
 
 class TvAttnPlan(ctypes.Structure):
@@ -38,7 +38,8 @@ class TvAttnPlan(ctypes.Structure):
 
 
 class TvSampleDesc(ctypes.Structure):
-    _fields_ = [("batch", ctypes.c_int32), ("num_nodes", ctypes.c_int32), ("vocab", ctypes.c_int32)]
+    _fields_ = [("batch", ctypes.c_int32), ("num_nodes", ctypes.c_int32), ("vocab", ctypes.c_int32),
+                ("node_counts", ctypes.c_void_p)]
 
 
 class TvSamplePlan(ctypes.Structure):
@@ -180,9 +181,9 @@ def tv_commit_path(desc, paged_k, paged_v, block_table, prefix_lens, accepted_pa
 
 # ------------------------------------------------------------ torch conveniences
 
-def attn_desc(q, k_cache, block_table, softmax_scale: float = 0.0) -> TvAttnDesc:
+def attn_desc(q, k_cache, block_table, softmax_scale: float = 0.0, node_counts=None) -> TvAttnDesc:
     """Descriptor from tensors: q [B][N][Hq][D], cache [nb][16][Hkv][D],
-    block_table [B][max_blocks]."""
+    block_table [B][max_blocks], optional node_counts [B] int32 (ragged trees)."""
     import torch
     B, N, Hq, D = q.shape
     nb, bs, Hkv, D2 = k_cache.shape
@@ -191,7 +192,7 @@ def attn_desc(q, k_cache, block_table, softmax_scale: float = 0.0) -> TvAttnDesc
     dt = {torch.bfloat16: TV_BF16, torch.float32: TV_F32}.get(q.dtype)
     if dt is None:
         raise TypeError(f"unsupported dtype {q.dtype}")
-    return TvAttnDesc(B, N, Hq, Hkv, D, bs, block_table.shape[1], nb, dt, float(softmax_scale))
+    return TvAttnDesc(B, N, Hq, Hkv, D, bs, block_table.shape[1], nb, dt, float(softmax_scale), _ptr(node_counts))
 
 
 def _check_cuda(*ts):
@@ -201,16 +202,17 @@ def _check_cuda(*ts):
 
 
 def tree_attention(q, k_cache, v_cache, block_table, prefix_lens, parent_idx, softmax_scale: float = 0.0,
-                   out=None, workspace=None, dev_status=None, stream=None):
-    """Run tv_tree_attention; allocates `out` (and workspace) when not given."""
+                   out=None, workspace=None, dev_status=None, stream=None, node_counts=None):
+    """Run tv_tree_attention; allocates `out` (and workspace) when not given.
+    parent_idx None: every tree is a chain; node_counts [B]: ragged trees."""
     import torch
-    _check_cuda(q, k_cache, v_cache, block_table, prefix_lens, parent_idx, out, workspace, dev_status)
+    _check_cuda(q, k_cache, v_cache, block_table, prefix_lens, parent_idx, out, workspace, dev_status, node_counts)
     if k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
         raise TypeError("q, k_cache and v_cache must share a dtype")
-    for t in (block_table, prefix_lens, parent_idx):
-        if t.dtype != torch.int32:
-            raise TypeError("block_table, prefix_lens and parent_idx must be int32")
-    desc = attn_desc(q, k_cache, block_table, softmax_scale)
+    for t in (block_table, prefix_lens, parent_idx, node_counts):
+        if t is not None and t.dtype != torch.int32:
+            raise TypeError("block_table, prefix_lens, parent_idx and node_counts must be int32")
+    desc = attn_desc(q, k_cache, block_table, softmax_scale, node_counts)
     if out is None:
         out = torch.empty_like(q)
     ws_bytes = tv_tree_attention_workspace_size(desc)
@@ -224,11 +226,12 @@ def tree_attention(q, k_cache, v_cache, block_table, prefix_lens, parent_idx, so
 
 
 def verify_sample(p, q, tree_tokens, parent_idx, uniforms, accepted_path=None, accepted_len=None,
-                  bonus_token=None, dev_status=None, stream=None, logits: bool = False):
+                  bonus_token=None, dev_status=None, stream=None, logits: bool = False, node_counts=None):
     """Run tv_verify_sample (or, with logits=True, tv_verify_sample_logits on the
-    two models' logits); returns (accepted_path, accepted_len, bonus_token)."""
+    two models' logits); returns (accepted_path, accepted_len, bonus_token).
+    parent_idx None: every tree is a chain; node_counts [B]: ragged trees."""
     import torch
-    _check_cuda(p, q, tree_tokens, parent_idx, uniforms, dev_status)
+    _check_cuda(p, q, tree_tokens, parent_idx, uniforms, dev_status, node_counts)
     if p.dtype != torch.float32 or q.dtype != torch.float32 or uniforms.dtype != torch.float32:
         raise TypeError("p, q and uniforms must be float32")
     B, N, V = p.shape
@@ -239,7 +242,7 @@ def verify_sample(p, q, tree_tokens, parent_idx, uniforms, accepted_path=None, a
         accepted_len = torch.empty((B,), dtype=torch.int32, device=dev)
     if bonus_token is None:
         bonus_token = torch.empty((B,), dtype=torch.int32, device=dev)
-    desc = TvSampleDesc(B, N, V)
+    desc = TvSampleDesc(B, N, V, _ptr(node_counts))
     call = tv_verify_sample_logits if logits else tv_verify_sample
     s = call(desc, p, q, tree_tokens, parent_idx, uniforms, accepted_path, accepted_len, bonus_token, None, 0,
              dev_status, stream)
@@ -249,10 +252,11 @@ def verify_sample(p, q, tree_tokens, parent_idx, uniforms, accepted_path=None, a
 
 
 def commit_path(k_cache, v_cache, block_table, prefix_lens, accepted_path, accepted_len, new_prefix_lens=None,
-                dev_status=None, stream=None):
+                dev_status=None, stream=None, node_counts=None):
     """Run tv_commit_path on the caches in place; returns new_prefix_lens."""
     import torch
-    _check_cuda(k_cache, v_cache, block_table, prefix_lens, accepted_path, accepted_len, new_prefix_lens, dev_status)
+    _check_cuda(k_cache, v_cache, block_table, prefix_lens, accepted_path, accepted_len, new_prefix_lens, dev_status,
+                node_counts)
     for t in (block_table, prefix_lens, accepted_path, accepted_len):
         if t.dtype != torch.int32:
             raise TypeError("block_table, prefix_lens, accepted_path and accepted_len must be int32")
@@ -263,7 +267,7 @@ def commit_path(k_cache, v_cache, block_table, prefix_lens, accepted_path, accep
     dt = {torch.bfloat16: TV_BF16, torch.float32: TV_F32}.get(k_cache.dtype)
     if dt is None:
         raise TypeError(f"unsupported dtype {k_cache.dtype}")
-    desc = TvAttnDesc(B, N, hkv, hkv, d, bs, block_table.shape[1], nb, dt, 0.0)
+    desc = TvAttnDesc(B, N, hkv, hkv, d, bs, block_table.shape[1], nb, dt, 0.0, _ptr(node_counts))
     if new_prefix_lens is None:
         new_prefix_lens = torch.empty_like(prefix_lens)
     s = tv_commit_path(desc, k_cache, v_cache, block_table, prefix_lens, accepted_path, accepted_len,

@@ -112,12 +112,13 @@ tv_status verify_sample_common(const tv_sample_desc* desc, const float* p, const
                                bool logits) {
     tv_status s = check_sample_desc(desc);
     if (s != TV_OK) return s;
-    if (!p || !q || !tree_tokens || !parent_idx || !uniforms || !accepted_path || !accepted_len || !bonus_token)
+    if (!p || !q || !tree_tokens || !uniforms || !accepted_path || !accepted_len || !bonus_token)
         return TV_ERR_INVALID_ARG;
     tv_sample_plan plan;
     make_sample_plan(desc, &plan);
     tv::SampleArgs a = {};
-    a.p = p; a.q = q; a.tokens = tree_tokens; a.parent = parent_idx; a.uniforms = uniforms;
+    a.p = p; a.q = q; a.tokens = tree_tokens; a.parent = parent_idx; a.counts = desc->node_counts;
+    a.uniforms = uniforms;
     a.path = accepted_path; a.len = accepted_len; a.bonus = bonus_token; a.status = dev_status;
     a.B = desc->batch; a.N = desc->num_nodes; a.V = desc->vocab;
     a.cluster = plan.cluster_ctas; a.threads = plan.threads; a.slice = plan.slice; a.smem_bytes = plan.smem_bytes;
@@ -168,8 +169,7 @@ tv_status tv_tree_attention(const tv_attn_desc* desc, const void* q, const void*
                             void* stream) {
     tv_status s = check_attn_desc(desc);
     if (s != TV_OK) return s;
-    if (!q || !paged_k || !paged_v || !block_table || !prefix_lens || !parent_idx || !out)
-        return TV_ERR_INVALID_ARG;
+    if (!q || !paged_k || !paged_v || !block_table || !prefix_lens || !out) return TV_ERR_INVALID_ARG;
     tv_attn_plan plan;
     make_plan(desc, &plan);
     if (plan.kernel == 0) {
@@ -185,7 +185,7 @@ tv_status tv_tree_attention(const tv_attn_desc* desc, const void* q, const void*
     tv::AttnArgs a = {};
     a.q = q; a.k = paged_k; a.v = paged_v;
     a.block_table = block_table; a.prefix_lens = prefix_lens; a.parent = parent_idx;
-    a.out = out; a.status = dev_status;
+    a.counts = desc->node_counts; a.out = out; a.status = dev_status;
     a.B = desc->batch; a.N = desc->num_nodes; a.Hq = desc->num_q_heads; a.Hkv = desc->num_kv_heads;
     a.G = a.Hq / a.Hkv; a.D = desc->head_dim; a.max_blocks = desc->max_blocks_per_seq;
     a.num_blocks = desc->num_blocks; a.splits = plan.num_splits; a.row_tiles = plan.row_tiles;
@@ -235,7 +235,8 @@ tv_status tv_commit_path(const tv_attn_desc* desc, void* paged_k, void* paged_v,
     if ((reinterpret_cast<uintptr_t>(paged_k) | reinterpret_cast<uintptr_t>(paged_v)) & 15) return TV_ERR_INVALID_ARG;
     tv::CommitArgs a = {};
     a.k = paged_k; a.v = paged_v; a.block_table = block_table; a.prefix_lens = prefix_lens;
-    a.path = accepted_path; a.len = accepted_len; a.new_prefix_lens = new_prefix_lens; a.status = dev_status;
+    a.path = accepted_path; a.len = accepted_len; a.counts = desc->node_counts;
+    a.new_prefix_lens = new_prefix_lens; a.status = dev_status;
     a.B = desc->batch; a.N = desc->num_nodes; a.Hkv = desc->num_kv_heads;
     a.row_bytes = desc->head_dim * (desc->dtype == TV_BF16 ? 2 : 4);
     a.max_blocks = desc->max_blocks_per_seq; a.num_blocks = desc->num_blocks;

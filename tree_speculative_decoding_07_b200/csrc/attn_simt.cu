@@ -53,18 +53,23 @@ __global__ void __launch_bounds__(SIMT_WARPS * 32) attn_simt_kernel(AttnArgs a) 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int N = a.N, G = a.G;
     const int L = a.prefix_lens[b];
-    const int total = L + N;
-    const int rows_total = G * N;
+    bool bad_count;
+    const int n = seq_nodes(a.counts, b, N, bad_count);  // this sequence's tree nodes
+    const int total = L + n;
+    const int rows_total = G * n;
     const int r0 = tile * SIMT_ROWS;
+    if (!bad_count && r0 >= rows_total) return;  // a row tile past a short tree
 
-    if (tid == 0) s_bad = (L < 0 || (total + TV_BLOCK - 1) / TV_BLOCK > a.max_blocks) ? TV_ERR_BLOCK_TABLE : 0;
-    for (int i = tid; i < N; i += blockDim.x) par[i] = a.parent[(size_t)b * N + i];
+    if (tid == 0)
+        s_bad = bad_count ? TV_ERR_INVALID_ARG
+                          : (L < 0 || (total + TV_BLOCK - 1) / TV_BLOCK > a.max_blocks) ? TV_ERR_BLOCK_TABLE : 0;
+    for (int i = tid; i < n; i += blockDim.x) par[i] = parent_at(a.parent, b, N, i);
     __syncthreads();
-    for (int i = tid; i < N; i += blockDim.x)
+    for (int i = tid; i < n; i += blockDim.x)
         if (!parent_ok(par, i)) s_bad = TV_ERR_TREE;
     __syncthreads();
     const bool tree_bad = s_bad != 0;
-    for (int i = tid; i < N; i += blockDim.x) {
+    for (int i = tid; i < n; i += blockDim.x) {
         uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
         if (!tree_bad)
             for (int j = i; j >= 0; j = par[j]) {
@@ -180,6 +185,11 @@ template <typename T>
 __global__ void attn_combine_kernel(AttnArgs a) {
     const size_t row = blockIdx.x;
     const size_t rows = (size_t)a.B * a.N * a.Hq;
+    {
+        const int b = (int)(row / ((size_t)a.N * a.Hq)), node = (int)((row / a.Hq) % a.N);
+        bool bad_count;
+        if (node >= seq_nodes(a.counts, b, a.N, bad_count)) return;  // no such node in this sequence
+    }
     float mx = -INFINITY;
     bool nan = false;
     for (int s = 0; s < a.splits; ++s) {

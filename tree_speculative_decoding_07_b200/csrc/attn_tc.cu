@@ -88,6 +88,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int split = blockIdx.x, tile = blockIdx.y;
     const int b = blockIdx.z / a.Hkv, kvh = blockIdx.z % a.Hkv;
     const int N = a.N, G = a.G, S = a.splits;
+    // the prefix length and the sequence's node count decide everything below:
+    // both loads are issued before any set-up
+    const int L = a.prefix_lens[b];
+    bool bad_count;
+    const int n = seq_nodes(a.counts, b, N, bad_count);
+    // row tiles past a short tree have no rows; every split of such a tile leaves
+    // here, so no merge waits on it
+    if (!bad_count && tile * TM >= G * n) return;
     const uint32_t raw = smem_u32(dsmem);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* base_ptr = dsmem + (base - raw);
@@ -143,10 +151,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
         tc_fence_before();
     }
-    // the prefix length decides the split range and so the first block ids: it is
-    // loaded first, and the tree's parent array only after the id copies are issued
-    const int L = a.prefix_lens[b];
-    const int total = L + N;
+    // the prefix length decides the split range and so the first block ids; the
+    // tree's parent array is read only after the id copies are issued
+    const int total = L + n;
     const bool bad_len = L < 0 || (total + TV_BLOCK - 1) / TV_BLOCK > a.max_blocks;
     int t0, t1;
     split_range(bad_len ? 0 : total, S, split, t0, t1);
@@ -169,7 +176,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     };
     if (warp == 0 || warp == 3)
         for (int jt = 0; jt < ID_AHEAD; ++jt) prefetch_ids(jt);
-    for (int i = tid; i < N; i += TC_THREADS) s_par[i] = a.parent[(size_t)b * N + i];
+    for (int i = tid; i < n; i += TC_THREADS) s_par[i] = parent_at(a.parent, b, N, i);
     __syncthreads();
     // a kernel launched after this one with programmatic stream serialisation may
     // start its set-up now; it waits for this grid before reading anything
@@ -303,11 +310,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // ---------------- softmax groups: one thread per query row / TMEM lane
         const int st = tid - 128;  // 0..255
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        for (int i = st; i < N; i += 256)
+        for (int i = st; i < n; i += 256)
             if (!parent_ok(s_par, i)) s_bad = TV_ERR_TREE;
         if (st == 0 && bad_len) s_bad = TV_ERR_BLOCK_TABLE;
+        if (st == 0 && bad_count) s_bad = TV_ERR_INVALID_ARG;
         const int gr = tile * TM + r;
-        const bool row_ok = gr < G * N;
+        const bool row_ok = gr < G * n;
         const int node = row_ok ? gr / G : 0;
         const int head = kvh * G + (row_ok ? gr % G : 0);
         uint32_t an0 = 0, an1 = 0, an2 = 0, an3 = 0;
@@ -501,7 +509,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const int own = max(0, min(TM, (split + 1) * R) - split * R);
             for (int item = tid; item < own * (HD / 4); item += TC_THREADS) {
                 const int rt = split * R + item / (HD / 4), gr = tile * TM + rt;
-                if (gr >= G * N) continue;
+                if (gr >= G * n) continue;
                 const int node = gr / G, head = kvh * G + gr % G;
                 uint2 ov;
                 ov.x = pack_bf16(NAN, NAN);
@@ -511,21 +519,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
         } else
         switch (S) {
-            case 2: merge_rows<TM, TC_THREADS, 2>(a, part, split, tile, b, kvh, tid); break;
-            case 3: merge_rows<TM, TC_THREADS, 3>(a, part, split, tile, b, kvh, tid); break;
-            case 4: merge_rows<TM, TC_THREADS, 4>(a, part, split, tile, b, kvh, tid); break;
-            case 5: merge_rows<TM, TC_THREADS, 5>(a, part, split, tile, b, kvh, tid); break;
-            case 6: merge_rows<TM, TC_THREADS, 6>(a, part, split, tile, b, kvh, tid); break;
-            case 7: merge_rows<TM, TC_THREADS, 7>(a, part, split, tile, b, kvh, tid); break;
-            case 8: merge_rows<TM, TC_THREADS, 8>(a, part, split, tile, b, kvh, tid); break;
-            case 9: merge_rows<TM, TC_THREADS, 9>(a, part, split, tile, b, kvh, tid); break;
-            case 10: merge_rows<TM, TC_THREADS, 10>(a, part, split, tile, b, kvh, tid); break;
-            case 11: merge_rows<TM, TC_THREADS, 11>(a, part, split, tile, b, kvh, tid); break;
-            case 12: merge_rows<TM, TC_THREADS, 12>(a, part, split, tile, b, kvh, tid); break;
-            case 13: merge_rows<TM, TC_THREADS, 13>(a, part, split, tile, b, kvh, tid); break;
-            case 14: merge_rows<TM, TC_THREADS, 14>(a, part, split, tile, b, kvh, tid); break;
-            case 15: merge_rows<TM, TC_THREADS, 15>(a, part, split, tile, b, kvh, tid); break;
-            default: merge_rows<TM, TC_THREADS, 16>(a, part, split, tile, b, kvh, tid); break;
+            case 2: merge_rows<TM, TC_THREADS, 2>(a, part, split, tile, b, kvh, tid, G * n); break;
+            case 3: merge_rows<TM, TC_THREADS, 3>(a, part, split, tile, b, kvh, tid, G * n); break;
+            case 4: merge_rows<TM, TC_THREADS, 4>(a, part, split, tile, b, kvh, tid, G * n); break;
+            case 5: merge_rows<TM, TC_THREADS, 5>(a, part, split, tile, b, kvh, tid, G * n); break;
+            case 6: merge_rows<TM, TC_THREADS, 6>(a, part, split, tile, b, kvh, tid, G * n); break;
+            case 7: merge_rows<TM, TC_THREADS, 7>(a, part, split, tile, b, kvh, tid, G * n); break;
+            case 8: merge_rows<TM, TC_THREADS, 8>(a, part, split, tile, b, kvh, tid, G * n); break;
+            case 9: merge_rows<TM, TC_THREADS, 9>(a, part, split, tile, b, kvh, tid, G * n); break;
+            case 10: merge_rows<TM, TC_THREADS, 10>(a, part, split, tile, b, kvh, tid, G * n); break;
+            case 11: merge_rows<TM, TC_THREADS, 11>(a, part, split, tile, b, kvh, tid, G * n); break;
+            case 12: merge_rows<TM, TC_THREADS, 12>(a, part, split, tile, b, kvh, tid, G * n); break;
+            case 13: merge_rows<TM, TC_THREADS, 13>(a, part, split, tile, b, kvh, tid, G * n); break;
+            case 14: merge_rows<TM, TC_THREADS, 14>(a, part, split, tile, b, kvh, tid, G * n); break;
+            case 15: merge_rows<TM, TC_THREADS, 15>(a, part, split, tile, b, kvh, tid, G * n); break;
+            default: merge_rows<TM, TC_THREADS, 16>(a, part, split, tile, b, kvh, tid, G * n); break;
         }
         __syncthreads();
         if (tid == 0 && atomicAdd(arrive + 1, 1u) == (unsigned)(S - 1)) {

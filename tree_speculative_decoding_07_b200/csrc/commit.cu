@@ -29,23 +29,27 @@ __global__ void __launch_bounds__(CM_THREADS) commit_kernel(const CommitArgs a) 
     const int N = a.N;
     const int L = a.prefix_lens[b];
     const int n = a.len[b];
+    bool bad_count;
+    const int nodes = seq_nodes(a.counts, b, N, bad_count);  // this sequence's tree nodes
     const int32_t* path = a.path + (size_t)b * N;
     const int32_t* bt = a.block_table + (size_t)b * a.max_blocks;
     const bool lead = h == 0 && tid == 0;
-    if (n < 0) {  // flagged by the walk: nothing is committed
+    if (n < 0 || (nodes == 0 && n == 0 && !bad_count)) {
+        // flagged by the walk, or no tree this step: nothing is committed
         if (lead) a.new_prefix_lens[b] = L;
         return;
     }
     // validation, identical in every CTA of the sequence
     int bad = 0;
-    if (L < 0 || n > N - 1 || (long long)L + N > (long long)a.max_blocks * TV_BLOCK) bad = TV_ERR_INVALID_ARG;
+    if (bad_count || L < 0 || n > nodes - 1 || (long long)L + nodes > (long long)a.max_blocks * TV_BLOCK)
+        bad = TV_ERR_INVALID_ARG;
     if (!bad)
         for (int k = tid; k < n; k += CM_THREADS) {
             const int prev = k == 0 ? 0 : path[k - 1];
-            if (path[k] <= prev || path[k] >= N) bad = TV_ERR_TREE;
+            if (path[k] <= prev || path[k] >= nodes) bad = TV_ERR_TREE;
         }
     if (!bad)
-        for (int bi = L / TV_BLOCK + tid; bi <= (L + N - 1) / TV_BLOCK; bi += CM_THREADS) {
+        for (int bi = L / TV_BLOCK + tid; bi <= (L + nodes - 1) / TV_BLOCK; bi += CM_THREADS) {
             const int id = bt[bi];
             if (id < 0 || id >= a.num_blocks) bad = TV_ERR_BLOCK_TABLE;
         }

@@ -12,7 +12,8 @@ struct AttnArgs {
     const void* v;
     const int32_t* block_table;
     const int32_t* prefix_lens;
-    const int32_t* parent;
+    const int32_t* parent;  // [B][N]; NULL: every tree is a chain (parent of node i is i - 1)
+    const int32_t* counts;  // [B] nodes per sequence (0..N); NULL: N for every sequence
     void* out;
     float* o_part;      // CUDA-core path: [splits][B][N][Hq][D] fp32 partial outputs (normalised);
                         // tensor-core path: [groups][splits][128] partial rows of 272 bytes
@@ -40,7 +41,8 @@ struct SampleArgs {
     const float* p;
     const float* q;
     const int32_t* tokens;
-    const int32_t* parent;
+    const int32_t* parent;  // [B][N]; NULL: every tree is a chain
+    const int32_t* counts;  // [B] nodes per sequence (0..N); NULL: N for every sequence
     const float* uniforms;
     int32_t* path;
     int32_t* len;
@@ -62,6 +64,7 @@ struct CommitArgs {
     const int32_t* prefix_lens;
     const int32_t* path;   // [B][N] accepted node indices, root excluded
     const int32_t* len;    // [B] accepted lengths (< 0: flagged, no commit)
+    const int32_t* counts; // [B] tree nodes per sequence (0..N); NULL: N for every sequence
     int32_t* new_prefix_lens;
     int32_t* status;
     int B, N, Hkv, row_bytes, max_blocks, num_blocks;

@@ -52,6 +52,9 @@ struct SampleShared {
     double warp_part2[MAX_THREADS / 32];
     double peer[2][MAX_CLUSTER];   // values from every CTA of the cluster, by exchange parity
     double peer2[2][MAX_CLUSTER];  // second values of two-value exchanges
+    // logits mode: the softmax of the row in buffer x is p = exp(l - row_mp[x]) * row_zp_inv[x]
+    double row_zp_inv[2], row_zq_inv[2];
+    float row_mp[2], row_mq[2];
     unsigned long long peer_bar[2];
     unsigned long long row_bar[2];
     int timeout;
@@ -143,9 +146,6 @@ struct Walker {
     int passes;      // cluster exchanges so far
     int row_uses[2];
     bool row_pending[2];
-    // logits mode: the softmax of the row in buffer x is p = exp(l - mp) * zp_inv
-    float row_mp[2], row_mq[2];
-    double row_zp_inv[2], row_zq_inv[2];
 
     __device__ float* ps(int x) const { return buf + (size_t)2 * x * a.slice; }
     __device__ float* qs(int x) const { return ps(x) + a.slice; }
@@ -231,7 +231,7 @@ struct Walker {
     // the C values with the same shuffle tree -- sums, or maxima when take_max -- so
     // all CTAs and all warps obtain the same bits and take the same branches.  The
     // per-CTA values stay in sh.peer / sh.peer2 at the parity of the exchange.
-    __device__ void exchange(int nv, double v0, double v1, bool take_max, double& r0, double& r1) {
+    __device__ __forceinline__ void exchange(int nv, double v0, double v1, bool take_max, double& r0, double& r1) {
         const int par = passes & 1;
         const uint32_t use = (uint32_t)(passes >> 1);
         ++passes;
@@ -320,11 +320,13 @@ struct Walker {
             pl[i] = (float)((double)pl[i] * zpi);
             ql[i] = (float)((double)ql[i] * zqi);
         }
+        if (tid == 0) {
+            sh.row_mp[x] = mpf;
+            sh.row_mq[x] = mqf;
+            sh.row_zp_inv[x] = zpi;
+            sh.row_zq_inv[x] = zqi;
+        }
         __syncthreads();
-        row_mp[x] = mpf;
-        row_mq[x] = mqf;
-        row_zp_inv[x] = zpi;
-        row_zq_inv[x] = zqi;
     }
 };
 
@@ -355,14 +357,15 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
     Walker w{a, sh, reinterpret_cast<float*>(sample_dyn), b, rank, C, lo, n, tid, lane, warp, nwarps,
-             ((n + nwarps - 1) / nwarps + 127) / 128 * 128, a.vec4 != 0, 0, {0, 0}, {false, false},
-             {0.f, 0.f}, {0.f, 0.f}, {0.0, 0.0}, {0.0, 0.0}};
+             ((n + nwarps - 1) / nwarps + 127) / 128 * 128, a.vec4 != 0, 0, {0, 0}, {false, false}};
     // the root's row is needed unless its first child is accepted: start it now
     w.issue_row(0, 0);
 
     // ---- tree and tokens; a malformed sequence gets -1 outputs
-    for (int i = tid; i < N; i += blockDim.x) {
-        sh.parent[i] = a.parent[(size_t)b * N + i];
+    bool bad_count;
+    const int nn = seq_nodes(a.counts, b, N, bad_count);  // this sequence's tree nodes
+    for (int i = tid; i < nn; i += blockDim.x) {
+        sh.parent[i] = parent_at(a.parent, b, N, i);
         sh.token[i] = a.tokens[(size_t)b * N + i];
     }
     // every CTA's barriers must exist before a peer pushes to them (the first pass);
@@ -372,18 +375,21 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
     else
         __syncthreads();
     bool bad_local = false;
-    for (int i = tid; i < N; i += blockDim.x) {
+    for (int i = tid; i < nn; i += blockDim.x) {
         const int p = sh.parent[i];
         bad_local |= (i == 0) ? p != -1 : (p < 0 || p >= i || sh.token[i] < 0 || sh.token[i] >= a.V);
     }
     int32_t* path_out = a.path + (size_t)b * N;
-    if (__syncthreads_or(bad_local)) {
+    if (__syncthreads_or(bad_local) || bad_count || nn == 0) {
+        // a malformed sequence gets -1 outputs; an empty one (no tree this step)
+        // accepts nothing and draws no token
         if (rank == 0) {
             for (int i = tid; i < N; i += blockDim.x) path_out[i] = -1;
             if (tid == 0) {
-                a.len[b] = -1;
+                const bool empty = nn == 0 && !bad_count;
+                a.len[b] = empty ? 0 : -1;
                 a.bonus[b] = -1;
-                report(a.status, TV_ERR_TREE);
+                if (!empty) report(a.status, bad_count ? TV_ERR_INVALID_ARG : TV_ERR_TREE);
             }
         }
         w.wait_row(0);
@@ -405,14 +411,14 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
             w.wait_row(x);
             w.prep_row(x);
         }
-        while (accepted < 0 && scan < N) {
+        while (accepted < 0 && scan < nn) {
             // warp 0 collects the next (up to 32) children of u in ascending order and
             // gathers their draft tokens' p, q and acceptance draws
             if (warp == 0) {
-                int found = 0, next = N;
-                for (int c0 = scan; c0 < N; c0 += 32) {
+                int found = 0, next = nn;
+                for (int c0 = scan; c0 < nn; c0 += 32) {
                     const int c = c0 + lane;
-                    const bool kid = c < N && sh.parent[c] == u;
+                    const bool kid = c < nn && sh.parent[c] == u;
                     const unsigned m = __ballot_sync(0xffffffffu, kid);
                     const int pos = found + __popc(m & ((1u << lane) - 1u));
                     if (kid && pos < 32) sh.ch_node[pos] = c;
@@ -431,10 +437,10 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
                     const int c = sh.ch_node[lane];
                     const size_t row = ((size_t)b * N + u) * (size_t)a.V;
                     if (LOGITS) {
-                        const float ep = expf(__ldg(a.p + row + sh.token[c]) - w.row_mp[x]);
-                        const float eq = expf(__ldg(a.q + row + sh.token[c]) - w.row_mq[x]);
-                        sh.ch_p[lane] = (double)(float)((double)ep * w.row_zp_inv[x]);
-                        sh.ch_q[lane] = (double)(float)((double)eq * w.row_zq_inv[x]);
+                        const float ep = expf(__ldg(a.p + row + sh.token[c]) - sh.row_mp[x]);
+                        const float eq = expf(__ldg(a.q + row + sh.token[c]) - sh.row_mq[x]);
+                        sh.ch_p[lane] = (double)(float)((double)ep * sh.row_zp_inv[x]);
+                        sh.ch_q[lane] = (double)(float)((double)eq * sh.row_zq_inv[x]);
                     } else {
                         sh.ch_p[lane] = (double)__ldg(a.p + row + sh.token[c]);
                         sh.ch_q[lane] = (double)__ldg(a.q + row + sh.token[c]);

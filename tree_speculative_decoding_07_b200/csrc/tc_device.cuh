@@ -213,7 +213,7 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
 // Each item is 8 columns of one row, so a thread issues all its loads at once.
 template <int ROWS, int THREADS, int S_>
 __device__ __forceinline__ void merge_rows(const AttnArgs& a, const uint8_t* part, int split, int tile, int b, int kvh,
-                                           int tid) {
+                                           int tid, int nrows) {
     constexpr int R = (ROWS + S_ - 1) / S_;
     constexpr int NC = HD / 8;
     const int own = max(0, min(ROWS, (split + 1) * R) - split * R);
@@ -221,7 +221,7 @@ __device__ __forceinline__ void merge_rows(const AttnArgs& a, const uint8_t* par
         const int rr = item / NC, cc = item % NC;
         const int rt = split * R + rr;
         const int gr = tile * ROWS + rt;
-        if (gr >= a.G * a.N) continue;
+        if (gr >= nrows) continue;  // rows of nodes past the sequence's tree
         float ls[S_];
         uint4 v[S_];
 #pragma unroll

@@ -30,6 +30,24 @@ template <> struct Elem<__nv_bfloat16> {
 // A tree is well formed when node 0 is the root (parent -1) and every other
 // node's parent precedes it; then ancestor walks terminate and the nodes are
 // in topological order.
+// Nodes of sequence b: counts[b], or N when no counts are given.  A count
+// outside [0, N] sets `bad` and yields N (the caller reports the error and
+// writes no valid output for the sequence).
+__device__ __forceinline__ int seq_nodes(const int32_t* counts, int b, int N, bool& bad) {
+    if (!counts) {
+        bad = false;
+        return N;
+    }
+    const int n = counts[b];
+    bad = n < 0 || n > N;
+    return bad ? N : n;
+}
+
+// Parent of node i of sequence b; a NULL parent array means a chain.
+__device__ __forceinline__ int32_t parent_at(const int32_t* parent, int b, int N, int i) {
+    return parent ? parent[(size_t)b * N + i] : i - 1;
+}
+
 __device__ __forceinline__ bool parent_ok(const int32_t* parent, int i) {
     int p = parent[i];
     return i == 0 ? p == -1 : (p >= 0 && p < i);
