@@ -18,8 +18,21 @@ decoding):
   Acceptance Condition"), applied root-down with sibling retries (glossary,
   "SpecInfer").
 
+* :func:`verify_sample_logits` -- the same walk on the row softmax of the two
+  models' logits (p and q are the models' output distributions).
+* :func:`commit_path` -- the accepted path joins the cached prefix (blog,
+  "KV cache management and prefix sharing"; glossary, "KV cache management
+  challenges").
+* :func:`tree_attention_ragged`, :func:`verify_sample_ragged`,
+  :func:`commit_path_ragged`, :func:`chain_parents` -- ragged batches (each
+  sequence its own tree) and chains (linear speculation).
+* :func:`topk_rows`, :func:`fill_topk_tokens` -- top-k branching (glossary,
+  tree-structure optimisation, "Top-k branching").
+* :func:`tree_shape_dp`, :func:`tree_value` -- the budget-constrained tree shape
+  by dynamic programming (glossary, "Budget-constrained optimisation").
+
 Every function is pinned by ``tests/test_oracle_*.py`` against values the
-pages print, closed forms and library routines.
+pages print, closed forms, exhaustive search and library routines.
 """
 from __future__ import annotations
 
@@ -252,6 +265,123 @@ def commit_path_ragged(k_cache, v_cache, block_table, prefix_lens, accepted_path
         new_pl[b] = npl[0]
         st = st or s
     return k, v, new_pl, st
+
+
+def topk_rows(x, k: int):
+    """Top-k of each row of x [..][V]: (indices, values), values descending and
+    equal values by ascending index (a stable sort of -x)."""
+    x = np.asarray(x)
+    V = x.shape[-1]
+    flat = x.reshape(-1, V)
+    idx = np.empty((flat.shape[0], k), np.int32)
+    for r in range(flat.shape[0]):
+        idx[r] = np.argsort(-flat[r].astype(np.float64), kind="stable")[:k]
+    vals = np.take_along_axis(flat, idx.astype(np.int64), axis=1)
+    return idx.reshape(x.shape[:-1] + (k,)), vals.reshape(x.shape[:-1] + (k,))
+
+
+def fill_topk_tokens(q, parent_idx, rank, node_counts=None) -> np.ndarray:
+    """Top-k branching (glossary "Tree-based speculative decoding", section on
+    tree-structure optimisation, "Top-k branching": each node expands the draft
+    model's top-k tokens as its children).  Child c of node u with rank r gets
+    the r-th most probable token of u's draft distribution q[b][u] (r = 0 the
+    most probable; ties by lower token id).  Returns tree_tokens [B][N] with
+    the root's entry 0 and padding nodes -1."""
+    q = np.asarray(q)
+    B, N, V = q.shape
+    par = np.asarray(parent_idx, np.int32)
+    rk = np.asarray(rank, np.int32)
+    tokens = np.full((B, N), -1, np.int32)
+    for b in range(B):
+        n = N if node_counts is None else int(node_counts[b])
+        if n == 0:
+            continue
+        tokens[b, 0] = 0
+        for u in range(n):
+            kids = [c for c in range(1, n) if par[b, c] == u]
+            if not kids:
+                continue
+            kk = max(int(rk[b, c]) for c in kids) + 1
+            idx, _ = topk_rows(q[b, u], kk)
+            for c in kids:
+                tokens[b, c] = idx[int(rk[b, c])]
+    return tokens
+
+
+def tree_value(parent, rank, accept) -> float:
+    """Expected accepted tokens of a tree under positional acceptance: the sum
+    over non-root nodes of the product, along the root path, of accept[rank] of
+    each edge (the rank-r candidate of a node is accepted with probability
+    accept[r], whatever the depth)."""
+    n = len(parent)
+    reach = np.zeros(n)
+    reach[0] = 1.0
+    for c in range(1, n):
+        reach[c] = reach[parent[c]] * accept[rank[c]]
+    return float(reach[1:].sum())
+
+
+def tree_shape_dp(accept, budget: int, max_depth: int | None = None):
+    """Budget-constrained tree shape (glossary, "Budget-constrained
+    optimisation": allocate branches under a node budget so that the whole
+    tree's expected accepted tokens is largest; solved by dynamic programming,
+    as Sequoia does).  accept[r] is the probability that a node's rank-r
+    candidate is accepted (positional acceptance, independent of depth); a node
+    has children of ranks 0..m-1 (m <= len(accept)); the tree has at most
+    `budget` nodes (root included) and depth at most max_depth.
+
+    F[d][n]: best value of a subtree of exactly n nodes with at most d levels
+    below its root; G[i][s]: best value of children of ranks i.. holding s
+    nodes in all.  F[d][n] = G[0][n - 1] with G[i][s] = max over t of
+    accept[i] * (1 + F[d-1][t]) + G[i+1][s-t].  Ties go to the smallest t and
+    the smallest total size.  Returns (parent, rank, value): nodes numbered by
+    depth, then by the ranks along their path."""
+    accept = [float(a) for a in accept]
+    k = len(accept)
+    D = budget - 1 if max_depth is None else min(max_depth, budget - 1)
+    NEG = float("-inf")
+    F = [[NEG] * (budget + 1) for _ in range(D + 1)]
+    choice = [None] * (D + 1)  # choice[d][i][s] = t
+    for d in range(D + 1):
+        F[d][1] = 0.0
+        if d == 0:
+            continue
+        G = [[NEG] * budget for _ in range(k + 1)]
+        ch = [[0] * budget for _ in range(k + 1)]
+        G[k][0] = 0.0
+        for i in range(k - 1, -1, -1):
+            G[i][0] = 0.0
+            for s in range(1, budget):
+                best, arg = NEG, 0
+                for t in range(1, s + 1):
+                    if F[d - 1][t] == NEG or G[i + 1][s - t] == NEG:
+                        continue
+                    v = accept[i] * (1.0 + F[d - 1][t]) + G[i + 1][s - t]
+                    if v > best:
+                        best, arg = v, t
+                G[i][s], ch[i][s] = best, arg
+        for n in range(2, budget + 1):
+            F[d][n] = G[0][n - 1]
+        choice[d] = ch
+    n_best = max(range(1, budget + 1), key=lambda n: (F[D][n], -n))
+    # rebuild: children of a node with d levels and n nodes, rank by rank
+    paths = []  # (path of ranks, ) for every node
+
+    def build(path, d, n):
+        paths.append(path)
+        s, i = n - 1, 0
+        while s > 0:
+            t = choice[d][i][s]
+            build(path + (i,), d - 1, t)
+            s -= t
+            i += 1
+
+    build((), D, n_best)
+    paths.sort(key=lambda pth: (len(pth), pth))
+    index = {pth: j for j, pth in enumerate(paths)}
+    parent = np.array([-1] + [index[pth[:-1]] for pth in paths[1:]], np.int32)
+    rank = np.array([-1] + [pth[-1] for pth in paths[1:]], np.int32)
+    return parent, rank, F[D][n_best]
 
 
 def softmax_rows(logits) -> np.ndarray:

@@ -1,0 +1,110 @@
+"""Pins for the oracle's tree construction: top-k branching and the
+budget-constrained shape (glossary "Tree-based speculative decoding", the
+section on tree-structure optimisation: "Top-k branching" and
+"Budget-constrained optimisation", solved by dynamic programming).
+
+Pins: top-k against a brute-force sort and hand-made ties; the filled tokens
+on a hand-worked tree; the DP against exhaustive enumeration of every tree
+within the budget; a width-1 budget against the pages' chain formula
+(1 - a^(g+1)) / (1 - a) (glossary, "linear vs tree" table); the depth cap;
+monotonicity in the budget."""
+import itertools
+
+import numpy as np
+import pytest
+
+import oracle
+
+
+def test_topk_rows_against_brute_force_and_ties():
+    x = np.array([[0.1, 0.5, 0.2, 0.5, 0.0, 0.2]], np.float32)
+    idx, val = oracle.topk_rows(x, 4)
+    assert idx.tolist() == [[1, 3, 2, 5]]  # equal values: lower index first
+    np.testing.assert_array_equal(val, x[:, [1, 3, 2, 5]])
+    rng = np.random.default_rng(1)
+    y = rng.integers(0, 5, (20, 30)).astype(np.float32)  # many ties
+    idx, _ = oracle.topk_rows(y, 7)
+    for r in range(20):
+        want = sorted(range(30), key=lambda i: (-y[r, i], i))[:7]
+        assert idx[r].tolist() == want
+
+
+def test_fill_topk_tokens_hand_example():
+    # root -> {1 (rank 0), 2 (rank 1)}, 1 -> {3 (rank 0)}; node 2 and 3 are leaves
+    q = np.zeros((1, 4, 6), np.float32)
+    q[0, 0] = [0.1, 0.3, 0.05, 0.3, 0.2, 0.05]    # order 1, 3, 4, 0, ...
+    q[0, 1] = [0.0, 0.0, 0.0, 0.0, 0.0, 1.0]      # order 5, ...
+    q[0, 2] = q[0, 3] = 1.0 / 6                    # leaves: never read
+    parent = np.array([[-1, 0, 0, 1]], np.int32)
+    rank = np.array([[-1, 0, 1, 0]], np.int32)
+    assert oracle.fill_topk_tokens(q, parent, rank).tolist() == [[0, 1, 3, 5]]
+    # ragged: a one-node tree has only its root
+    assert oracle.fill_topk_tokens(q, parent, rank, node_counts=[1]).tolist() == [[0, -1, -1, -1]]
+
+
+def _all_trees(budget, k, depth):
+    """Every tree (as (parent, rank)) with at most `budget` nodes, children of
+    ranks 0..m-1 (m <= k) and depth <= `depth`."""
+    def subtrees(n, d):
+        # ordered child lists for a root with exactly n nodes
+        if n == 1:
+            yield []
+            return
+        if d == 0:
+            return
+        for m in range(1, k + 1):
+            for sizes in itertools.product(range(1, n), repeat=m):
+                if sum(sizes) != n - 1:
+                    continue
+                for kids in itertools.product(*[list(subtrees(s, d - 1)) for s in sizes]):
+                    yield list(kids)
+
+    for n in range(1, budget + 1):
+        for t in subtrees(n, depth):
+            parent, rank = [-1], [-1]
+
+            def walk(children, me):
+                for r, ch in enumerate(children):
+                    parent.append(me)
+                    rank.append(r)
+                    walk(ch, len(parent) - 1)
+
+            walk(t, 0)
+            yield parent, rank
+
+
+@pytest.mark.parametrize("accept,budget,depth", [
+    ([0.6, 0.25, 0.1], 7, 6), ([0.9, 0.05], 7, 3), ([0.5, 0.3, 0.15], 6, 2), ([0.35, 0.3, 0.2], 7, 6),
+    ([0.8], 5, 4),
+])
+def test_dp_equals_exhaustive_search(accept, budget, depth):
+    best = max(oracle.tree_value(p, r, accept) for p, r in _all_trees(budget, len(accept), depth))
+    parent, rank, value = oracle.tree_shape_dp(accept, budget, depth)
+    assert abs(value - best) <= 1e-12
+    assert abs(oracle.tree_value(parent, rank, accept) - value) <= 1e-12
+    # the returned tree obeys the constraints and is numbered parent-first
+    n = len(parent)
+    assert n <= budget and parent[0] == -1 and all(0 <= parent[c] < c for c in range(1, n))
+    depth_of = [0] * n
+    for c in range(1, n):
+        depth_of[c] = depth_of[parent[c]] + 1
+    assert max(depth_of) <= depth
+    for u in range(n):
+        ranks = sorted(rank[c] for c in range(1, n) if parent[c] == u)
+        assert ranks == list(range(len(ranks))) and len(ranks) <= len(accept)
+
+
+@pytest.mark.parametrize("a,n", [(0.5, 2), (0.7, 6), (0.9, 12), (0.3, 9)])
+def test_width_one_budget_is_the_chain_formula(a, n):
+    parent, rank, value = oracle.tree_shape_dp([a], n)
+    assert parent.tolist() == [-1] + list(range(n - 1))
+    # emitted tokens per step = accepted + the bonus: (1 - a^(g+1)) / (1 - a), g = n - 1 drafts
+    assert abs((1.0 + value) - (1 - a ** n) / (1 - a)) <= 1e-12
+
+
+def test_depth_cap_and_budget_monotonicity():
+    parent, rank, value = oracle.tree_shape_dp([0.8], 10, max_depth=3)
+    assert len(parent) == 4 and abs(value - (0.8 + 0.64 + 0.512)) <= 1e-12
+    acc = [0.55, 0.2, 0.1, 0.05]
+    vals = [oracle.tree_shape_dp(acc, n, 5)[2] for n in range(1, 25)]
+    assert all(b >= a for a, b in zip(vals, vals[1:]))
