@@ -364,6 +364,50 @@ def time_logits_walk(tv, wl, d, flush, stream, W, K, ref):
                     "before each"}
 
 
+def time_fill_topk(tv, wl, d, flush, stream, W, K):
+    """tv_tree_fill_topk (top-k branching: every child's token from its parent's
+    draft row, ranks = sibling order) on the workload's own tree and q rows,
+    timed alone from its own graph with L2 flushed before each launch."""
+    import torch
+    B, N = wl.batch, wl.num_nodes
+    tokens = torch.empty((B, N), dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    desc = tv.TvSampleDesc(B, N, wl.vocab, tv._ptr(d.get("node_counts")))
+
+    def call(st):
+        s = tv.tv_tree_fill_topk(desc, d["q"], d["parent_idx"], None, tokens, status, st)
+        if s:
+            raise tv.TreeVerifyError(s, "tv_tree_fill_topk")
+
+    call(stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call(torch.cuda.current_stream())
+    for _ in range(W):
+        flush.zero_()
+        g.replay()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} from the top-k fill")
+    us = float(np.mean([e0.elapsed_time(e1) for e0, e1 in evs])) * 1e3
+    internal = 0
+    for b in range(B):
+        n = int(wl.counts[b])
+        internal += len({int(x) for x in wl.parent_idx[b, 1:n]})
+    nbytes = internal * wl.vocab * 4 + int(wl.counts.sum()) * 8
+    del g
+    return {"us": us, "rows": internal, "bytes": nbytes, "achieved_gbs": nbytes / (us * 1e-6) / 1e9 if us else None,
+            "note": "tv_tree_fill_topk on the workload's tree (each internal node's q row read once); mean over "
+                    "launches, L2 flushed before each"}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -470,6 +514,7 @@ def run_ours(args, rank, world, local_rank):
     walk = {"path": path.cpu().numpy(), "alen": alen.cpu().numpy(), "bonus": bonus.cpu().numpy()}
     commit = time_commit(tv, wl, d, flush, stream, W, min(K, 200))
     logits_walk = time_logits_walk(tv, wl, d, flush, stream, W, min(K, 200), walk)
+    fill = time_fill_topk(tv, wl, d, flush, stream, W, min(K, 200))
     total_ms = float(sum(step_ms))
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())}")
@@ -553,6 +598,7 @@ def run_ours(args, rank, world, local_rank):
         "median_us_per_step": float(np.median(step_ms)) * 1e3,
         "commit": commit,
         "sample_logits": logits_walk,
+        "tree_fill_topk": fill,
         "e2e": {"value": e2e_value, "unit": "nodes/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": K2},
         "gpu_launches": K * (aplan.launches + splan.launches),

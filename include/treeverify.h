@@ -287,6 +287,64 @@ TV_API tv_status tv_commit_path(const tv_attn_desc *desc, void *paged_k, void *p
                                 const int32_t *accepted_path, const int32_t *accepted_len,
                                 int32_t *new_prefix_lens, int32_t *dev_status, void *stream);
 
+/*
+ * Building the draft tree: top-k branching.  Glossary "Tree-based speculative
+ * decoding", section on tree-structure optimisation, "Top-k branching": each
+ * node expands the draft model's k most probable tokens as its children.
+ *
+ * For every node u of every sequence b that has children, child c receives the
+ * rank[b][c]-th most probable token of q[b][u] (rank 0 = the most probable;
+ * equal values rank the lower token id first; -0.0 ranks below +0.0):
+ * tree_tokens[b][c] = that token id.  Only the rows of nodes with children are
+ * read; the root's entry and padding entries of tree_tokens are not written.
+ *   desc         batch, num_nodes (capacity, <= 1024), vocab, node_counts as for
+ *                tv_verify_sample
+ *   q            [batch][num_nodes][vocab] float32 device: u's draft
+ *                distribution, or its logits (same order); no NaN
+ *   parent_idx   [batch][num_nodes] int32 device, or NULL (chains)
+ *   rank         [batch][num_nodes] int32 device, or NULL: then a child's rank is
+ *                its position among its siblings in ascending node index
+ *   tree_tokens  [batch][num_nodes] int32 device, written for children
+ * A node may have at most 32 children and ranks lie in [0, 32) and below
+ * vocab; otherwise that node's children get token -1.  A malformed tree (or a
+ * bad node count) sets every child entry of the sequence to -1.  Both write
+ * TV_ERR_TREE (TV_ERR_INVALID_ARG for a count) to *dev_status.  One launch on
+ * `stream`; nothing is allocated.
+ */
+TV_API tv_status tv_tree_fill_topk(const tv_sample_desc *desc, const float *q, const int32_t *parent_idx,
+                                   const int32_t *rank, int32_t *tree_tokens, int32_t *dev_status,
+                                   void *stream);
+
+/*
+ * Building the draft tree: the budget-constrained shape.  Glossary, same
+ * section, "Budget-constrained optimisation": under a node budget, allocate the
+ * branches so that the whole tree's expected number of accepted tokens is
+ * largest; dynamic programming solves it (as Sequoia does at run time).
+ *
+ * Model: accept[r] is the probability that a node's rank-r candidate is
+ * accepted, the same at every depth (positional acceptance); a node's children
+ * have ranks 0 .. m-1 with m <= num_ranks; a tree's value is the sum over its
+ * non-root nodes of the product of accept[rank] along the root path (the
+ * expected accepted tokens; one more token, the bonus, is always emitted).  The
+ * call returns a tree of at most `budget` nodes (root included) and depth at
+ * most max_depth (0 = no cap) with the largest value.  Ties go to the smaller
+ * subtree sizes in rank order and then to the smaller tree.
+ *   accept             num_ranks host doubles in [0, 1]
+ *   parent_idx, rank   host int32 arrays of `budget` entries, written: nodes
+ *                      numbered by depth, then by the ranks along their path
+ *                      (parents before children, siblings in rank order, so
+ *                      the output feeds tv_tree_fill_topk and the verifier);
+ *                      root parent -1 and rank -1; entries past the tree -1
+ *   num_nodes          host int32, written: the tree's size
+ *   expected_accepted  host double, written: the tree's value
+ * Host computation only (no device work): num_ranks <= 32, budget <= 256,
+ * else TV_ERR_UNSUPPORTED; a null pointer, budget < 1, max_depth < 0 or an
+ * accept value outside [0, 1]: TV_ERR_INVALID_ARG.
+ */
+TV_API tv_status tv_tree_shape(const double *accept, int32_t num_ranks, int32_t budget, int32_t max_depth,
+                               int32_t *parent_idx, int32_t *rank, int32_t *num_nodes,
+                               double *expected_accepted);
+
 /* Static string for a status code. */
 TV_API const char *tv_status_string(int32_t status);
 

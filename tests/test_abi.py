@@ -126,3 +126,10 @@ def test_commit_rejects_bad_arguments_before_launch():
     assert tv.tv_commit_path(d, a + 8, a, a, a, a, a, a + 64, stream=0) == tv.TV_ERR_INVALID_ARG
     bad = _desc(head_dim=96)
     assert tv.tv_commit_path(bad, a, a, a, a, a, a, a + 64, stream=0) == tv.TV_ERR_UNSUPPORTED
+
+
+def test_fill_topk_rejects_bad_arguments_before_launch():
+    assert tv.tv_tree_fill_topk(tv.TvSampleDesc(0, 4, 10), 256, 256, 256, 256, stream=0) == tv.TV_ERR_INVALID_ARG
+    assert tv.tv_tree_fill_topk(tv.TvSampleDesc(1, 4, 10), None, 256, 256, 256, stream=0) == tv.TV_ERR_INVALID_ARG
+    assert tv.tv_tree_fill_topk(tv.TvSampleDesc(1, 4, 10), 256, 256, 256, None, stream=0) == tv.TV_ERR_INVALID_ARG
+    assert tv.tv_tree_fill_topk(tv.TvSampleDesc(1, 1025, 10), 256, 256, 256, 256, stream=0) == tv.TV_ERR_UNSUPPORTED

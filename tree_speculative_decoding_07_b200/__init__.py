@@ -76,11 +76,14 @@ def lib() -> ctypes.CDLL:
         L.tv_verify_sample.argtypes = [ctypes.POINTER(TvSampleDesc), P, P, P, P, P, P, P, P, P, sz, P, P]
         L.tv_commit_path.argtypes = [ctypes.POINTER(TvAttnDesc), P, P, P, P, P, P, P, P, P]
         L.tv_verify_sample_logits.argtypes = [ctypes.POINTER(TvSampleDesc), P, P, P, P, P, P, P, P, P, sz, P, P]
+        L.tv_tree_fill_topk.argtypes = [ctypes.POINTER(TvSampleDesc), P, P, P, P, P, P]
+        L.tv_tree_shape.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, P, P]
         L.tv_status_string.argtypes = [ctypes.c_int32]
         L.tv_status_string.restype = ctypes.c_char_p
         L.tv_version.restype = ctypes.c_int32
         for name in ("tv_tree_attention_plan", "tv_tree_attention", "tv_tree_attention_static",
-                     "tv_verify_sample_plan", "tv_verify_sample", "tv_commit_path", "tv_verify_sample_logits"):
+                     "tv_verify_sample_plan", "tv_verify_sample", "tv_commit_path", "tv_verify_sample_logits",
+                     "tv_tree_fill_topk", "tv_tree_shape"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -170,6 +173,58 @@ def tv_verify_sample_logits(desc, target_logits, draft_logits, tree_tokens, pare
                                              _ptr(accepted_path), _ptr(accepted_len), _ptr(bonus_token),
                                              _ptr(workspace), int(workspace_bytes), _ptr(dev_status),
                                              _stream(stream)))
+
+
+def tv_tree_fill_topk(desc, q, parent_idx, rank, tree_tokens, dev_status=None, stream=None) -> int:
+    return int(lib().tv_tree_fill_topk(ctypes.byref(desc), _ptr(q), _ptr(parent_idx), _ptr(rank), _ptr(tree_tokens),
+                                       _ptr(dev_status), _stream(stream)))
+
+
+def tv_tree_shape(accept, num_ranks: int, budget: int, max_depth: int, parent_idx, rank, num_nodes,
+                  expected_accepted) -> int:
+    """Host pointers (numpy arrays or ctypes addresses)."""
+    return int(lib().tv_tree_shape(_hptr(accept), int(num_ranks), int(budget), int(max_depth), _hptr(parent_idx),
+                                   _hptr(rank), _hptr(num_nodes), _hptr(expected_accepted)))
+
+
+def _hptr(a):
+    if a is None:
+        return None
+    if isinstance(a, int):
+        return ctypes.c_void_p(a)
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def tree_shape(accept, budget: int, max_depth: int = 0):
+    """Budget-constrained tree shape; returns (parent_idx, rank, expected_accepted)
+    as numpy arrays trimmed to the tree's size."""
+    import numpy as np
+    acc = np.ascontiguousarray(accept, dtype=np.float64)
+    parent = np.empty(max(int(budget), 1), np.int32)
+    rank = np.empty_like(parent)
+    n = np.zeros(1, np.int32)
+    val = np.zeros(1, np.float64)
+    s = tv_tree_shape(acc, acc.size, budget, max_depth, parent, rank, n, val)
+    if s != TV_OK:
+        raise TreeVerifyError(s, "tv_tree_shape")
+    return parent[:n[0]].copy(), rank[:n[0]].copy(), float(val[0])
+
+
+def fill_topk(q, parent_idx=None, rank=None, tree_tokens=None, node_counts=None, dev_status=None, stream=None):
+    """Run tv_tree_fill_topk; returns tree_tokens (allocated, filled with -1, when
+    not given)."""
+    import torch
+    _check_cuda(q, parent_idx, rank, tree_tokens, node_counts, dev_status)
+    if q.dtype != torch.float32:
+        raise TypeError("q must be float32")
+    B, N, V = q.shape
+    if tree_tokens is None:
+        tree_tokens = torch.full((B, N), -1, dtype=torch.int32, device=q.device)
+    desc = TvSampleDesc(B, N, V, _ptr(node_counts))
+    s = tv_tree_fill_topk(desc, q, parent_idx, rank, tree_tokens, dev_status, stream)
+    if s != TV_OK:
+        raise TreeVerifyError(s, "tv_tree_fill_topk")
+    return tree_tokens
 
 
 def tv_commit_path(desc, paged_k, paged_v, block_table, prefix_lens, accepted_path, accepted_len, new_prefix_lens,

@@ -16,6 +16,8 @@ NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
     "--expt-relaxed-constexpr",
+    # host arithmetic rounds each operation (the tree-shape DP compares sums exactly)
+    "-Xcompiler", "-ffp-contract=off",
 ]
 
 

@@ -244,6 +244,32 @@ tv_status tv_commit_path(const tv_attn_desc* desc, void* paged_k, void* paged_v,
 }
 
 
+tv_status tv_tree_fill_topk(const tv_sample_desc* desc, const float* q, const int32_t* parent_idx,
+                            const int32_t* rank, int32_t* tree_tokens, int32_t* dev_status, void* stream) {
+    tv_status s = check_sample_desc(desc);
+    if (s != TV_OK) return s;
+    if (!q || !tree_tokens) return TV_ERR_INVALID_ARG;
+    tv::FillArgs a = {};
+    a.q = q; a.parent = parent_idx; a.rank = rank; a.counts = desc->node_counts; a.tokens = tree_tokens;
+    a.status = dev_status;
+    a.B = desc->batch; a.N = desc->num_nodes; a.V = desc->vocab;
+    tv::fill_topk_plan(a.V, &a.cluster, &a.slice, &a.smem_bytes);
+    if ((int64_t)a.cluster * a.B * a.N > INT32_MAX) return TV_ERR_UNSUPPORTED;
+    a.vec4 = (a.V % 4 == 0) && !(reinterpret_cast<uintptr_t>(q) & 15);
+    return tv::launch_fill_topk(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? TV_OK : TV_ERR_CUDA;
+}
+
+tv_status tv_tree_shape(const double* accept, int32_t num_ranks, int32_t budget, int32_t max_depth,
+                        int32_t* parent_idx, int32_t* rank, int32_t* num_nodes, double* expected_accepted) {
+    if (!accept || !parent_idx || !rank || !num_nodes || !expected_accepted) return TV_ERR_INVALID_ARG;
+    if (num_ranks < 1 || budget < 1 || max_depth < 0) return TV_ERR_INVALID_ARG;
+    if (num_ranks > 32 || budget > 256) return TV_ERR_UNSUPPORTED;
+    for (int i = 0; i < num_ranks; ++i)
+        if (!(accept[i] >= 0.0 && accept[i] <= 1.0)) return TV_ERR_INVALID_ARG;
+    *num_nodes = tv::tree_shape_dp(accept, num_ranks, budget, max_depth, parent_idx, rank, expected_accepted);
+    return TV_OK;
+}
+
 tv_status tv_verify_sample(const tv_sample_desc* desc, const float* p, const float* q, const int32_t* tree_tokens,
                            const int32_t* parent_idx, const float* uniforms, int32_t* accepted_path,
                            int32_t* accepted_len, int32_t* bonus_token, void* workspace, size_t workspace_bytes,

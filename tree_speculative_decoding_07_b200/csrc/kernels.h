@@ -73,4 +73,22 @@ cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st);
 size_t commit_smem_bytes(int N, int row_bytes);
 int sample_max_cluster();
 
+// Top-k branching: child tokens from each parent's draft distribution (one launch).
+struct FillArgs {
+    const float* q;          // [B][N][V] draft distributions (or logits: the order is the same)
+    const int32_t* parent;   // [B][N]; NULL: chains
+    const int32_t* rank;     // [B][N] child ranks; NULL: a child's position among its siblings
+    const int32_t* counts;   // [B] nodes per sequence; NULL: N
+    int32_t* tokens;         // [B][N] written for children only
+    int32_t* status;
+    int B, N, V;
+    int cluster, slice, smem_bytes, vec4;
+};
+void fill_topk_plan(int V, int* cluster, int* slice, int* smem_bytes);
+cudaError_t launch_fill_topk(const FillArgs& a, cudaStream_t st);
+
+// Budget-constrained tree shape (host).  Returns the node count.
+int tree_shape_dp(const double* accept, int k, int budget, int max_depth, int32_t* parent, int32_t* rank,
+                  double* value);
+
 }  // namespace tv

@@ -1,0 +1,349 @@
+// treebuild.cu -- building the draft tree the verifier checks (glossary
+// "Tree-based speculative decoding", section on tree-structure optimisation):
+//
+//  * top-k branching: each node expands the draft model's k most probable
+//    tokens as its children.  fill_topk_kernel gives child c of node u the
+//    rank(c)-th most probable token of u's draft distribution (ties to the
+//    lower token id), reading only the rows of nodes that have children.
+//  * budget-constrained optimisation: under a node budget, allocate branches so
+//    the whole tree's expected accepted tokens is largest, by dynamic
+//    programming (tree_shape_dp, host code: the table is small).
+//
+// fill_topk_kernel: one thread-block cluster per (sequence, node).  Each CTA of
+// the cluster stages its slice of the node's row in shared memory, finds the
+// slice's top kk (kk = the largest child rank + 1) by kk rounds of a block-wide
+// maximum over 64-bit keys (value bits mapped to an unsigned order in the high
+// half, the complemented token id in the low half, so equal values rank the
+// lower id first), and stores its kk keys into the lead CTA's shared memory;
+// the lead CTA merges the C * kk keys the same way and writes the children's
+// tokens.  Clusters of leaves leave after reading the tree.
+#include <cooperative_groups.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "kernels.h"
+#include "tv_common.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace tv {
+namespace {
+
+constexpr int FT_THREADS = 256;
+constexpr int FT_MAX_K = 32;        // largest child rank + 1
+constexpr int FT_MAX_CLUSTER = 16;
+
+// float -> unsigned with the same order (negative values below positive ones)
+__device__ __forceinline__ uint32_t ordered_bits(float v) {
+    const uint32_t u = __float_as_uint(v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ unsigned long long make_key(float v, int idx) {
+    return ((unsigned long long)ordered_bits(v) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)idx);
+}
+
+__device__ __forceinline__ int key_index(unsigned long long k) {
+    return (int)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
+}
+
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
+        v = w > v ? w : v;
+    }
+    return v;
+}
+
+struct FillShared {
+    int32_t parent[1024];
+    int32_t kid[FT_MAX_K];                                   // children of the node, ascending
+    int32_t kid_rank[FT_MAX_K];
+    unsigned long long warp_best[FT_THREADS / 32];
+    unsigned long long mine[FT_MAX_K];                       // this CTA's top kk
+    unsigned long long all[FT_MAX_CLUSTER * FT_MAX_K];       // lead CTA: every CTA's top kk
+    int nkids, kk;
+    int bad;        // the whole sequence is malformed (count or tree): no child entry is valid
+    int bad_node;   // this node's children cannot be expanded (too many, or a bad rank)
+};
+
+// Largest key below `below` held by this thread in its elements of `vals`
+// (index base + i for vals[i]), then the block-wide maximum.
+__device__ unsigned long long block_max_below(const float* vals, int count, int base, unsigned long long below,
+                                              FillShared& sh) {
+    unsigned long long best = 0ull;
+    for (int i = threadIdx.x; i < count; i += FT_THREADS) {
+        const unsigned long long k = make_key(vals[i], base + i);
+        if (k < below && k > best) best = k;
+    }
+    best = warp_max_u64(best);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) sh.warp_best[warp] = best;
+    __syncthreads();
+    unsigned long long r = lane < FT_THREADS / 32 ? sh.warp_best[lane] : 0ull;
+    r = warp_max_u64(r);
+    __syncthreads();  // warp_best is reused by the next round
+    return r;
+}
+
+__global__ void __launch_bounds__(FT_THREADS) fill_topk_kernel(const FillArgs a) {
+    extern __shared__ float4 ft_dyn[];
+    float* slice = reinterpret_cast<float*>(ft_dyn);
+    __shared__ FillShared sh;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int C = a.cluster;
+    const int crank = C > 1 ? (int)cluster.block_rank() : 0;
+    const int row = blockIdx.x / C;            // (sequence, node)
+    const int b = row / a.N, u = row % a.N;
+    const int tid = threadIdx.x;
+    const int N = a.N;
+
+    bool bad_count;
+    const int n = seq_nodes(a.counts, b, N, bad_count);
+    for (int i = tid; i < n; i += FT_THREADS) sh.parent[i] = parent_at(a.parent, b, N, i);
+    if (tid == 0) {
+        sh.nkids = 0;
+        sh.bad = bad_count ? TV_ERR_INVALID_ARG : 0;
+        sh.bad_node = 0;
+    }
+    __syncthreads();
+    int bad_local = 0;
+    for (int i = tid; i < n; i += FT_THREADS)
+        if (!parent_ok(sh.parent, i)) bad_local = TV_ERR_TREE;
+    if (bad_local) atomicMax(&sh.bad, bad_local);
+    // children of u in ascending index, by one warp (ballots keep the order)
+    if (tid < 32 && !bad_count && u < n) {
+        int found = 0;
+        for (int c0 = u + 1; c0 < n; c0 += 32) {
+            const int c = c0 + tid;
+            const bool kid = c < n && sh.parent[c] == u;
+            const unsigned m = __ballot_sync(0xffffffffu, kid);
+            const int pos = found + __popc(m & ((1u << tid) - 1u));
+            if (kid && pos < FT_MAX_K) {
+                sh.kid[pos] = c;
+                sh.kid_rank[pos] = a.rank ? a.rank[(size_t)b * N + c] : pos;
+            }
+            found += __popc(m);
+        }
+        if (tid == 0) sh.nkids = found;
+    }
+    __syncthreads();
+    const int nk = sh.nkids;
+    if (tid == 0 && !sh.bad) {
+        int kk = 0, err = nk > FT_MAX_K ? TV_ERR_TREE : 0;
+        for (int j = 0; j < min(nk, FT_MAX_K); ++j) {
+            const int r = sh.kid_rank[j];
+            if (r < 0 || r >= FT_MAX_K || r >= a.V) err = TV_ERR_TREE;
+            kk = max(kk, r + 1);
+        }
+        sh.kk = kk;
+        sh.bad_node = err;
+    }
+    __syncthreads();
+    if (sh.bad) {
+        // a malformed sequence: every cluster of it sees the same, and the root's
+        // cluster alone clears all of its child entries and reports
+        if (u == 0 && crank == 0) {
+            for (int c = 1 + tid; c < min(n, N); c += FT_THREADS) a.tokens[(size_t)b * N + c] = -1;
+            if (tid == 0) report(a.status, sh.bad);
+        }
+        return;
+    }
+    if (sh.bad_node) {
+        // this node's children (all of them, also past the first 32) get -1
+        if (crank == 0) {
+            for (int c = u + 1 + tid; c < n; c += FT_THREADS)
+                if (sh.parent[c] == u) a.tokens[(size_t)b * N + c] = -1;
+            if (tid == 0) report(a.status, sh.bad_node);
+        }
+        return;
+    }
+    if (u >= n || nk == 0) return;  // no such node, or a leaf: nothing to expand (cluster-uniform)
+    const int kk = sh.kk;
+
+    // ---- this CTA's slice of u's draft row, staged in shared memory
+    const int lo = min(a.V, crank * a.slice);
+    const int cnt = min(a.V, lo + a.slice) - lo;
+    const float* src = a.q + ((size_t)b * N + u) * (size_t)a.V + lo;
+    if (a.vec4) {
+        const float4* s4 = reinterpret_cast<const float4*>(src);
+        for (int i = tid; i < cnt / 4; i += FT_THREADS) ft_dyn[i] = __ldg(s4 + i);
+        for (int i = (cnt & ~3) + tid; i < cnt; i += FT_THREADS) slice[i] = __ldg(src + i);
+    } else {
+        for (int i = tid; i < cnt; i += FT_THREADS) slice[i] = __ldg(src + i);
+    }
+    __syncthreads();
+    // ---- the slice's top kk keys (0 = none: the slice has fewer entries)
+    unsigned long long below = ~0ull;
+    for (int r = 0; r < kk; ++r) {
+        const unsigned long long k = block_max_below(slice, cnt, lo, below, sh);
+        if (tid == 0) sh.mine[r] = k;
+        below = k;
+    }
+    __syncthreads();
+    // ---- gather every CTA's keys in the lead CTA
+    if (C > 1) {
+        cluster.sync();  // every CTA of the cluster is running before shared memory is shared
+        unsigned long long* dst = cluster.map_shared_rank(sh.all, 0);
+        for (int r = tid; r < kk; r += FT_THREADS) dst[crank * FT_MAX_K + r] = sh.mine[r];
+        cluster.sync();  // the stores are visible to the lead CTA
+        if (crank != 0) return;
+    } else {
+        for (int r = tid; r < kk; r += FT_THREADS) sh.all[r] = sh.mine[r];
+        __syncthreads();
+    }
+    // ---- lead CTA: merge C * kk keys, rank by rank, and write the children's tokens
+    if (tid < 32) {
+        unsigned long long prev = ~0ull;
+        const int total = C * FT_MAX_K;
+        for (int r = 0; r < kk; ++r) {
+            unsigned long long best = 0ull;
+            for (int i = tid; i < total; i += 32) {
+                const int cr = i / FT_MAX_K, j = i % FT_MAX_K;
+                if (j >= kk || cr >= C) continue;
+                const unsigned long long k = sh.all[i];
+                if (k < prev && k > best) best = k;
+            }
+            best = warp_max_u64(best);
+            if (tid == 0) sh.mine[r] = best;
+            prev = best;
+        }
+        __syncwarp();
+        for (int j = tid; j < nk; j += 32) {
+            const unsigned long long k = sh.mine[sh.kid_rank[j]];
+            a.tokens[(size_t)b * N + sh.kid[j]] = k ? key_index(k) : -1;
+        }
+    }
+}
+
+}  // namespace
+
+void fill_topk_plan(int V, int* cluster, int* slice, int* smem_bytes) {
+    int c = (V + 8191) / 8192;
+    if (c > FT_MAX_CLUSTER) c = FT_MAX_CLUSTER;
+    if (c < 1) c = 1;
+    int s = (V + c - 1) / c;
+    s = (s + 3) / 4 * 4;
+    *cluster = c;
+    *slice = s;
+    *smem_bytes = (int)(sizeof(float) * (size_t)s);
+}
+
+cudaError_t launch_fill_topk(const FillArgs& a, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(fill_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, a.smem_bytes);
+    if (e != cudaSuccess) return e;
+    if (a.cluster > 8) {
+        e = cudaFuncSetAttribute(fill_topk_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3((unsigned)a.cluster * (unsigned)a.B * (unsigned)a.N, 1, 1);
+    cfg.blockDim = dim3(FT_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = a.smem_bytes;
+    cfg.stream = st;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = a.cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.cluster > 1 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, fill_topk_kernel, a);
+}
+
+// ---------------------------------------------------------------- budget DP
+
+// F[d][n]: best expected accepted tokens of a subtree of exactly n nodes with at
+// most d levels below its root; G[i][s]: best value of the children of ranks
+// i.. holding s nodes in all:  G[i][s] = max_t accept[i] (1 + F[d-1][t]) +
+// G[i+1][s-t], F[d][n] = G[0][n-1].  Ties go to the smallest t, and among equal
+// totals to the smallest tree.  Nodes are numbered by depth, then by the ranks
+// along their path.
+int tree_shape_dp(const double* accept, int k, int budget, int max_depth, int32_t* parent, int32_t* rank,
+                  double* value) {
+    const double NEG = -INFINITY;
+    const int D = (max_depth <= 0 || max_depth > budget - 1) ? budget - 1 : max_depth;
+    std::vector<std::vector<double>> F(D + 1, std::vector<double>(budget + 1, NEG));
+    // choice[d][i * budget + s] = t
+    std::vector<std::vector<int32_t>> choice(D + 1);
+    std::vector<double> G((size_t)(k + 1) * budget), Gnext;
+    for (int d = 0; d <= D; ++d) {
+        F[d][1] = 0.0;
+        if (d == 0) continue;
+        std::vector<int32_t>& ch = choice[d];
+        ch.assign((size_t)(k + 1) * budget, 0);
+        std::fill(G.begin(), G.end(), NEG);
+        G[(size_t)k * budget + 0] = 0.0;
+        for (int i = k - 1; i >= 0; --i) {
+            double* gi = &G[(size_t)i * budget];
+            const double* gn = &G[(size_t)(i + 1) * budget];
+            gi[0] = 0.0;
+            for (int s = 1; s < budget; ++s) {
+                double best = NEG;
+                int arg = 0;
+                for (int t = 1; t <= s; ++t) {
+                    const double f = F[d - 1][t], g = gn[s - t];
+                    if (f == NEG || g == NEG) continue;
+                    const double grow = 1.0 + f;
+                    const double take = accept[i] * grow;
+                    const double v = take + g;
+                    if (v > best) {
+                        best = v;
+                        arg = t;
+                    }
+                }
+                gi[s] = best;
+                ch[(size_t)i * budget + s] = arg;
+            }
+        }
+        for (int nn = 2; nn <= budget; ++nn) F[d][nn] = G[nn - 1];
+    }
+    int n_best = 1;
+    for (int nn = 2; nn <= budget; ++nn)
+        if (F[D][nn] > F[D][n_best]) n_best = nn;
+    // rebuild the rank paths of every node
+    std::vector<std::vector<int>> paths;
+    struct Item { std::vector<int> path; int d, n; };
+    std::vector<Item> stack{{{}, D, n_best}};
+    while (!stack.empty()) {
+        Item it = stack.back();
+        stack.pop_back();
+        paths.push_back(it.path);
+        int s = it.n - 1, i = 0;
+        while (s > 0) {
+            const int t = choice[it.d][(size_t)i * budget + s];
+            std::vector<int> p = it.path;
+            p.push_back(i);
+            stack.push_back({p, it.d - 1, t});
+            s -= t;
+            ++i;
+        }
+    }
+    std::sort(paths.begin(), paths.end(), [](const std::vector<int>& x, const std::vector<int>& y) {
+        if (x.size() != y.size()) return x.size() < y.size();
+        return x < y;
+    });
+    const int n = (int)paths.size();
+    for (int j = 0; j < budget; ++j) {
+        parent[j] = -1;
+        rank[j] = -1;
+    }
+    for (int j = 1; j < n; ++j) {
+        std::vector<int> up(paths[j].begin(), paths[j].end() - 1);
+        // the parent's path is shorter, so it sits before j in the sorted list
+        const int p = (int)(std::lower_bound(paths.begin(), paths.begin() + j, up,
+                                             [](const std::vector<int>& x, const std::vector<int>& y) {
+                                                 if (x.size() != y.size()) return x.size() < y.size();
+                                                 return x < y;
+                                             }) -
+                            paths.begin());
+        parent[j] = p;
+        rank[j] = paths[j].back();
+    }
+    *value = F[D][n_best];
+    return n;
+}
+
+}  // namespace tv
