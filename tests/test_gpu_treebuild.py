@@ -124,3 +124,16 @@ def test_shape_tokens_walk_end_to_end():
     torch.cuda.synchronize()
     got = {"accepted_path": path.cpu().numpy(), "accepted_len": alen.cpu().numpy(), "bonus_token": bonus.cpu().numpy()}
     compare_sampler(got, oracle.verify_sample(p, q, tokens, parent, u))
+
+
+@pytest.mark.parametrize("V", [40, 5000, 151936])
+def test_wide_nodes_take_several_passes(V):
+    """A root with 32 children (ranks 0..31) and a node with 12 (ranks past 8
+    take more than one pass over the row), on tie-heavy rows."""
+    N = 45
+    parent = np.array([[-1] + [0] * 32 + [1] * 12] * 2, np.int32)
+    rng = np.random.default_rng(V)
+    q = rng.integers(0, 10, (2, N, V)).astype(np.float32)
+    q[1] = rng.random((N, V)).astype(np.float32)
+    _check(q, parent, _sibling_ranks(parent))
+    _check(q, parent, None)

@@ -10,13 +10,14 @@
 //    programming (tree_shape_dp, host code: the table is small).
 //
 // fill_topk_kernel: one thread-block cluster per (sequence, node).  Each CTA of
-// the cluster stages its slice of the node's row in shared memory, finds the
-// slice's top kk (kk = the largest child rank + 1) by kk rounds of a block-wide
-// maximum over 64-bit keys (value bits mapped to an unsigned order in the high
-// half, the complemented token id in the low half, so equal values rank the
-// lower id first), and stores its kk keys into the lead CTA's shared memory;
-// the lead CTA merges the C * kk keys the same way and writes the children's
-// tokens.  Clusters of leaves leave after reading the tree.
+// the cluster reads its slice of the node's row once, every thread keeping its
+// own top K (K = kk rounded up to a power of two, kk = the largest child rank +
+// 1) of 64-bit keys in registers (value bits mapped to an unsigned order in the
+// high half, the complemented token id in the low half, so equal values rank
+// the lower id first); kk block-wide rounds then pick the CTA's top kk, which
+// go to the lead CTA's shared memory; the lead CTA merges the C * kk keys and
+// writes the children's tokens.  Clusters of leaves leave after reading the
+// tree.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -32,7 +33,9 @@ namespace {
 
 constexpr int FT_THREADS = 256;
 constexpr int FT_MAX_K = 32;        // largest child rank + 1
-constexpr int FT_MAX_CLUSTER = 16;
+// at most 8 CTAs per row: 16-CTA clusters measured at 31 clusters in flight on
+// the whole GPU, which left the 46 expanding rows of a 64-node tree two waves deep
+constexpr int FT_MAX_CLUSTER = 8;
 
 // float -> unsigned with the same order (negative values below positive ones)
 __device__ __forceinline__ uint32_t ordered_bits(float v) {
@@ -69,28 +72,76 @@ struct FillShared {
     int bad_node;   // this node's children cannot be expanded (too many, or a bad rank)
 };
 
-// Largest key below `below` held by this thread in its elements of `vals`
-// (index base + i for vals[i]), then the block-wide maximum.
-__device__ unsigned long long block_max_below(const float* vals, int count, int base, unsigned long long below,
-                                              FillShared& sh) {
-    unsigned long long best = 0ull;
-    for (int i = threadIdx.x; i < count; i += FT_THREADS) {
-        const unsigned long long k = make_key(vals[i], base + i);
-        if (k < below && k > best) best = k;
+// Insert key into a descending list of K keys held in registers (the smallest
+// falls off); keys that do not beat the last entry are skipped cheaply.
+template <int K>
+__device__ __forceinline__ void list_insert(unsigned long long (&L)[K], unsigned long long x, unsigned long long below) {
+    if (x <= L[K - 1] || x >= below) return;
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        const unsigned long long hi = L[j] > x ? L[j] : x;
+        x = L[j] > x ? x : L[j];
+        L[j] = hi;
     }
-    best = warp_max_u64(best);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) sh.warp_best[warp] = best;
-    __syncthreads();
-    unsigned long long r = lane < FT_THREADS / 32 ? sh.warp_best[lane] : 0ull;
-    r = warp_max_u64(r);
-    __syncthreads();  // warp_best is reused by the next round
-    return r;
+}
+
+// The CTA's next `take` keys (take <= K) below `below` among src[0, cnt) (token
+// ids lo + i), into sh.mine[r0, r0 + take): one pass over global memory with a
+// K-entry list per thread, then `take` rounds in which every thread offers its
+// best remaining key and the block-wide winner drops it.  Keys of 0 mean "none"
+// (the slice has fewer entries).
+template <int K>
+__device__ void slice_topk(const float* src, int cnt, int lo, bool vec4, int take, int r0, unsigned long long below,
+                           FillShared& sh) {
+    unsigned long long L[K];
+#pragma unroll
+    for (int j = 0; j < K; ++j) L[j] = 0ull;
+    const int tid = threadIdx.x;
+    if (vec4) {
+        const float4* s4 = reinterpret_cast<const float4*>(src);
+        const int n4 = cnt >> 2;
+        int i = tid;
+        for (; i + FT_THREADS < n4; i += 2 * FT_THREADS) {
+            const float4 v0 = __ldg(s4 + i), v1 = __ldg(s4 + i + FT_THREADS);
+            const int e0 = lo + 4 * i, e1 = e0 + 4 * FT_THREADS;
+            list_insert<K>(L, make_key(v0.x, e0), below);
+            list_insert<K>(L, make_key(v0.y, e0 + 1), below);
+            list_insert<K>(L, make_key(v0.z, e0 + 2), below);
+            list_insert<K>(L, make_key(v0.w, e0 + 3), below);
+            list_insert<K>(L, make_key(v1.x, e1), below);
+            list_insert<K>(L, make_key(v1.y, e1 + 1), below);
+            list_insert<K>(L, make_key(v1.z, e1 + 2), below);
+            list_insert<K>(L, make_key(v1.w, e1 + 3), below);
+        }
+        for (; i < n4; i += FT_THREADS) {
+            const float4 v = __ldg(s4 + i);
+            const int e = lo + 4 * i;
+            list_insert<K>(L, make_key(v.x, e), below);
+            list_insert<K>(L, make_key(v.y, e + 1), below);
+            list_insert<K>(L, make_key(v.z, e + 2), below);
+            list_insert<K>(L, make_key(v.w, e + 3), below);
+        }
+        for (int e = (cnt & ~3) + tid; e < cnt; e += FT_THREADS) list_insert<K>(L, make_key(__ldg(src + e), lo + e), below);
+    } else {
+        for (int e = tid; e < cnt; e += FT_THREADS) list_insert<K>(L, make_key(__ldg(src + e), lo + e), below);
+    }
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int r = 0; r < take; ++r) {
+        const unsigned long long w = warp_max_u64(L[0]);
+        if (lane == 0) sh.warp_best[warp] = w;
+        __syncthreads();
+        const unsigned long long best = warp_max_u64(lane < FT_THREADS / 32 ? sh.warp_best[lane] : 0ull);
+        if (tid == 0) sh.mine[r0 + r] = best;
+        if (best != 0ull && L[0] == best) {  // keys are unique: one thread drops its head
+#pragma unroll
+            for (int j = 0; j + 1 < K; ++j) L[j] = L[j + 1];
+            L[K - 1] = 0ull;
+        }
+        __syncthreads();  // warp_best is reused by the next round
+    }
 }
 
 __global__ void __launch_bounds__(FT_THREADS) fill_topk_kernel(const FillArgs a) {
-    extern __shared__ float4 ft_dyn[];
-    float* slice = reinterpret_cast<float*>(ft_dyn);
     __shared__ FillShared sh;
     cg::cluster_group cluster = cg::this_cluster();
     const int C = a.cluster;
@@ -163,26 +214,33 @@ __global__ void __launch_bounds__(FT_THREADS) fill_topk_kernel(const FillArgs a)
     if (u >= n || nk == 0) return;  // no such node, or a leaf: nothing to expand (cluster-uniform)
     const int kk = sh.kk;
 
-    // ---- this CTA's slice of u's draft row, staged in shared memory
-    const int lo = min(a.V, crank * a.slice);
-    const int cnt = min(a.V, lo + a.slice) - lo;
-    const float* src = a.q + ((size_t)b * N + u) * (size_t)a.V + lo;
-    if (a.vec4) {
-        const float4* s4 = reinterpret_cast<const float4*>(src);
-        for (int i = tid; i < cnt / 4; i += FT_THREADS) ft_dyn[i] = __ldg(s4 + i);
-        for (int i = (cnt & ~3) + tid; i < cnt; i += FT_THREADS) slice[i] = __ldg(src + i);
-    } else {
-        for (int i = tid; i < cnt; i += FT_THREADS) slice[i] = __ldg(src + i);
+    // ---- the top kk keys of this CTA's slice of u's draft row, read once
+    {
+        const int lo = min(a.V, crank * a.slice);
+        const int cnt = min(a.V, lo + a.slice) - lo;
+        const float* src = a.q + ((size_t)b * N + u) * (size_t)a.V + lo;
+        const bool v4 = a.vec4 != 0;
+        if (kk <= 1) {
+            slice_topk<1>(src, cnt, lo, v4, kk, 0, ~0ull, sh);
+        } else if (kk <= 2) {
+            slice_topk<2>(src, cnt, lo, v4, kk, 0, ~0ull, sh);
+        } else if (kk <= 4) {
+            slice_topk<4>(src, cnt, lo, v4, kk, 0, ~0ull, sh);
+        } else {
+            // eight ranks per pass over the slice (more than eight children is rare)
+            unsigned long long below = ~0ull;
+            for (int r0 = 0; r0 < kk; r0 += 8) {
+                const int take = min(8, kk - r0);
+                slice_topk<8>(src, cnt, lo, v4, take, r0, below, sh);
+                below = sh.mine[r0 + take - 1];
+                if (below == 0ull) {  // the slice ran out: the remaining ranks are empty
+                    for (int r = r0 + take + threadIdx.x; r < kk; r += FT_THREADS) sh.mine[r] = 0ull;
+                    __syncthreads();
+                    break;
+                }
+            }
+        }
     }
-    __syncthreads();
-    // ---- the slice's top kk keys (0 = none: the slice has fewer entries)
-    unsigned long long below = ~0ull;
-    for (int r = 0; r < kk; ++r) {
-        const unsigned long long k = block_max_below(slice, cnt, lo, below, sh);
-        if (tid == 0) sh.mine[r] = k;
-        below = k;
-    }
-    __syncthreads();
     // ---- gather every CTA's keys in the lead CTA
     if (C > 1) {
         cluster.sync();  // every CTA of the cluster is running before shared memory is shared
@@ -221,23 +279,17 @@ __global__ void __launch_bounds__(FT_THREADS) fill_topk_kernel(const FillArgs a)
 }  // namespace
 
 void fill_topk_plan(int V, int* cluster, int* slice, int* smem_bytes) {
-    int c = (V + 8191) / 8192;
+    int c = (V + 16383) / 16384;
     if (c > FT_MAX_CLUSTER) c = FT_MAX_CLUSTER;
     if (c < 1) c = 1;
     int s = (V + c - 1) / c;
     s = (s + 3) / 4 * 4;
     *cluster = c;
     *slice = s;
-    *smem_bytes = (int)(sizeof(float) * (size_t)s);
+    *smem_bytes = 0;  // the slice is scanned straight from global memory
 }
 
 cudaError_t launch_fill_topk(const FillArgs& a, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(fill_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, a.smem_bytes);
-    if (e != cudaSuccess) return e;
-    if (a.cluster > 8) {
-        e = cudaFuncSetAttribute(fill_topk_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-    }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     cfg.gridDim = dim3((unsigned)a.cluster * (unsigned)a.B * (unsigned)a.N, 1, 1);
