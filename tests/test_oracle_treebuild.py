@@ -108,3 +108,15 @@ def test_depth_cap_and_budget_monotonicity():
     acc = [0.55, 0.2, 0.1, 0.05]
     vals = [oracle.tree_shape_dp(acc, n, 5)[2] for n in range(1, 25)]
     assert all(b >= a for a, b in zip(vals, vals[1:]))
+
+
+def test_ties_follow_the_stated_rule():
+    """Equal values: the smaller subtree goes to the lower rank, then the
+    smaller tree wins (the reading the library documents)."""
+    # root children sized (1, 2) or (2, 1) tie at 0.5 * 1 + 0.5 * 1.5 = 1.25: the rank-0 child stays a leaf
+    parent, rank, value = oracle.tree_shape_dp([0.5, 0.5], 4, 2)
+    assert value == 1.25
+    assert parent.tolist() == [-1, 0, 0, 2] and rank.tolist() == [-1, 0, 1, 0]
+    # a rank that is never accepted adds nothing: the tree without it is smaller
+    parent, rank, value = oracle.tree_shape_dp([0.5, 0.0], 3, 1)
+    assert parent.tolist() == [-1, 0] and value == 0.5
