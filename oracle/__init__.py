@@ -30,6 +30,8 @@ decoding):
   tree-structure optimisation, "Top-k branching").
 * :func:`tree_shape_dp`, :func:`tree_value` -- the budget-constrained tree shape
   by dynamic programming (glossary, "Budget-constrained optimisation").
+* :func:`select_tree` -- the dynamic tree: the best-scoring ancestor-closed
+  candidates under a node budget (LLM Primer VI ch. 9, 9.2, EAGLE-2).
 
 Every function is pinned by ``tests/test_oracle_*.py`` against values the
 pages print, closed forms, exhaustive search and library routines.
@@ -382,6 +384,43 @@ def tree_shape_dp(accept, budget: int, max_depth: int | None = None):
     parent = np.array([-1] + [index[pth[:-1]] for pth in paths[1:]], np.int32)
     rank = np.array([-1] + [pth[-1] for pth in paths[1:]], np.int32)
     return parent, rank, F[D][n_best]
+
+
+def select_tree(cand_parent, cand_token, cand_prob, budget: int):
+    """Dynamic tree selection from a grown candidate set (EAGLE-2's dynamic
+    draft tree, LLM Primer VI ch. 9, 9.2; scored as the glossary's
+    budget-constrained optimisation, "the whole tree's expected accepted
+    tokens under a node budget").  Candidates 0..M-1 are topological
+    (cand_parent[c] < c, -1 = a child of the root); a candidate's score is the
+    product of cand_prob along its path (the draft's estimate that it is
+    accepted).  Take candidates by descending score, equal scores by lower
+    index, each one only if its parent is already in, until the tree holds
+    `budget` nodes with the root.  Returns (parent_idx, tree_tokens,
+    cand_index, value): node 0 is the root (parent -1, token -1, index -1),
+    nodes 1.. the selected candidates in the order taken; value = the sum of
+    their scores."""
+    par = [int(x) for x in cand_parent]
+    prob = [float(x) for x in cand_prob]
+    M = len(par)
+    score = [0.0] * M
+    for c in range(M):
+        score[c] = (score[par[c]] if par[c] >= 0 else 1.0) * prob[c]
+    order = sorted(range(M), key=lambda c: (-score[c], c))
+    node_of = {}
+    taken = []
+    for c in order:
+        if len(taken) >= budget - 1:
+            break
+        if par[c] < 0 or par[c] in node_of:
+            node_of[c] = len(taken) + 1
+            taken.append(c)
+    parent = np.array([-1] + [0 if par[c] < 0 else node_of[par[c]] for c in taken], np.int32)
+    tokens = np.array([-1] + [int(cand_token[c]) for c in taken], np.int32)
+    index = np.array([-1] + taken, np.int32)
+    value = 0.0
+    for c in taken:
+        value += score[c]
+    return parent, tokens, index, value
 
 
 def softmax_rows(logits) -> np.ndarray:

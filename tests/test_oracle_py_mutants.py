@@ -44,6 +44,10 @@ MUTANTS = [
         r = walk(""", RAGGED),
     ("ragged_empty_draws_a_token", '"bonus_token": np.full(B, -1, np.int32)', '"bonus_token": np.full(B, 0, np.int32)',
      RAGGED),
+    ("select_score_not_a_product", "score[c] = (score[par[c]] if par[c] >= 0 else 1.0) * prob[c]",
+     "score[c] = prob[c]", TREE),
+    ("select_ties_to_higher_index", "order = sorted(range(M), key=lambda c: (-score[c], c))",
+     "order = sorted(range(M), key=lambda c: (-score[c], -c))", TREE),
     ("softmax_wrong_axis", "return (e / e.sum(axis=-1, keepdims=True)).astype(np.float32)",
      "return (e / e.sum(axis=0, keepdims=True)).astype(np.float32)", LOGITS),
 ]

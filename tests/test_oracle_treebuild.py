@@ -120,3 +120,43 @@ def test_ties_follow_the_stated_rule():
     # a rank that is never accepted adds nothing: the tree without it is smaller
     parent, rank, value = oracle.tree_shape_dp([0.5, 0.0], 3, 1)
     assert parent.tolist() == [-1, 0] and value == 0.5
+
+
+def _closed_subsets(par, size):
+    M = len(par)
+    for k in range(size + 1):
+        for sub in itertools.combinations(range(M), k):
+            ss = set(sub)
+            if all(par[c] < 0 or par[c] in ss for c in sub):
+                yield sub
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_select_tree_is_the_best_closed_subset(seed):
+    rng = np.random.default_rng(seed)
+    M = int(rng.integers(3, 10))
+    par = [-1] + [int(rng.integers(-1, c)) for c in range(1, M)]
+    prob = rng.random(M) * 0.9 + 0.05
+    tok = rng.integers(0, 100, M)
+    score = np.zeros(M)
+    for c in range(M):
+        score[c] = (score[par[c]] if par[c] >= 0 else 1.0) * prob[c]
+    for budget in (1, 2, 4, M + 3):
+        parent, tokens, index, value = oracle.select_tree(par, tok, prob, budget)
+        best = max(sum(score[c] for c in sub) for sub in _closed_subsets(par, budget - 1))
+        assert abs(value - best) <= 1e-12
+        n = len(parent)
+        assert n == min(budget, M + 1) and parent[0] == -1 and index[0] == -1
+        for j in range(1, n):
+            c = index[j]
+            assert 0 <= parent[j] < j and tokens[j] == tok[c]
+            assert (par[c] < 0 and parent[j] == 0) or index[parent[j]] == par[c]
+
+
+def test_select_tree_ties_and_hand_example():
+    # root -> a (0.5), b (0.5); a -> c (1.0): scores a 0.5, b 0.5, c 0.5 -> order a, b, c by index
+    parent, tokens, index, value = oracle.select_tree([-1, -1, 0], [7, 8, 9], [0.5, 0.5, 1.0], 3)
+    assert index.tolist() == [-1, 0, 1] and parent.tolist() == [-1, 0, 0] and tokens.tolist() == [-1, 7, 8]
+    assert value == 1.0
+    parent, tokens, index, value = oracle.select_tree([-1, -1, 0], [7, 8, 9], [0.5, 0.4, 0.9], 3)
+    assert index.tolist() == [-1, 0, 2] and parent.tolist() == [-1, 0, 1] and abs(value - 0.95) < 1e-15
