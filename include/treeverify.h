@@ -345,6 +345,39 @@ TV_API tv_status tv_tree_shape(const double *accept, int32_t num_ranks, int32_t 
                                int32_t *parent_idx, int32_t *rank, int32_t *num_nodes,
                                double *expected_accepted);
 
+/*
+ * Building the draft tree: the dynamic tree (EAGLE-2's dynamic draft-tree
+ * expansion, LLM Primer VI ch. 9, 9.2: the target chooses among many draft
+ * paths, not one guess), selected as the glossary's budget-constrained
+ * optimisation (the whole tree's expected accepted tokens under a node budget)
+ * with the draft's own probabilities as the acceptance estimate.
+ *
+ * Candidates 0 .. num_candidates-1 were grown by the caller (for example by
+ * tv_tree_fill_topk level by level): cand_parent[c] < c is c's parent
+ * candidate, or -1 for a child of the root; cand_token[c] its token;
+ * cand_prob[c] in [0, 1] the draft probability of that token given its
+ * parent's path.  A candidate's score is the product of cand_prob along its
+ * path.  Candidates are taken by descending score, equal scores by lower
+ * index, each only if its parent is already taken (with probabilities <= 1
+ * this is the best-scoring ancestor-closed set), until the tree holds
+ * `budget` nodes including the root.
+ * Outputs (host arrays of `budget` entries, the rest set to -1): node 0 is
+ * the root (parent -1, token -1, candidate -1); nodes 1.. are the taken
+ * candidates in the order taken (so parents come first and siblings run from
+ * the best score down, the order the walk tries them in): parent_idx,
+ * tree_tokens (feed tv_tree_attention and tv_verify_sample; the root's token
+ * is the caller's last committed token), cand_index (which candidate each
+ * node is); *num_nodes; *expected_accepted = the sum of the taken scores.
+ * Host computation only.  Errors: null outputs, budget < 1, a negative count
+ * or a probability outside [0, 1]: TV_ERR_INVALID_ARG; candidates that are
+ * not topological: TV_ERR_TREE; more than 2^20 candidates or a budget over
+ * 1024: TV_ERR_UNSUPPORTED.
+ */
+TV_API tv_status tv_tree_select(const int32_t *cand_parent, const int32_t *cand_token, const double *cand_prob,
+                                int32_t num_candidates, int32_t budget, int32_t *parent_idx,
+                                int32_t *tree_tokens, int32_t *cand_index, int32_t *num_nodes,
+                                double *expected_accepted);
+
 /* Static string for a status code. */
 TV_API const char *tv_status_string(int32_t status);
 

@@ -34,3 +34,33 @@ def test_tree_shape_rejects_bad_arguments():
     assert tv.tv_tree_shape(np.full(33, 0.01), 33, 8, 0, parent, rank, n, val) == tv.TV_ERR_UNSUPPORTED
     assert tv.tv_tree_shape(acc, 2, 8, 0, parent, rank, n, val) == tv.TV_OK and 1 <= n[0] <= 8
     assert parent[0] == -1 and (parent[n[0]:] == -1).all()
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_library_select_equals_oracle(seed):
+    rng = np.random.default_rng(100 + seed)
+    M = int(rng.integers(0, 300))
+    par = np.array([int(rng.integers(-1, c)) if c else -1 for c in range(M)], np.int32)
+    prob = rng.random(M)
+    if seed % 3 == 0:
+        prob = np.round(prob * 4) / 4  # many exact ties
+    tok = rng.integers(0, 128256, M).astype(np.int32)
+    for budget in (1, 2, 17, 64, 1024):
+        got = tv.tree_select(par, tok, prob, budget)
+        ref = oracle.select_tree(par, tok, prob, budget)
+        for g, r in zip(got[:3], ref[:3]):
+            np.testing.assert_array_equal(g, r)
+        assert got[3] == ref[3]
+
+
+def test_tree_select_rejects_bad_arguments():
+    out = [np.zeros(8, np.int32) for _ in range(3)]
+    n = np.zeros(1, np.int32)
+    val = np.zeros(1)
+    par, tok, prob = np.array([-1, 0], np.int32), np.array([1, 2], np.int32), np.array([0.5, 0.5])
+    assert tv.tv_tree_select(par, tok, prob, 2, 8, *out, n, val) == tv.TV_OK and n[0] == 3
+    assert tv.tv_tree_select(np.array([-1, 1], np.int32), tok, prob, 2, 8, *out, n, val) == tv.TV_ERR_TREE
+    assert tv.tv_tree_select(par, tok, np.array([0.5, 1.5]), 2, 8, *out, n, val) == tv.TV_ERR_INVALID_ARG
+    assert tv.tv_tree_select(par, tok, prob, 2, 0, *out, n, val) == tv.TV_ERR_INVALID_ARG
+    assert tv.tv_tree_select(par, tok, prob, 2, 1025, *out, n, val) == tv.TV_ERR_UNSUPPORTED
+    assert tv.tv_tree_select(None, None, None, 0, 8, *out, n, val) == tv.TV_OK and n[0] == 1

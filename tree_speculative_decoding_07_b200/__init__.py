@@ -78,12 +78,13 @@ def lib() -> ctypes.CDLL:
         L.tv_verify_sample_logits.argtypes = [ctypes.POINTER(TvSampleDesc), P, P, P, P, P, P, P, P, P, sz, P, P]
         L.tv_tree_fill_topk.argtypes = [ctypes.POINTER(TvSampleDesc), P, P, P, P, P, P]
         L.tv_tree_shape.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, P, P]
+        L.tv_tree_select.argtypes = [P, P, P, ctypes.c_int32, ctypes.c_int32, P, P, P, P, P]
         L.tv_status_string.argtypes = [ctypes.c_int32]
         L.tv_status_string.restype = ctypes.c_char_p
         L.tv_version.restype = ctypes.c_int32
         for name in ("tv_tree_attention_plan", "tv_tree_attention", "tv_tree_attention_static",
                      "tv_verify_sample_plan", "tv_verify_sample", "tv_commit_path", "tv_verify_sample_logits",
-                     "tv_tree_fill_topk", "tv_tree_shape"):
+                     "tv_tree_fill_topk", "tv_tree_shape", "tv_tree_select"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -185,6 +186,33 @@ def tv_tree_shape(accept, num_ranks: int, budget: int, max_depth: int, parent_id
     """Host pointers (numpy arrays or ctypes addresses)."""
     return int(lib().tv_tree_shape(_hptr(accept), int(num_ranks), int(budget), int(max_depth), _hptr(parent_idx),
                                    _hptr(rank), _hptr(num_nodes), _hptr(expected_accepted)))
+
+
+def tv_tree_select(cand_parent, cand_token, cand_prob, num_candidates: int, budget: int, parent_idx, tree_tokens,
+                   cand_index, num_nodes, expected_accepted) -> int:
+    """Host pointers (numpy arrays or ctypes addresses)."""
+    return int(lib().tv_tree_select(_hptr(cand_parent), _hptr(cand_token), _hptr(cand_prob), int(num_candidates),
+                                    int(budget), _hptr(parent_idx), _hptr(tree_tokens), _hptr(cand_index),
+                                    _hptr(num_nodes), _hptr(expected_accepted)))
+
+
+def tree_select(cand_parent, cand_token, cand_prob, budget: int):
+    """Dynamic tree selection; returns (parent_idx, tree_tokens, cand_index,
+    expected_accepted) as numpy arrays trimmed to the tree's size."""
+    import numpy as np
+    par = np.ascontiguousarray(cand_parent, dtype=np.int32)
+    tok = np.ascontiguousarray(cand_token, dtype=np.int32)
+    prob = np.ascontiguousarray(cand_prob, dtype=np.float64)
+    parent = np.empty(max(int(budget), 1), np.int32)
+    tokens = np.empty_like(parent)
+    index = np.empty_like(parent)
+    n = np.zeros(1, np.int32)
+    val = np.zeros(1, np.float64)
+    s = tv_tree_select(par, tok, prob, par.size, budget, parent, tokens, index, n, val)
+    if s != TV_OK:
+        raise TreeVerifyError(s, "tv_tree_select")
+    k = int(n[0])
+    return parent[:k].copy(), tokens[:k].copy(), index[:k].copy(), float(val[0])
 
 
 def _hptr(a):

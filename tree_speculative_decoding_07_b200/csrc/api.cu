@@ -270,6 +270,22 @@ tv_status tv_tree_shape(const double* accept, int32_t num_ranks, int32_t budget,
     return TV_OK;
 }
 
+tv_status tv_tree_select(const int32_t* cand_parent, const int32_t* cand_token, const double* cand_prob,
+                         int32_t num_candidates, int32_t budget, int32_t* parent_idx, int32_t* tree_tokens,
+                         int32_t* cand_index, int32_t* num_nodes, double* expected_accepted) {
+    if (!parent_idx || !tree_tokens || !cand_index || !num_nodes || !expected_accepted) return TV_ERR_INVALID_ARG;
+    if (num_candidates < 0 || budget < 1) return TV_ERR_INVALID_ARG;
+    if (num_candidates > 0 && (!cand_parent || !cand_token || !cand_prob)) return TV_ERR_INVALID_ARG;
+    if (num_candidates > (1 << 20) || budget > 1024) return TV_ERR_UNSUPPORTED;
+    for (int c = 0; c < num_candidates; ++c)
+        if (!(cand_prob[c] >= 0.0 && cand_prob[c] <= 1.0)) return TV_ERR_INVALID_ARG;
+    const int n = tv::tree_select(cand_parent, cand_token, cand_prob, num_candidates, budget, parent_idx, tree_tokens,
+                                  cand_index, expected_accepted);
+    if (n < 0) return TV_ERR_TREE;
+    *num_nodes = n;
+    return TV_OK;
+}
+
 tv_status tv_verify_sample(const tv_sample_desc* desc, const float* p, const float* q, const int32_t* tree_tokens,
                            const int32_t* parent_idx, const float* uniforms, int32_t* accepted_path,
                            int32_t* accepted_len, int32_t* bonus_token, void* workspace, size_t workspace_bytes,

@@ -91,4 +91,8 @@ cudaError_t launch_fill_topk(const FillArgs& a, cudaStream_t st);
 int tree_shape_dp(const double* accept, int k, int budget, int max_depth, int32_t* parent, int32_t* rank,
                   double* value);
 
+// Dynamic tree selection from a candidate set (host).  Returns the node count, -1 if not topological.
+int tree_select(const int32_t* cand_parent, const int32_t* cand_token, const double* cand_prob, int M, int budget,
+                int32_t* parent_idx, int32_t* tree_tokens, int32_t* cand_index, double* value);
+
 }  // namespace tv

@@ -398,4 +398,49 @@ int tree_shape_dp(const double* accept, int k, int budget, int max_depth, int32_
     return n;
 }
 
+// ---------------------------------------------------------------- dynamic selection
+
+// Candidates 0..M-1 are topological (parent < index, -1 = a child of the root);
+// score = product of prob along the path.  Take candidates by descending score,
+// equal scores by lower index, each only if its parent is already taken, until
+// the tree holds `budget` nodes with the root.  Returns the node count, or -1
+// when the candidates are not topological.
+int tree_select(const int32_t* cand_parent, const int32_t* cand_token, const double* cand_prob, int M, int budget,
+                int32_t* parent_idx, int32_t* tree_tokens, int32_t* cand_index, double* value) {
+    std::vector<double> score(M);
+    for (int c = 0; c < M; ++c) {
+        const int p = cand_parent[c];
+        if (p < -1 || p >= c) return -1;
+        const double up = p >= 0 ? score[p] : 1.0;
+        score[c] = up * cand_prob[c];
+    }
+    std::vector<int> order(M);
+    for (int c = 0; c < M; ++c) order[c] = c;
+    std::sort(order.begin(), order.end(), [&](int x, int y) {
+        if (score[x] != score[y]) return score[x] > score[y];
+        return x < y;
+    });
+    std::vector<int> node_of(M, -1);
+    for (int j = 0; j < budget; ++j) {
+        parent_idx[j] = -1;
+        tree_tokens[j] = -1;
+        cand_index[j] = -1;
+    }
+    int n = 1;
+    double total = 0.0;
+    for (int k = 0; k < M && n < budget; ++k) {
+        const int c = order[k];
+        const int p = cand_parent[c];
+        if (p >= 0 && node_of[p] < 0) continue;
+        node_of[c] = n;
+        parent_idx[n] = p >= 0 ? node_of[p] : 0;
+        tree_tokens[n] = cand_token[c];
+        cand_index[n] = c;
+        ++n;
+    }
+    for (int j = 1; j < n; ++j) total += score[cand_index[j]];
+    *value = total;
+    return n;
+}
+
 }  // namespace tv
