@@ -21,9 +21,26 @@
  *                     root-down, depth first; a rejected child hands the
  *                     renormalised residual to its next sibling).
  *
+ * Around the step:
+ *
+ *  tv_verify_sample_logits  the same walk on the two models' logits, the row
+ *                     softmax formed inside the walk.
+ *  tv_commit_path     after verification, the accepted path joins the cached
+ *                     prefix (blog, "KV cache management and prefix sharing";
+ *                     glossary, "KV cache management challenges").
+ *  tv_tree_shape, tv_tree_fill_topk, tv_tree_select  building the tree that is
+ *                     verified (glossary, tree-structure optimisation: top-k
+ *                     branching and budget-constrained optimisation; LLM
+ *                     Primer VI ch. 9, 9.2: EAGLE-2's dynamic tree).
+ *
+ * Ragged batches (trees of different sizes in one call) go through the
+ * descriptors' node_counts; a NULL parent_idx means chains (linear
+ * speculation).
+ *
  * Conventions shared by all calls
  *  - Every array pointer is a caller-owned DEVICE pointer unless stated
- *    otherwise; descriptors and plan structs are host memory.  The library
+ *    otherwise (tv_tree_shape and tv_tree_select work on host arrays);
+ *    descriptors and plan structs are host memory.  The library
  *    never allocates device memory and never synchronises the stream.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Work is enqueued asynchronously on it.
