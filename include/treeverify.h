@@ -395,6 +395,23 @@ TV_API tv_status tv_tree_select(const int32_t *cand_parent, const int32_t *cand_
                                 int32_t *tree_tokens, int32_t *cand_index, int32_t *num_nodes,
                                 double *expected_accepted);
 
+/*
+ * tv_tree_select for a whole batch, laid out for the ragged calls: sequence b's
+ * candidates are entries cand_offsets[b] .. cand_offsets[b+1]-1 of the
+ * candidate arrays (parent indices local to the sequence), and its tree goes
+ * to row b of parent_idx, tree_tokens and cand_index ([batch][budget] host
+ * int32), its size to node_counts[b] and its value to expected_accepted[b].
+ * The outputs are the arrays tv_tree_attention, tv_verify_sample and
+ * tv_commit_path take (num_nodes = budget, desc.node_counts = node_counts on
+ * the device).  Every sequence is checked before anything is written; the
+ * errors are tv_tree_select's, and cand_offsets must start at 0 and not
+ * decrease (TV_ERR_INVALID_ARG).
+ */
+TV_API tv_status tv_tree_select_batch(int32_t batch, const int32_t *cand_offsets, const int32_t *cand_parent,
+                                      const int32_t *cand_token, const double *cand_prob, int32_t budget,
+                                      int32_t *parent_idx, int32_t *tree_tokens, int32_t *cand_index,
+                                      int32_t *node_counts, double *expected_accepted);
+
 /* Static string for a status code. */
 TV_API const char *tv_status_string(int32_t status);
 

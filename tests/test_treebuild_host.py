@@ -64,3 +64,36 @@ def test_tree_select_rejects_bad_arguments():
     assert tv.tv_tree_select(par, tok, prob, 2, 0, *out, n, val) == tv.TV_ERR_INVALID_ARG
     assert tv.tv_tree_select(par, tok, prob, 2, 1025, *out, n, val) == tv.TV_ERR_UNSUPPORTED
     assert tv.tv_tree_select(None, None, None, 0, 8, *out, n, val) == tv.TV_OK and n[0] == 1
+
+
+def test_batch_select_equals_per_sequence_oracle():
+    rng = np.random.default_rng(7)
+    B, budget = 9, 24
+    sizes = rng.integers(0, 60, B)
+    sizes[0] = 0
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    par, tok, prob = [], [], []
+    for m in sizes:
+        par += [int(rng.integers(-1, c)) if c else -1 for c in range(m)]
+        tok += list(rng.integers(0, 1000, m))
+        prob += list(np.round(rng.random(m) * 8) / 8)
+    parent, tokens, index, counts, val = tv.tree_select_batch(off, par, tok, prob, budget)
+    for b in range(B):
+        o, m = off[b], sizes[b]
+        rp, rt, ri, rv = oracle.select_tree(par[o:o + m], tok[o:o + m], prob[o:o + m], budget)
+        n = len(rp)
+        assert counts[b] == n and val[b] == rv
+        np.testing.assert_array_equal(parent[b, :n], rp)
+        np.testing.assert_array_equal(tokens[b, :n], rt)
+        np.testing.assert_array_equal(index[b, :n], ri)
+        assert (parent[b, n:] == -1).all()
+    # a bad sequence anywhere: nothing is written
+    bad_par = list(par)
+    bad_par[off[3] + 1] = 5
+    counts2 = np.full(B, 77, np.int32)
+    out = [np.full((B, budget), 77, np.int32) for _ in range(3)]
+    val2 = np.zeros(B)
+    s = tv.lib().tv_tree_select_batch(B, tv._hptr(off), tv._hptr(np.array(bad_par, np.int32)),
+                                      tv._hptr(np.array(tok, np.int32)), tv._hptr(np.array(prob)), budget,
+                                      *[tv._hptr(x) for x in out], tv._hptr(counts2), tv._hptr(val2))
+    assert s == tv.TV_ERR_TREE and (counts2 == 77).all() and all((x == 77).all() for x in out)

@@ -79,12 +79,13 @@ def lib() -> ctypes.CDLL:
         L.tv_tree_fill_topk.argtypes = [ctypes.POINTER(TvSampleDesc), P, P, P, P, P, P]
         L.tv_tree_shape.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, P, P]
         L.tv_tree_select.argtypes = [P, P, P, ctypes.c_int32, ctypes.c_int32, P, P, P, P, P]
+        L.tv_tree_select_batch.argtypes = [ctypes.c_int32, P, P, P, P, ctypes.c_int32, P, P, P, P, P]
         L.tv_status_string.argtypes = [ctypes.c_int32]
         L.tv_status_string.restype = ctypes.c_char_p
         L.tv_version.restype = ctypes.c_int32
         for name in ("tv_tree_attention_plan", "tv_tree_attention", "tv_tree_attention_static",
                      "tv_verify_sample_plan", "tv_verify_sample", "tv_commit_path", "tv_verify_sample_logits",
-                     "tv_tree_fill_topk", "tv_tree_shape", "tv_tree_select"):
+                     "tv_tree_fill_topk", "tv_tree_shape", "tv_tree_select", "tv_tree_select_batch"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -213,6 +214,27 @@ def tree_select(cand_parent, cand_token, cand_prob, budget: int):
         raise TreeVerifyError(s, "tv_tree_select")
     k = int(n[0])
     return parent[:k].copy(), tokens[:k].copy(), index[:k].copy(), float(val[0])
+
+
+def tree_select_batch(cand_offsets, cand_parent, cand_token, cand_prob, budget: int):
+    """tv_tree_select over a batch; returns (parent_idx, tree_tokens, cand_index)
+    as [B][budget] int32 arrays, node_counts [B] and expected_accepted [B]."""
+    import numpy as np
+    off = np.ascontiguousarray(cand_offsets, dtype=np.int32)
+    B = off.size - 1
+    par = np.ascontiguousarray(cand_parent, dtype=np.int32)
+    tok = np.ascontiguousarray(cand_token, dtype=np.int32)
+    prob = np.ascontiguousarray(cand_prob, dtype=np.float64)
+    parent = np.empty((B, int(budget)), np.int32)
+    tokens = np.empty_like(parent)
+    index = np.empty_like(parent)
+    counts = np.empty(B, np.int32)
+    val = np.empty(B, np.float64)
+    s = int(lib().tv_tree_select_batch(B, _hptr(off), _hptr(par), _hptr(tok), _hptr(prob), int(budget),
+                                       _hptr(parent), _hptr(tokens), _hptr(index), _hptr(counts), _hptr(val)))
+    if s != TV_OK:
+        raise TreeVerifyError(s, "tv_tree_select_batch")
+    return parent, tokens, index, counts, val
 
 
 def _hptr(a):

@@ -286,6 +286,40 @@ tv_status tv_tree_select(const int32_t* cand_parent, const int32_t* cand_token, 
     return TV_OK;
 }
 
+tv_status tv_tree_select_batch(int32_t batch, const int32_t* cand_offsets, const int32_t* cand_parent,
+                               const int32_t* cand_token, const double* cand_prob, int32_t budget,
+                               int32_t* parent_idx, int32_t* tree_tokens, int32_t* cand_index, int32_t* node_counts,
+                               double* expected_accepted) {
+    if (batch < 1 || !cand_offsets || !node_counts || !parent_idx || !tree_tokens || !cand_index ||
+        !expected_accepted)
+        return TV_ERR_INVALID_ARG;
+    if (budget < 1) return TV_ERR_INVALID_ARG;
+    if (budget > 1024) return TV_ERR_UNSUPPORTED;
+    if (cand_offsets[0] != 0) return TV_ERR_INVALID_ARG;
+    for (int b = 0; b < batch; ++b)
+        if (cand_offsets[b + 1] < cand_offsets[b]) return TV_ERR_INVALID_ARG;
+    // every sequence is checked before any output is written
+    for (int b = 0; b < batch; ++b) {
+        const int32_t o = cand_offsets[b], m = cand_offsets[b + 1] - o;
+        for (int c = 0; c < m; ++c) {
+            if (!cand_parent || !cand_token || !cand_prob) return TV_ERR_INVALID_ARG;
+            if (!(cand_prob[o + c] >= 0.0 && cand_prob[o + c] <= 1.0)) return TV_ERR_INVALID_ARG;
+            if (cand_parent[o + c] < -1 || cand_parent[o + c] >= c) return TV_ERR_TREE;
+        }
+    }
+    for (int b = 0; b < batch; ++b) {
+        const int32_t o = cand_offsets[b], m = cand_offsets[b + 1] - o;
+        int32_t n = 0;
+        tv_status s = tv_tree_select(m ? cand_parent + o : nullptr, m ? cand_token + o : nullptr,
+                                     m ? cand_prob + o : nullptr, m, budget, parent_idx + (size_t)b * budget,
+                                     tree_tokens + (size_t)b * budget, cand_index + (size_t)b * budget, &n,
+                                     expected_accepted + b);
+        if (s != TV_OK) return s;
+        node_counts[b] = n;
+    }
+    return TV_OK;
+}
+
 tv_status tv_verify_sample(const tv_sample_desc* desc, const float* p, const float* q, const int32_t* tree_tokens,
                            const int32_t* parent_idx, const float* uniforms, int32_t* accepted_path,
                            int32_t* accepted_len, int32_t* bonus_token, void* workspace, size_t workspace_bytes,
