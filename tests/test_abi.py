@@ -133,3 +133,28 @@ def test_fill_topk_rejects_bad_arguments_before_launch():
     assert tv.tv_tree_fill_topk(tv.TvSampleDesc(1, 4, 10), None, 256, 256, 256, stream=0) == tv.TV_ERR_INVALID_ARG
     assert tv.tv_tree_fill_topk(tv.TvSampleDesc(1, 4, 10), 256, 256, 256, None, stream=0) == tv.TV_ERR_INVALID_ARG
     assert tv.tv_tree_fill_topk(tv.TvSampleDesc(1, 1025, 10), 256, 256, 256, 256, stream=0) == tv.TV_ERR_UNSUPPORTED
+
+
+def test_struct_layout_matches_the_header(tmp_path):
+    """The binding's ctypes structs have the C header's sizes and field offsets
+    (compiled with the host C compiler against include/treeverify.h)."""
+    import subprocess
+    structs = {"tv_attn_desc": tv.TvAttnDesc, "tv_attn_plan": tv.TvAttnPlan, "tv_sample_desc": tv.TvSampleDesc,
+               "tv_sample_plan": tv.TvSamplePlan}
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "treeverify.h"', "int main(void) {"]
+    for cname, cls in structs.items():
+        lines.append(f'printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in cls._fields_:
+            lines.append(f'printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ["return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    include = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    subprocess.check_call(["gcc", "-std=c11", "-I", include, "-o", str(exe), str(src)])
+    got = dict(((l.split()[0], l.split()[1]), int(l.split()[2])) for l in subprocess.check_output([str(exe)], text=True)
+               .splitlines())
+    for cname, cls in structs.items():
+        assert got[(cname, "size")] == ctypes.sizeof(cls), cname
+        for fname, _ in cls._fields_:
+            assert got[(cname, fname)] == getattr(cls, fname).offset, (cname, fname)
