@@ -72,7 +72,7 @@ extern "C" {
 typedef enum {
     TV_OK = 0,
     TV_ERR_INVALID_ARG = 1,   /* bad descriptor field, null pointer, bad size */
-    TV_ERR_UNSUPPORTED = 2,   /* valid but not supported by this build (e.g. head_dim) */
+    TV_ERR_UNSUPPORTED = 2,   /* valid but not supported by the library (e.g. head_dim) */
     TV_ERR_TREE = 3,          /* device: parent_idx not topological, or token out of range */
     TV_ERR_BLOCK_TABLE = 4,   /* device: block id outside [0, num_blocks) */
     TV_ERR_WORKSPACE = 5,     /* workspace null or smaller than the *_workspace_size value */

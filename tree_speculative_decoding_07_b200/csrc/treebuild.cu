@@ -137,7 +137,7 @@ __device__ void slice_topk(const float* src, int cnt, int lo, bool vec4, int tak
             for (int j = 0; j + 1 < K; ++j) L[j] = L[j + 1];
             L[K - 1] = 0ull;
         }
-        __syncthreads();  // warp_best is reused by the next round
+        __syncthreads();  // warp_best is reused for the next rank
     }
 }
 
