@@ -30,6 +30,9 @@ decoding):
   tree-structure optimisation, "Top-k branching").
 * :func:`tree_shape_dp`, :func:`tree_value` -- the budget-constrained tree shape
   by dynamic programming (glossary, "Budget-constrained optimisation").
+* :func:`step_speedup`, :func:`tree_shape_for_cost` -- the step's speedup
+  over plain decoding and the tree size that maximises it (LLM Primer VI
+  ch. 9, 9.3).
 * :func:`select_tree` -- the dynamic tree: the best-scoring ancestor-closed
   candidates under a node budget (LLM Primer VI ch. 9, 9.2, EAGLE-2).
 
@@ -384,6 +387,31 @@ def tree_shape_dp(accept, budget: int, max_depth: int | None = None):
     parent = np.array([-1] + [index[pth[:-1]] for pth in paths[1:]], np.int32)
     rank = np.array([-1] + [pth[-1] for pth in paths[1:]], np.int32)
     return parent, rank, F[D][n_best]
+
+
+def step_speedup(expected_accepted: float, num_nodes: int, draft_cost: float, alpha: float) -> float:
+    """Speedup of one speculative step over plain decoding (LLM Primer VI
+    ch. 9, 9.3): tokens emitted per step over the step's cost in decode steps,
+    (1 + E) / (draft_cost + 1 + alpha * N), where E is the expected accepted
+    tokens, the 1 is the bonus token, N = num_nodes - 1 draft tokens,
+    draft_cost = T_draft / T_decode and alpha the verification overhead per
+    position."""
+    return (1.0 + expected_accepted) / (draft_cost + 1.0 + alpha * (num_nodes - 1))
+
+
+def tree_shape_for_cost(accept, max_budget: int, max_depth: int | None, draft_cost: float, alpha: float):
+    """The tree size that pays (LLM Primer VI ch. 9, 9.3: a fixed N misses the
+    optimum; the glossary: Sequoia sizes the tree for the hardware): for every
+    budget n = 1..max_budget take :func:`tree_shape_dp`'s tree and its
+    :func:`step_speedup`; return the first best one as (parent, rank, value,
+    speedup)."""
+    best = None
+    for n in range(1, max_budget + 1):
+        parent, rank, value = tree_shape_dp(accept, n, max_depth)
+        sp = step_speedup(value, len(parent), draft_cost, alpha)
+        if best is None or sp > best[3]:
+            best = (parent, rank, value, sp)
+    return best
 
 
 def select_tree(cand_parent, cand_token, cand_prob, budget: int):

@@ -48,6 +48,10 @@ MUTANTS = [
      "score[c] = prob[c]", TREE),
     ("select_ties_to_higher_index", "order = sorted(range(M), key=lambda c: (-score[c], c))",
      "order = sorted(range(M), key=lambda c: (-score[c], -c))", TREE),
+    ("speedup_counts_the_root_as_a_draft", "return (1.0 + expected_accepted) / (draft_cost + 1.0 + alpha * (num_nodes - 1))",
+     "return (1.0 + expected_accepted) / (draft_cost + 1.0 + alpha * num_nodes)", TREE),
+    ("speedup_without_the_bonus", "return (1.0 + expected_accepted) / (draft_cost + 1.0 + alpha * (num_nodes - 1))",
+     "return expected_accepted / (draft_cost + 1.0 + alpha * (num_nodes - 1))", TREE),
     ("softmax_wrong_axis", "return (e / e.sum(axis=-1, keepdims=True)).astype(np.float32)",
      "return (e / e.sum(axis=0, keepdims=True)).astype(np.float32)", LOGITS),
 ]

@@ -160,3 +160,30 @@ def test_select_tree_ties_and_hand_example():
     assert value == 1.0
     parent, tokens, index, value = oracle.select_tree([-1, -1, 0], [7, 8, 9], [0.5, 0.4, 0.9], 3)
     assert index.tolist() == [-1, 0, 2] and parent.tolist() == [-1, 0, 1] and abs(value - 0.95) < 1e-15
+
+
+@pytest.mark.parametrize("p,lo,hi", [(0.8, 6, 8), (0.9, 10, 12)])
+def test_chain_speedup_peaks_where_the_pages_say(p, lo, hi):
+    """LLM Primer VI ch. 9, 9.3: the speedup (1 + E) / (T_draft/T_decode + 1 + alpha N)
+    peaks near N = 6-8 draft tokens for p = 0.8 and N = 10-12 for p = 0.9 (alpha in
+    0.05-0.15; taken here at 0.1 with free drafting)."""
+    parent, rank, value, sp = oracle.tree_shape_for_cost([p], 40, None, 0.0, 0.1)
+    N = len(parent) - 1
+    assert lo <= N <= hi
+    assert abs(sp - ((1 - p ** (N + 1)) / (1 - p)) / (1 + 0.1 * N)) <= 1e-12
+    # every other chain length is no better
+    for n in range(1, 41):
+        assert ((1 - p ** n) / (1 - p)) / (1 + 0.1 * (n - 1)) <= sp + 1e-12
+
+
+def test_speedup_limits():
+    # p -> 1: the speedup grows towards 1/alpha and never reaches it (the pages' ceiling)
+    parent, rank, value, sp = oracle.tree_shape_for_cost([1.0], 60, None, 0.0, 0.1)
+    assert len(parent) == 60 and sp < 10.0 and sp > 8.5
+    # no verification overhead and free drafting: the largest best tree wins
+    acc = [0.6, 0.25, 0.1]
+    _, _, v_all = oracle.tree_shape_dp(acc, 12, 4)
+    parent, rank, value, sp = oracle.tree_shape_for_cost(acc, 12, 4, 0.0, 0.0)
+    assert value == v_all and sp == 1.0 + v_all
+    # drafting that costs a whole decode step halves the speedup of a one-node tree
+    assert oracle.step_speedup(0.0, 1, 1.0, 0.1) == 0.5
