@@ -363,6 +363,27 @@ TV_API tv_status tv_tree_shape(const double *accept, int32_t num_ranks, int32_t 
                                double *expected_accepted);
 
 /*
+ * The tree size that pays.  LLM Primer VI ch. 9, 9.3: a step's speedup over
+ * plain decoding is E[emitted tokens] / (T_draft/T_decode + 1 + alpha N), with
+ * alpha the verification overhead per position (0.05-0.15) and N the draft
+ * tokens, so an engine that fixes N misses the optimum; the glossary: Sequoia
+ * sizes the tree for the hardware.
+ *
+ * For every budget n = 1 .. max_budget the best tree of tv_tree_shape (same
+ * accept, num_ranks, max_depth) is scored by (1 + E) / (draft_cost + 1 +
+ * alpha (size - 1)), E its expected accepted tokens (the 1 is the bonus
+ * token), draft_cost = T_draft / T_decode; the call returns the tree with the
+ * largest speedup (the smallest on ties) in the same format as tv_tree_shape,
+ * with *speedup.  Arrays hold max_budget entries.  Host computation only;
+ * errors as tv_tree_shape's, and draft_cost or alpha negative or not finite:
+ * TV_ERR_INVALID_ARG.
+ */
+TV_API tv_status tv_tree_shape_for_cost(const double *accept, int32_t num_ranks, int32_t max_budget,
+                                        int32_t max_depth, double draft_cost, double alpha,
+                                        int32_t *parent_idx, int32_t *rank, int32_t *num_nodes,
+                                        double *expected_accepted, double *speedup);
+
+/*
  * Building the draft tree: the dynamic tree (EAGLE-2's dynamic draft-tree
  * expansion, LLM Primer VI ch. 9, 9.2: the target chooses among many draft
  * paths, not one guess), selected as the glossary's budget-constrained

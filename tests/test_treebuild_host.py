@@ -97,3 +97,27 @@ def test_batch_select_equals_per_sequence_oracle():
                                       tv._hptr(np.array(tok, np.int32)), tv._hptr(np.array(prob)), budget,
                                       *[tv._hptr(x) for x in out], tv._hptr(counts2), tv._hptr(val2))
     assert s == tv.TV_ERR_TREE and (counts2 == 77).all() and all((x == 77).all() for x in out)
+
+
+@pytest.mark.parametrize("accept,budget,depth,cost,alpha", [
+    ([0.8], 40, 0, 0.0, 0.1), ([0.9], 40, 0, 0.0, 0.1), ([0.6, 0.25, 0.1], 48, 6, 0.3, 0.05),
+    ([0.55, 0.2, 0.1, 0.05], 64, 0, 0.1, 0.15), ([0.7, 0.2], 30, 3, 0.0, 0.0), ([1.0], 50, 0, 0.0, 0.1),
+    ([0.5, 0.5], 20, 4, 1.0, 0.02),
+])
+def test_library_cost_aware_shape_equals_oracle(accept, budget, depth, cost, alpha):
+    p, r, v, sp = tv.tree_shape_for_cost(accept, budget, depth, cost, alpha)
+    po, ro, vo, spo = oracle.tree_shape_for_cost(accept, budget, depth or None, cost, alpha)
+    np.testing.assert_array_equal(p, po)
+    np.testing.assert_array_equal(r, ro)
+    assert v == vo and sp == spo
+
+
+def test_cost_aware_shape_rejects_bad_costs():
+    out = [np.zeros(8, np.int32), np.zeros(8, np.int32), np.zeros(1, np.int32), np.zeros(1), np.zeros(1)]
+    acc = np.array([0.5])
+    f = tv.lib().tv_tree_shape_for_cost
+    assert f(tv._hptr(acc), 1, 8, 0, 0.0, 0.1, *[tv._hptr(x) for x in out]) == tv.TV_OK
+    assert f(tv._hptr(acc), 1, 8, 0, -1.0, 0.1, *[tv._hptr(x) for x in out]) == tv.TV_ERR_INVALID_ARG
+    assert f(tv._hptr(acc), 1, 8, 0, 0.0, float("nan"), *[tv._hptr(x) for x in out]) == tv.TV_ERR_INVALID_ARG
+    assert f(tv._hptr(acc), 1, 8, 0, float("inf"), 0.1, *[tv._hptr(x) for x in out]) == tv.TV_ERR_INVALID_ARG
+    assert f(tv._hptr(acc), 1, 300, 0, 0.0, 0.1, *[tv._hptr(x) for x in out]) == tv.TV_ERR_UNSUPPORTED

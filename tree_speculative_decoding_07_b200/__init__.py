@@ -79,13 +79,16 @@ def lib() -> ctypes.CDLL:
         L.tv_tree_fill_topk.argtypes = [ctypes.POINTER(TvSampleDesc), P, P, P, P, P, P]
         L.tv_tree_shape.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, P, P]
         L.tv_tree_select.argtypes = [P, P, P, ctypes.c_int32, ctypes.c_int32, P, P, P, P, P]
+        L.tv_tree_shape_for_cost.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_double,
+                                             ctypes.c_double, P, P, P, P, P]
         L.tv_tree_select_batch.argtypes = [ctypes.c_int32, P, P, P, P, ctypes.c_int32, P, P, P, P, P]
         L.tv_status_string.argtypes = [ctypes.c_int32]
         L.tv_status_string.restype = ctypes.c_char_p
         L.tv_version.restype = ctypes.c_int32
         for name in ("tv_tree_attention_plan", "tv_tree_attention", "tv_tree_attention_static",
                      "tv_verify_sample_plan", "tv_verify_sample", "tv_commit_path", "tv_verify_sample_logits",
-                     "tv_tree_fill_topk", "tv_tree_shape", "tv_tree_select", "tv_tree_select_batch"):
+                     "tv_tree_fill_topk", "tv_tree_shape", "tv_tree_select", "tv_tree_select_batch",
+                     "tv_tree_shape_for_cost"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -214,6 +217,24 @@ def tree_select(cand_parent, cand_token, cand_prob, budget: int):
         raise TreeVerifyError(s, "tv_tree_select")
     k = int(n[0])
     return parent[:k].copy(), tokens[:k].copy(), index[:k].copy(), float(val[0])
+
+
+def tree_shape_for_cost(accept, max_budget: int, max_depth: int = 0, draft_cost: float = 0.0, alpha: float = 0.1):
+    """The tree size with the best step speedup; returns (parent_idx, rank,
+    expected_accepted, speedup), the arrays trimmed to the tree's size."""
+    import numpy as np
+    acc = np.ascontiguousarray(accept, dtype=np.float64)
+    parent = np.empty(max(int(max_budget), 1), np.int32)
+    rank = np.empty_like(parent)
+    n = np.zeros(1, np.int32)
+    val = np.zeros(1, np.float64)
+    sp = np.zeros(1, np.float64)
+    s = int(lib().tv_tree_shape_for_cost(_hptr(acc), acc.size, int(max_budget), int(max_depth), float(draft_cost),
+                                         float(alpha), _hptr(parent), _hptr(rank), _hptr(n), _hptr(val), _hptr(sp)))
+    if s != TV_OK:
+        raise TreeVerifyError(s, "tv_tree_shape_for_cost")
+    k = int(n[0])
+    return parent[:k].copy(), rank[:k].copy(), float(val[0]), float(sp[0])
 
 
 def tree_select_batch(cand_offsets, cand_parent, cand_token, cand_prob, budget: int):

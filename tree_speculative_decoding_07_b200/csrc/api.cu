@@ -270,6 +270,20 @@ tv_status tv_tree_shape(const double* accept, int32_t num_ranks, int32_t budget,
     return TV_OK;
 }
 
+tv_status tv_tree_shape_for_cost(const double* accept, int32_t num_ranks, int32_t max_budget, int32_t max_depth,
+                                 double draft_cost, double alpha, int32_t* parent_idx, int32_t* rank,
+                                 int32_t* num_nodes, double* expected_accepted, double* speedup) {
+    if (!accept || !parent_idx || !rank || !num_nodes || !expected_accepted || !speedup) return TV_ERR_INVALID_ARG;
+    if (num_ranks < 1 || max_budget < 1 || max_depth < 0) return TV_ERR_INVALID_ARG;
+    if (!(draft_cost >= 0.0) || !(alpha >= 0.0) || isinf(draft_cost) || isinf(alpha)) return TV_ERR_INVALID_ARG;
+    if (num_ranks > 32 || max_budget > 256) return TV_ERR_UNSUPPORTED;
+    for (int i = 0; i < num_ranks; ++i)
+        if (!(accept[i] >= 0.0 && accept[i] <= 1.0)) return TV_ERR_INVALID_ARG;
+    *num_nodes = tv::tree_shape_for_cost(accept, num_ranks, max_budget, max_depth, draft_cost, alpha, parent_idx, rank,
+                                         expected_accepted, speedup);
+    return TV_OK;
+}
+
 tv_status tv_tree_select(const int32_t* cand_parent, const int32_t* cand_token, const double* cand_prob,
                          int32_t num_candidates, int32_t budget, int32_t* parent_idx, int32_t* tree_tokens,
                          int32_t* cand_index, int32_t* num_nodes, double* expected_accepted) {

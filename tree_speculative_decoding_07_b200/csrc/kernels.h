@@ -91,6 +91,10 @@ cudaError_t launch_fill_topk(const FillArgs& a, cudaStream_t st);
 int tree_shape_dp(const double* accept, int k, int budget, int max_depth, int32_t* parent, int32_t* rank,
                   double* value);
 
+// The budget whose best tree maximises the step speedup (host).  Returns the node count.
+int tree_shape_for_cost(const double* accept, int k, int max_budget, int max_depth, double draft_cost, double alpha,
+                        int32_t* parent, int32_t* rank, double* value, double* speedup);
+
 // Dynamic tree selection from a candidate set (host).  Returns the node count, -1 if not topological.
 int tree_select(const int32_t* cand_parent, const int32_t* cand_token, const double* cand_prob, int M, int budget,
                 int32_t* parent_idx, int32_t* tree_tokens, int32_t* cand_index, double* value);

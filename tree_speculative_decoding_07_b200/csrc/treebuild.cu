@@ -313,18 +313,25 @@ cudaError_t launch_fill_topk(const FillArgs& a, cudaStream_t st) {
 // G[i+1][s-t], F[d][n] = G[0][n-1].  Ties go to the smallest t, and among equal
 // totals to the smallest tree.  Nodes are numbered by depth, then by the ranks
 // along their path.
-int tree_shape_dp(const double* accept, int k, int budget, int max_depth, int32_t* parent, int32_t* rank,
-                  double* value) {
+namespace {
+
+struct ShapeTable {
+    int budget, D;
+    std::vector<std::vector<double>> F;        // F[d][n]
+    std::vector<std::vector<int32_t>> choice;  // choice[d][i * budget + s] = t
+};
+
+void shape_table(const double* accept, int k, int budget, int D, ShapeTable& T) {
     const double NEG = -INFINITY;
-    const int D = (max_depth <= 0 || max_depth > budget - 1) ? budget - 1 : max_depth;
-    std::vector<std::vector<double>> F(D + 1, std::vector<double>(budget + 1, NEG));
-    // choice[d][i * budget + s] = t
-    std::vector<std::vector<int32_t>> choice(D + 1);
-    std::vector<double> G((size_t)(k + 1) * budget), Gnext;
+    T.budget = budget;
+    T.D = D;
+    T.F.assign(D + 1, std::vector<double>(budget + 1, NEG));
+    T.choice.assign(D + 1, std::vector<int32_t>());
+    std::vector<double> G((size_t)(k + 1) * budget);
     for (int d = 0; d <= D; ++d) {
-        F[d][1] = 0.0;
+        T.F[d][1] = 0.0;
         if (d == 0) continue;
-        std::vector<int32_t>& ch = choice[d];
+        std::vector<int32_t>& ch = T.choice[d];
         ch.assign((size_t)(k + 1) * budget, 0);
         std::fill(G.begin(), G.end(), NEG);
         G[(size_t)k * budget + 0] = 0.0;
@@ -336,7 +343,7 @@ int tree_shape_dp(const double* accept, int k, int budget, int max_depth, int32_
                 double best = NEG;
                 int arg = 0;
                 for (int t = 1; t <= s; ++t) {
-                    const double f = F[d - 1][t], g = gn[s - t];
+                    const double f = T.F[d - 1][t], g = gn[s - t];
                     if (f == NEG || g == NEG) continue;
                     const double grow = 1.0 + f;
                     const double take = accept[i] * grow;
@@ -350,22 +357,27 @@ int tree_shape_dp(const double* accept, int k, int budget, int max_depth, int32_
                 ch[(size_t)i * budget + s] = arg;
             }
         }
-        for (int nn = 2; nn <= budget; ++nn) F[d][nn] = G[nn - 1];
+        for (int nn = 2; nn <= budget; ++nn) T.F[d][nn] = G[nn - 1];
     }
-    int n_best = 1;
-    for (int nn = 2; nn <= budget; ++nn)
-        if (F[D][nn] > F[D][n_best]) n_best = nn;
-    // rebuild the rank paths of every node
+}
+
+bool path_less(const std::vector<int>& x, const std::vector<int>& y) {
+    if (x.size() != y.size()) return x.size() < y.size();
+    return x < y;
+}
+
+// The n-node tree of the table, numbered by depth, then by the ranks along the path.
+int shape_rebuild(const ShapeTable& T, int n_nodes, int32_t* parent, int32_t* rank) {
     std::vector<std::vector<int>> paths;
     struct Item { std::vector<int> path; int d, n; };
-    std::vector<Item> stack{{{}, D, n_best}};
+    std::vector<Item> stack{{{}, T.D, n_nodes}};
     while (!stack.empty()) {
         Item it = stack.back();
         stack.pop_back();
         paths.push_back(it.path);
         int s = it.n - 1, i = 0;
         while (s > 0) {
-            const int t = choice[it.d][(size_t)i * budget + s];
+            const int t = T.choice[it.d][(size_t)i * T.budget + s];
             std::vector<int> p = it.path;
             p.push_back(i);
             stack.push_back({p, it.d - 1, t});
@@ -373,29 +385,60 @@ int tree_shape_dp(const double* accept, int k, int budget, int max_depth, int32_
             ++i;
         }
     }
-    std::sort(paths.begin(), paths.end(), [](const std::vector<int>& x, const std::vector<int>& y) {
-        if (x.size() != y.size()) return x.size() < y.size();
-        return x < y;
-    });
+    std::sort(paths.begin(), paths.end(), path_less);
     const int n = (int)paths.size();
-    for (int j = 0; j < budget; ++j) {
+    for (int j = 0; j < T.budget; ++j) {
         parent[j] = -1;
         rank[j] = -1;
     }
     for (int j = 1; j < n; ++j) {
         std::vector<int> up(paths[j].begin(), paths[j].end() - 1);
         // the parent's path is shorter, so it sits before j in the sorted list
-        const int p = (int)(std::lower_bound(paths.begin(), paths.begin() + j, up,
-                                             [](const std::vector<int>& x, const std::vector<int>& y) {
-                                                 if (x.size() != y.size()) return x.size() < y.size();
-                                                 return x < y;
-                                             }) -
-                            paths.begin());
-        parent[j] = p;
+        parent[j] = (int)(std::lower_bound(paths.begin(), paths.begin() + j, up, path_less) - paths.begin());
         rank[j] = paths[j].back();
     }
-    *value = F[D][n_best];
     return n;
+}
+
+int depth_levels(int budget, int max_depth) {
+    return (max_depth <= 0 || max_depth > budget - 1) ? budget - 1 : max_depth;
+}
+
+}  // namespace
+
+int tree_shape_dp(const double* accept, int k, int budget, int max_depth, int32_t* parent, int32_t* rank,
+                  double* value) {
+    ShapeTable T;
+    shape_table(accept, k, budget, depth_levels(budget, max_depth), T);
+    int n_best = 1;
+    for (int nn = 2; nn <= budget; ++nn)
+        if (T.F[T.D][nn] > T.F[T.D][n_best]) n_best = nn;
+    *value = T.F[T.D][n_best];
+    return shape_rebuild(T, n_best, parent, rank);
+}
+
+// The size whose best tree gives the largest step speedup
+// (1 + E) / (draft_cost + 1 + alpha (n - 1)); the smallest such size on ties.
+int tree_shape_for_cost(const double* accept, int k, int max_budget, int max_depth, double draft_cost, double alpha,
+                        int32_t* parent, int32_t* rank, double* value, double* speedup) {
+    ShapeTable T;
+    shape_table(accept, k, max_budget, depth_levels(max_budget, max_depth), T);
+    int n_best = 1;
+    double best = -INFINITY;
+    for (int nn = 1; nn <= max_budget; ++nn) {
+        const double f = T.F[T.D][nn];
+        if (f == -INFINITY) continue;
+        const double gain = 1.0 + f;
+        const double cost = draft_cost + 1.0 + alpha * (double)(nn - 1);
+        const double sp = gain / cost;
+        if (sp > best) {
+            best = sp;
+            n_best = nn;
+        }
+    }
+    *value = T.F[T.D][n_best];
+    *speedup = best;
+    return shape_rebuild(T, n_best, parent, rank);
 }
 
 // ---------------------------------------------------------------- dynamic selection
