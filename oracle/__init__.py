@@ -33,6 +33,8 @@ decoding):
 * :func:`step_speedup`, :func:`tree_shape_for_cost` -- the step's speedup
   over plain decoding and the tree size that maximises it (LLM Primer VI
   ch. 9, 9.3).
+* :func:`merge_sequences` -- SpecInfer's token tree: several drafts' sequences
+  merged on their common prefixes (glossary, "SpecInfer").
 * :func:`select_tree` -- the dynamic tree: the best-scoring ancestor-closed
   candidates under a node budget (LLM Primer VI ch. 9, 9.2, EAGLE-2).
 
@@ -412,6 +414,32 @@ def tree_shape_for_cost(accept, max_budget: int, max_depth: int | None, draft_co
         if best is None or sp > best[3]:
             best = (parent, rank, value, sp)
     return best
+
+
+def merge_sequences(seqs):
+    """SpecInfer's token tree (glossary "Tree-based speculative decoding",
+    section "SpecInfer", token tree construction): every draft model generates
+    its own candidate sequence and the sequences are merged, candidates with a
+    common prefix sharing those nodes.  Node 0 is the root (the last committed
+    token); nodes are created in input order, each the first time its prefix
+    appears.  Returns (parent_idx, tree_tokens, node_of): node_of[k][j] is the
+    node of token j of sequence k."""
+    parent, tokens = [-1], [-1]
+    child = {}
+    node_of = []
+    for seq in seqs:
+        u = 0
+        path = []
+        for t in seq:
+            key = (u, int(t))
+            if key not in child:
+                child[key] = len(parent)
+                parent.append(u)
+                tokens.append(int(t))
+            u = child[key]
+            path.append(u)
+        node_of.append(path)
+    return np.array(parent, np.int32), np.array(tokens, np.int32), node_of
 
 
 def select_tree(cand_parent, cand_token, cand_prob, budget: int):

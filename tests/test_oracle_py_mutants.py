@@ -52,6 +52,7 @@ MUTANTS = [
      "return (1.0 + expected_accepted) / (draft_cost + 1.0 + alpha * num_nodes)", TREE),
     ("speedup_without_the_bonus", "return (1.0 + expected_accepted) / (draft_cost + 1.0 + alpha * (num_nodes - 1))",
      "return expected_accepted / (draft_cost + 1.0 + alpha * (num_nodes - 1))", TREE),
+    ("merge_keys_on_token_only", "            key = (u, int(t))", "            key = (0, int(t))", TREE),
     ("softmax_wrong_axis", "return (e / e.sum(axis=-1, keepdims=True)).astype(np.float32)",
      "return (e / e.sum(axis=0, keepdims=True)).astype(np.float32)", LOGITS),
 ]

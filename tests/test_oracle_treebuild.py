@@ -187,3 +187,40 @@ def test_speedup_limits():
     assert value == v_all and sp == 1.0 + v_all
     # drafting that costs a whole decode step halves the speedup of a one-node tree
     assert oracle.step_speedup(0.0, 1, 1.0, 0.1) == 0.5
+
+
+def test_merging_two_drafts_gives_the_pages_five_node_tree():
+    """Two drafts A1 A2 and B1 B2 merge into the blog's tree T0 -> A1 -> A2,
+    T0 -> B1 -> B2 (section 3, "Tree Attention Verification Matrix"), whose
+    ancestor mask is the one the pages print."""
+    from helpers import golden_lines
+    A1, A2, B1, B2 = 101, 102, 201, 202
+    parent, tokens, node_of = oracle.merge_sequences([[A1, A2], [B1, B2]])
+    assert tokens.tolist() == [-1, A1, A2, B1, B2]
+    assert parent.tolist() == [-1, 0, 1, 0, 3]
+    assert node_of == [[1, 2], [3, 4]]
+    rows = list(golden_lines("tree_mask_5node.txt"))
+    assert [int(x) for x in rows[0][1:]] == parent.tolist()  # the golden file's parent line
+    want = [[int(x) for x in row[1:]] for row in rows[1:]]
+    assert oracle.tree_mask(parent).tolist() == want
+
+
+def test_merged_prefixes_are_shared():
+    rng = np.random.default_rng(9)
+    seqs = [list(rng.integers(0, 3, rng.integers(0, 7))) for _ in range(12)]
+    seqs.append(list(seqs[0]))  # a repeated draft adds nothing
+    parent, tokens, node_of = oracle.merge_sequences(seqs)
+    prefixes = {tuple(s[:j + 1]) for s in seqs for j in range(len(s))}
+    assert len(parent) == 1 + len(prefixes)
+    assert all(0 <= parent[c] < c for c in range(1, len(parent)))
+    for s, nodes in zip(seqs, node_of):
+        # every draft is a root path of the tree
+        u = 0
+        for t, v in zip(s, nodes):
+            assert parent[v] == u and tokens[v] == t
+            u = v
+    # siblings carry distinct tokens
+    seen = set()
+    for c in range(1, len(parent)):
+        assert (parent[c], tokens[c]) not in seen
+        seen.add((parent[c], tokens[c]))
