@@ -363,6 +363,29 @@ TV_API tv_status tv_tree_shape(const double *accept, int32_t num_ranks, int32_t 
                                double *expected_accepted);
 
 /*
+ * Building the draft tree from several drafts: SpecInfer's token tree.
+ * Glossary "Tree-based speculative decoding", section "SpecInfer": each draft
+ * model (SSM) generates its own candidate sequence, and the sequences are
+ * merged into one token tree in which candidates with a common prefix share
+ * those nodes.
+ *
+ * Sequence k is tokens[seq_offsets[k] .. seq_offsets[k+1]) (token ids >= 0;
+ * seq_offsets has num_seqs + 1 entries, starts at 0 and does not decrease).
+ * Node 0 is the root (the last committed token: parent -1, token -1); walking
+ * each sequence from the root in input order, every (node, token) pair not
+ * seen before becomes the next node, so parents come before children and
+ * siblings appear in the order the drafts proposed them (the order the walk
+ * tries them).  Outputs (host int32): parent_idx and tree_tokens of max_nodes
+ * entries (the rest -1), node_of_token[j] = the node of tokens[j], *num_nodes.
+ * Host computation only.  Errors: null pointers, max_nodes < 1, bad offsets or
+ * a negative token: TV_ERR_INVALID_ARG (nothing written); a tree larger than
+ * max_nodes: TV_ERR_UNSUPPORTED (the outputs then hold a partial tree).
+ */
+TV_API tv_status tv_tree_merge(int32_t num_seqs, const int32_t *seq_offsets, const int32_t *tokens,
+                               int32_t max_nodes, int32_t *parent_idx, int32_t *tree_tokens,
+                               int32_t *node_of_token, int32_t *num_nodes);
+
+/*
  * The tree size that pays.  LLM Primer VI ch. 9, 9.3: a step's speedup over
  * plain decoding is E[emitted tokens] / (T_draft/T_decode + 1 + alpha N), with
  * alpha the verification overhead per position (0.05-0.15) and N the draft

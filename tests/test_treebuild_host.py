@@ -121,3 +121,30 @@ def test_cost_aware_shape_rejects_bad_costs():
     assert f(tv._hptr(acc), 1, 8, 0, 0.0, float("nan"), *[tv._hptr(x) for x in out]) == tv.TV_ERR_INVALID_ARG
     assert f(tv._hptr(acc), 1, 8, 0, float("inf"), 0.1, *[tv._hptr(x) for x in out]) == tv.TV_ERR_INVALID_ARG
     assert f(tv._hptr(acc), 1, 300, 0, 0.0, 0.1, *[tv._hptr(x) for x in out]) == tv.TV_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_library_merge_equals_oracle(seed):
+    rng = np.random.default_rng(300 + seed)
+    K = int(rng.integers(0, 9))
+    seqs = [list(rng.integers(0, 4 if seed % 2 else 128256, rng.integers(0, 12))) for _ in range(K)]
+    parent, tokens, node_of = tv.tree_merge(seqs)
+    rp, rt, rn = oracle.merge_sequences(seqs)
+    np.testing.assert_array_equal(parent, rp)
+    np.testing.assert_array_equal(tokens, rt)
+    assert [list(x) for x in node_of] == rn
+
+
+def test_merge_rejects_bad_arguments():
+    out = [np.zeros(4, np.int32), np.zeros(4, np.int32), np.zeros(8, np.int32), np.zeros(1, np.int32)]
+    off = np.array([0, 2, 4], np.int32)
+    tok = np.array([1, 2, 3, 4], np.int32)
+    f = tv.lib().tv_tree_merge
+    h = [tv._hptr(x) for x in out]
+    assert f(2, tv._hptr(off), tv._hptr(tok), 8, *[tv._hptr(x) for x in
+             (np.zeros(8, np.int32), np.zeros(8, np.int32), np.zeros(8, np.int32), out[3])]) == tv.TV_OK
+    assert out[3][0] == 5
+    assert f(2, tv._hptr(off), tv._hptr(tok), 4, *h) == tv.TV_ERR_UNSUPPORTED  # 5 nodes do not fit in 4
+    assert f(2, tv._hptr(np.array([1, 2, 4], np.int32)), tv._hptr(tok), 8, *h) == tv.TV_ERR_INVALID_ARG
+    assert f(2, tv._hptr(off), tv._hptr(np.array([1, -2, 3, 4], np.int32)), 8, *h) == tv.TV_ERR_INVALID_ARG
+    assert f(2, tv._hptr(off), tv._hptr(tok), 0, *h) == tv.TV_ERR_INVALID_ARG

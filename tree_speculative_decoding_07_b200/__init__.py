@@ -79,6 +79,7 @@ def lib() -> ctypes.CDLL:
         L.tv_tree_fill_topk.argtypes = [ctypes.POINTER(TvSampleDesc), P, P, P, P, P, P]
         L.tv_tree_shape.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, P, P]
         L.tv_tree_select.argtypes = [P, P, P, ctypes.c_int32, ctypes.c_int32, P, P, P, P, P]
+        L.tv_tree_merge.argtypes = [ctypes.c_int32, P, P, ctypes.c_int32, P, P, P, P]
         L.tv_tree_shape_for_cost.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_double,
                                              ctypes.c_double, P, P, P, P, P]
         L.tv_tree_select_batch.argtypes = [ctypes.c_int32, P, P, P, P, ctypes.c_int32, P, P, P, P, P]
@@ -88,7 +89,7 @@ def lib() -> ctypes.CDLL:
         for name in ("tv_tree_attention_plan", "tv_tree_attention", "tv_tree_attention_static",
                      "tv_verify_sample_plan", "tv_verify_sample", "tv_commit_path", "tv_verify_sample_logits",
                      "tv_tree_fill_topk", "tv_tree_shape", "tv_tree_select", "tv_tree_select_batch",
-                     "tv_tree_shape_for_cost"):
+                     "tv_tree_shape_for_cost", "tv_tree_merge"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -235,6 +236,27 @@ def tree_shape_for_cost(accept, max_budget: int, max_depth: int = 0, draft_cost:
         raise TreeVerifyError(s, "tv_tree_shape_for_cost")
     k = int(n[0])
     return parent[:k].copy(), rank[:k].copy(), float(val[0]), float(sp[0])
+
+
+def tree_merge(seqs, max_nodes: int = 1024):
+    """SpecInfer's token tree from several drafts' sequences; returns
+    (parent_idx, tree_tokens, node_of) with node_of a list of per-sequence
+    node arrays."""
+    import numpy as np
+    lens = [len(s) for s in seqs]
+    off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    tok = np.ascontiguousarray(np.concatenate([np.asarray(s, np.int64) for s in seqs]) if seqs else np.zeros(0),
+                               dtype=np.int32)
+    parent = np.empty(int(max_nodes), np.int32)
+    tokens = np.empty_like(parent)
+    node_of = np.empty(max(tok.size, 1), np.int32)
+    n = np.zeros(1, np.int32)
+    s = int(lib().tv_tree_merge(len(seqs), _hptr(off), _hptr(tok), int(max_nodes), _hptr(parent), _hptr(tokens),
+                                _hptr(node_of), _hptr(n)))
+    if s != TV_OK:
+        raise TreeVerifyError(s, "tv_tree_merge")
+    k = int(n[0])
+    return parent[:k].copy(), tokens[:k].copy(), [node_of[off[i]:off[i + 1]].copy() for i in range(len(seqs))]
 
 
 def tree_select_batch(cand_offsets, cand_parent, cand_token, cand_prob, budget: int):

@@ -284,6 +284,23 @@ tv_status tv_tree_shape_for_cost(const double* accept, int32_t num_ranks, int32_
     return TV_OK;
 }
 
+tv_status tv_tree_merge(int32_t num_seqs, const int32_t* seq_offsets, const int32_t* tokens, int32_t max_nodes,
+                        int32_t* parent_idx, int32_t* tree_tokens, int32_t* node_of_token, int32_t* num_nodes) {
+    if (num_seqs < 0 || !seq_offsets || !parent_idx || !tree_tokens || !num_nodes || max_nodes < 1)
+        return TV_ERR_INVALID_ARG;
+    if (seq_offsets[0] != 0) return TV_ERR_INVALID_ARG;
+    for (int k = 0; k < num_seqs; ++k)
+        if (seq_offsets[k + 1] < seq_offsets[k]) return TV_ERR_INVALID_ARG;
+    const int32_t total = seq_offsets[num_seqs];
+    if (total > 0 && (!tokens || !node_of_token)) return TV_ERR_INVALID_ARG;
+    for (int32_t j = 0; j < total; ++j)
+        if (tokens[j] < 0) return TV_ERR_INVALID_ARG;
+    const int n = tv::tree_merge(num_seqs, seq_offsets, tokens, max_nodes, parent_idx, tree_tokens, node_of_token);
+    if (n < 0) return TV_ERR_UNSUPPORTED;
+    *num_nodes = n;
+    return TV_OK;
+}
+
 tv_status tv_tree_select(const int32_t* cand_parent, const int32_t* cand_token, const double* cand_prob,
                          int32_t num_candidates, int32_t budget, int32_t* parent_idx, int32_t* tree_tokens,
                          int32_t* cand_index, int32_t* num_nodes, double* expected_accepted) {

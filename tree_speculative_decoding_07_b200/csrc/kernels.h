@@ -95,6 +95,11 @@ int tree_shape_dp(const double* accept, int k, int budget, int max_depth, int32_
 int tree_shape_for_cost(const double* accept, int k, int max_budget, int max_depth, double draft_cost, double alpha,
                         int32_t* parent, int32_t* rank, double* value, double* speedup);
 
+// SpecInfer's token-tree merge of several drafts' sequences (host).  Returns the
+// node count, -1 if it would exceed max_nodes.
+int tree_merge(int num_seqs, const int32_t* offsets, const int32_t* tokens, int max_nodes, int32_t* parent_idx,
+               int32_t* tree_tokens, int32_t* node_of);
+
 // Dynamic tree selection from a candidate set (host).  Returns the node count, -1 if not topological.
 int tree_select(const int32_t* cand_parent, const int32_t* cand_token, const double* cand_prob, int M, int budget,
                 int32_t* parent_idx, int32_t* tree_tokens, int32_t* cand_index, double* value);

@@ -21,6 +21,7 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <unordered_map>
 #include <vector>
 
 #include "kernels.h"
@@ -439,6 +440,42 @@ int tree_shape_for_cost(const double* accept, int k, int max_budget, int max_dep
     *value = T.F[T.D][n_best];
     *speedup = best;
     return shape_rebuild(T, n_best, parent, rank);
+}
+
+// ---------------------------------------------------------------- token-tree merge
+
+// Sequences k = 0.. (tokens[offsets[k] .. offsets[k+1])) merge into one tree:
+// node 0 is the root; walking a sequence from the root, each (node, token)
+// pair not seen before becomes a new node, so common prefixes share nodes and
+// nodes appear in input order.  Returns the node count, or -1 when it would
+// exceed max_nodes (nothing past max_nodes is written).
+int tree_merge(int num_seqs, const int32_t* offsets, const int32_t* tokens, int max_nodes, int32_t* parent_idx,
+               int32_t* tree_tokens, int32_t* node_of) {
+    std::unordered_map<uint64_t, int32_t> child;
+    parent_idx[0] = -1;
+    tree_tokens[0] = -1;
+    int n = 1;
+    for (int k = 0; k < num_seqs; ++k) {
+        int32_t u = 0;
+        for (int32_t j = offsets[k]; j < offsets[k + 1]; ++j) {
+            const uint64_t key = ((uint64_t)(uint32_t)u << 32) | (uint32_t)tokens[j];
+            auto it = child.find(key);
+            if (it == child.end()) {
+                if (n >= max_nodes) return -1;
+                parent_idx[n] = u;
+                tree_tokens[n] = tokens[j];
+                it = child.emplace(key, n).first;
+                ++n;
+            }
+            u = it->second;
+            node_of[j] = u;
+        }
+    }
+    for (int j = n; j < max_nodes; ++j) {
+        parent_idx[j] = -1;
+        tree_tokens[j] = -1;
+    }
+    return n;
 }
 
 // ---------------------------------------------------------------- dynamic selection
