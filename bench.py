@@ -665,10 +665,19 @@ def cpu_baseline(wl, h, budget_s: float = 20.0):
         if frac >= 1.0 and time.perf_counter() - t_start > budget_s / 2:
             break
     per_step = t_sum / steps
+    # the same step on one core, on a smaller attention sample (a few seconds at most)
+    oracle.set_threads(1)
+    try:
+        t1, n1, _ = oracle_step_times(wl, h, 1.0 / 256)
+    finally:
+        oracle.set_threads(cores)
     return {"value": int(wl.counts.sum()) / per_step, "unit": "nodes/s", "cores": cores, "kind": "oracle",
             "sample": f"{steps} oracle step(s): attention on {rows_done // steps} of {total} query rows "
                       f"(time scaled to all rows) plus the full fp64 acceptance walk; "
-                      f"{per_step * 1e3:.1f} ms per full step"}
+                      f"{per_step * 1e3:.1f} ms per full step",
+            "single_thread": {"value": int(wl.counts.sum()) / t1, "unit": "nodes/s", "cores": 1,
+                              "sample": f"one step: attention on {n1} of {total} query rows (time scaled to all "
+                                        f"rows) plus the full acceptance walk; {t1 * 1e3:.1f} ms per full step"}}
 
 
 def run_reference(args, rank, world):
