@@ -31,6 +31,7 @@ import numpy as np  # noqa: E402
 
 METRIC = "tree nodes verified/s and µs per verify step; achieved HBM GB/s vs B200 peak"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_SUSTAINED = 1400.0  # TFLOP/s, the profiling recipe's sustained figure
 NOMINAL_HBM_GBS = 8000.0  # the "~8 TB/s" spec figure, reported beside the measured copy bandwidth
 L2_FLUSH_BYTES = 512 << 20
 
@@ -408,6 +409,173 @@ def time_fill_topk(tv, wl, d, flush, stream, W, K):
                     "launches, L2 flushed before each"}
 
 
+def to_device(h: dict) -> dict:
+    import torch
+
+    def dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+    return {k: dev(v) for k, v in h.items()}
+
+
+class Step:
+    """One verification step of a workload on the device: the tree-attention
+    call and the acceptance walk, over `copies` independent copies of every
+    input (for back-to-back timing with a working set larger than L2)."""
+
+    def __init__(self, tv, wl, h, copies: int = 1):
+        import torch
+        self.tv, self.wl = tv, wl
+        base = to_device(h)
+        self.inputs = [base] + [{k: t.clone() for k, t in base.items()} for _ in range(copies - 1)]
+        d = base
+        B, N = wl.batch, wl.num_nodes
+        self.out = torch.empty_like(d["query"])
+        self.path = torch.empty((B, N), dtype=torch.int32, device="cuda")
+        self.alen = torch.empty((B,), dtype=torch.int32, device="cuda")
+        self.bonus = torch.empty((B,), dtype=torch.int32, device="cuda")
+        self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.adesc = tv.attn_desc(d["query"], d["k"], d["block_table"], node_counts=d.get("node_counts"))
+        self.aplan = tv.tv_tree_attention_plan(self.adesc)
+        self.ws_bytes = self.aplan.workspace_bytes
+        self.ws = torch.zeros(max(self.ws_bytes, 256), dtype=torch.uint8, device="cuda")
+        self.sdescs = [tv.TvSampleDesc(B, N, wl.vocab, tv._ptr(x.get("node_counts"))) for x in self.inputs]
+        self.splan = tv.tv_verify_sample_plan(self.sdescs[0])
+        self.adescs = [tv.attn_desc(x["query"], x["k"], x["block_table"], node_counts=x.get("node_counts"))
+                       for x in self.inputs]
+
+    def attn(self, st, i: int = 0):
+        d = self.inputs[i]
+        s = self.tv.tv_tree_attention(self.adescs[i], d["query"], d["k"], d["v"], d["block_table"], d["prefix_lens"],
+                                      d["parent_idx"], self.out, self.ws, self.ws_bytes, self.status, st)
+        if s:
+            raise self.tv.TreeVerifyError(s, "tv_tree_attention")
+
+    def sample(self, st, i: int = 0):
+        d = self.inputs[i]
+        s = self.tv.tv_verify_sample(self.sdescs[i], d["p"], d["q"], d["tokens"], d["parent_idx"], d["uniforms"],
+                                     self.path, self.alen, self.bonus, None, 0, self.status, st)
+        if s:
+            raise self.tv.TreeVerifyError(s, "tv_verify_sample")
+
+    def graph(self, fn):
+        """Capture fn(stream) into a CUDA graph."""
+        import torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn(torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        return g
+
+    def check_status(self, what: str):
+        if int(self.status.item()) != 0:
+            raise RuntimeError(f"device status {int(self.status.item())} after {what}")
+
+    def walk(self) -> dict:
+        return {"path": self.path.cpu().numpy(), "alen": self.alen.cpu().numpy(), "bonus": self.bonus.cpu().numpy()}
+
+
+def timed_replays(graph, flush, stream, W: int, K: int):
+    """Device time of each of K replays of graph (ms), L2 flushed before each."""
+    import torch
+    for _ in range(W):
+        flush.zero_()
+        graph.replay()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return [e0.elapsed_time(e1) for e0, e1 in ev]
+
+
+def back_to_back_us(graph, per_graph: int, stream, W: int, reps: int) -> float:
+    """Device time per unit (µs) of `reps` replays of a graph holding
+    `per_graph` units launched back to back (no flush, no gap)."""
+    import torch
+    for _ in range(W):
+        graph.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / (reps * per_graph)
+
+
+def rotation_copies(read_bytes: int, input_bytes: int, l2_bytes: int, mem_cap: int = 24 << 30) -> int:
+    """Input copies for back-to-back timing: at least 4, and enough that one
+    pass over them reads at least twice the L2 size, within a memory cap."""
+    want = max(4, -(-2 * l2_bytes // max(read_bytes, 1)))
+    return int(max(4, min(want, mem_cap // max(input_bytes, 1))))
+
+
+def tensor_flops(wl) -> int:
+    """Attention FLOPs of one call: 2 * 2 * D per (query row, visible key), with
+    every query row of a sequence's KV head reading the whole prefix plus the
+    tree block (the MMA tile computes the masked entries too)."""
+    G = wl.num_q_heads // wl.num_kv_heads
+    tok = (wl.prefix_lens.astype(np.int64) + wl.counts).astype(np.int64)
+    return int(4 * wl.head_dim * (tok * wl.counts * G).sum() * wl.num_kv_heads)
+
+
+def measure_config(tv, name: str, seed: int, W: int, K: int, flush, stream, peaks: dict, full: bool):
+    """GPU-only figures of one workload: the attention call and the walk, each
+    timed alone with L2 flushed before every launch, and back to back over
+    rotating input copies."""
+    import torch
+    wl, h = make_inputs(name, seed=seed)
+    a_bytes = attention_bytes(wl)
+    in_bytes = int(sum(v.nbytes for v in h.values()))
+    l2 = int(getattr(torch.cuda.get_device_properties(torch.cuda.current_device()), "L2_cache_size", 126 << 20))
+    copies = rotation_copies(a_bytes + 8 * wl.vocab * 3, in_bytes, l2)
+    st = Step(tv, wl, h, copies)
+    st.attn(stream)
+    st.sample(stream)
+    torch.cuda.synchronize()
+    st.check_status(name)
+    walk = st.walk()
+    s_bytes = sampler_bytes(wl, h, walk["path"], walk["alen"])
+    g_a = st.graph(lambda s: st.attn(s))
+    g_s = st.graph(lambda s: st.sample(s))
+    attn_ms = timed_replays(g_a, flush, stream, W, K)
+    samp_ms = timed_replays(g_s, flush, stream, W, K)
+    g_ab = st.graph(lambda s: [st.attn(s, i) for i in range(copies)])
+    g_sb = st.graph(lambda s: [st.sample(s, i) for i in range(copies)])
+    g_tb = st.graph(lambda s: [(st.attn(s, i), st.sample(s, i)) for i in range(copies)])
+    reps = max(3, min(200, K // copies + 1))
+    a_b2b = back_to_back_us(g_ab, copies, stream, 2, reps)
+    s_b2b = back_to_back_us(g_sb, copies, stream, 2, reps)
+    t_b2b = back_to_back_us(g_tb, copies, stream, 2, reps)
+    st.check_status(name)
+    hbm = peaks["hbm"]
+    a_us = float(np.mean(attn_ms)) * 1e3
+    res = {
+        "workload": workload_config(name, wl, 1)["workload"],
+        "attention_us": a_us, "sample_us": float(np.mean(samp_ms)) * 1e3,
+        "attention_hbm_frac": a_bytes / (a_us * 1e-6) / 1e9 / hbm,
+        "back_to_back": {"copies": copies, "step_us": t_b2b, "attention_us": a_b2b, "sample_us": s_b2b,
+                         "attention_hbm_frac": a_bytes / (a_b2b * 1e-6) / 1e9 / hbm,
+                         "step_hbm_frac": (a_bytes + s_bytes) / (t_b2b * 1e-6) / 1e9 / hbm,
+                         "nodes_per_s": int(wl.counts.sum()) / (t_b2b * 1e-6)},
+        "attention_bytes": a_bytes, "sampler_bytes": s_bytes,
+        "kernel": "attn_tc" if st.aplan.kernel == 0 else "attn_simt", "splits": st.aplan.num_splits,
+    }
+    if wl.dtype == "bf16":
+        fl = tensor_flops(wl)
+        res["attention_tflops"] = fl / (a_us * 1e-6) / 1e12
+        res["attention_tensor_frac_sustained"] = res["attention_tflops"] / peaks["bf16_sustained"]
+        res["back_to_back"]["attention_tensor_frac_sustained"] = fl / (a_b2b * 1e-6) / 1e12 / peaks["bf16_sustained"]
+    del g_a, g_s, g_ab, g_sb, g_tb
+    return res, (wl, h, st, walk, attn_ms, samp_ms)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -416,43 +584,15 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     wl, h = make_inputs(args.workload, seed=1 + 1000 * rank)
-
-    def dev(a):
-        if a.dtype == np.uint16:
-            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
-        return torch.from_numpy(np.ascontiguousarray(a)).cuda()
-
-    d = {k: dev(v) for k, v in h.items()}
-    out = torch.empty_like(d["query"])
+    st = Step(tv, wl, h)
+    d = st.inputs[0]
     B, N = wl.batch, wl.num_nodes
-    path = torch.empty((B, N), dtype=torch.int32, device="cuda")
-    alen = torch.empty((B,), dtype=torch.int32, device="cuda")
-    bonus = torch.empty((B,), dtype=torch.int32, device="cuda")
-    status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    adesc = tv.attn_desc(d["query"], d["k"], d["block_table"], node_counts=d.get("node_counts"))
-    aplan = tv.tv_tree_attention_plan(adesc)
-    ws_bytes = aplan.workspace_bytes
-    ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
-    sdesc = tv.TvSampleDesc(B, N, wl.vocab, tv._ptr(d.get("node_counts")))
-    splan = tv.tv_verify_sample_plan(sdesc)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
-    def attn_call(st):
-        s1 = tv.tv_tree_attention(adesc, d["query"], d["k"], d["v"], d["block_table"], d["prefix_lens"],
-                                  d["parent_idx"], out, ws, ws_bytes, status, st)
-        if s1:
-            raise tv.TreeVerifyError(s1, "tv_tree_attention")
-
-    def sample_call(st):
-        s2 = tv.tv_verify_sample(sdesc, d["p"], d["q"], d["tokens"], d["parent_idx"], d["uniforms"], path, alen,
-                                 bonus, None, 0, status, st)
-        if s2:
-            raise tv.TreeVerifyError(s2, "tv_verify_sample")
-
     def step():
-        attn_call(stream)
-        sample_call(stream)
+        st.attn(stream)
+        st.sample(stream)
 
     # ---- device-resident timing (L2 flushed before every step).  The step is
     # replayed from one CUDA graph (attention, then the walk, launched with a
@@ -463,15 +603,9 @@ def run_ours(args, rank, world, local_rank):
     for _ in range(2):
         step()
     torch.cuda.synchronize()
-    g_step, g_attn, g_samp = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step):
-        attn_call(torch.cuda.current_stream())
-        sample_call(torch.cuda.current_stream())
-    with torch.cuda.graph(g_attn):
-        attn_call(torch.cuda.current_stream())
-    with torch.cuda.graph(g_samp):
-        sample_call(torch.cuda.current_stream())
-    torch.cuda.synchronize()
+    g_step = st.graph(lambda s: (st.attn(s), st.sample(s)))
+    g_attn = st.graph(lambda s: st.attn(s))
+    g_samp = st.graph(lambda s: st.sample(s))
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     for _ in range(W):
         flush.zero_()
@@ -496,37 +630,24 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     step_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
+    st.check_status("the timed steps")
 
-    def kernel_ms(graph):
-        for _ in range(W):
-            flush.zero_()
-            graph.replay()
-        for k in range(K):
-            flush.zero_()
-            ev[k][0].record(stream)
-            graph.replay()
-            ev[k][1].record(stream)
-        torch.cuda.synchronize()
-        return [e0.elapsed_time(e1) for e0, e1 in ev]
-
-    attn_ms = kernel_ms(g_attn)
-    samp_ms = kernel_ms(g_samp)
-    walk = {"path": path.cpu().numpy(), "alen": alen.cpu().numpy(), "bonus": bonus.cpu().numpy()}
+    attn_ms = timed_replays(g_attn, flush, stream, W, K)
+    samp_ms = timed_replays(g_samp, flush, stream, W, K)
+    walk = st.walk()
     commit = time_commit(tv, wl, d, flush, stream, W, min(K, 200))
     logits_walk = time_logits_walk(tv, wl, d, flush, stream, W, min(K, 200), walk)
     fill = time_fill_topk(tv, wl, d, flush, stream, W, min(K, 200))
     total_ms = float(sum(step_ms))
-    if int(status.item()) != 0:
-        raise RuntimeError(f"device status {int(status.item())}")
 
     # ---- end to end: host (pinned) inputs -> device -> results back, every step
     pin = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16) if v.dtype == np.uint16
                                else np.ascontiguousarray(v)).pin_memory() for k, v in h.items()}
     h2d = int(sum(v.numel() * v.element_size() for v in pin.values()))
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    path_h = torch.empty(path.shape, dtype=torch.int32).pin_memory()
-    alen_h = torch.empty(alen.shape, dtype=torch.int32).pin_memory()
-    bonus_h = torch.empty(bonus.shape, dtype=torch.int32).pin_memory()
+    out_h = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+    path_h = torch.empty(st.path.shape, dtype=torch.int32).pin_memory()
+    alen_h = torch.empty(st.alen.shape, dtype=torch.int32).pin_memory()
+    bonus_h = torch.empty(st.bonus.shape, dtype=torch.int32).pin_memory()
     d2h = sum(t.numel() * t.element_size() for t in (out_h, path_h, alen_h, bonus_h))
     K2 = max(3, min(K, 50))
 
@@ -535,10 +656,10 @@ def run_ours(args, rank, world, local_rank):
             dst = d[key]
             (dst.view(torch.int16) if dst.dtype == torch.bfloat16 else dst).copy_(t, non_blocking=True)
         step()
-        out_h.copy_(out, non_blocking=True)
-        path_h.copy_(path, non_blocking=True)
-        alen_h.copy_(alen, non_blocking=True)
-        bonus_h.copy_(bonus, non_blocking=True)
+        out_h.copy_(st.out, non_blocking=True)
+        path_h.copy_(st.path, non_blocking=True)
+        alen_h.copy_(st.alen, non_blocking=True)
+        bonus_h.copy_(st.bonus, non_blocking=True)
 
     for _ in range(3):
         e2e_step()
@@ -552,6 +673,21 @@ def run_ours(args, rank, world, local_rank):
     a1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = a0.elapsed_time(a1)
+    st.check_status("the end-to-end steps")
+
+    # ---- every workload, GPU only (back-to-back figures beside the flushed ones)
+    peak, peak_kind, pk = load_peaks()
+    peaks = {"hbm": peak, "bf16_sustained": float(pk.get("bf16_tflops_sustained", FALLBACK_BF16_SUSTAINED))}
+    configs = {}
+    if not args.no_configs:
+        for name in ("tiny", "l8b", "l70b", "mix", "long", "ragged"):
+            try:
+                r, _ = measure_config(tv, name, 1 + 1000 * rank if name == args.workload else None, W,
+                                      min(K, 200), flush, stream, peaks, full=False)
+                configs[name] = r
+            except Exception as e:  # a failure is reported, not hidden
+                configs[name] = {"error": f"{type(e).__name__}: {e}"}
+            torch.cuda.empty_cache()
 
     total_ms, e2e_ms = reduce_max([total_ms, e2e_ms], world, "cuda")
     if rank != 0:
@@ -561,12 +697,11 @@ def run_ours(args, rank, world, local_rank):
     ms_step = total_ms / K
     value = job_throughput(world, nodes, K, total_ms)
     e2e_value = job_throughput(world, nodes, K2, e2e_ms)
-    peak, peak_kind, _ = load_peaks()
     a_bytes = attention_bytes(wl)
     s_bytes = sampler_bytes(wl, h, walk["path"], walk["alen"])
     attn_avg_s = (sum(attn_ms) / K) / 1e3
     achieved = a_bytes / attn_avg_s / 1e9
-    kernel_key = "attn_tc" if aplan.kernel == 0 else "attn_simt"
+    kernel_key = "attn_tc" if st.aplan.kernel == 0 else "attn_simt"
     line = {
         "metric": METRIC,
         "value": value,
@@ -601,12 +736,29 @@ def run_ours(args, rank, world, local_rank):
         "tree_fill_topk": fill,
         "e2e": {"value": e2e_value, "unit": "nodes/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": K2},
-        "gpu_launches": K * (aplan.launches + splan.launches),
+        "gpu_launches": K * (st.aplan.launches + st.splan.launches),
         "clocks": clk,
         "wall_s": t_wall,
     }
+    if args.workload in configs and "back_to_back" in configs[args.workload]:
+        line["back_to_back"] = dict(configs[args.workload]["back_to_back"],
+                                    note="steps replayed back to back from one graph over rotating input copies "
+                                         "(one pass over the copies reads at least twice the L2 size); no flush, "
+                                         "so launch gaps overlap with the previous kernel's tail")
+    if configs:
+        line["configs"] = configs
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, h, budget_s=args.cpu_budget)
+        ref = line["cpu_baseline"].pop("walk")
+        same = ((walk["alen"] == ref["accepted_len"]) & (walk["bonus"] == ref["bonus_token"])
+                & (walk["path"] == ref["accepted_path"]).all(axis=1))
+        line["walk_check"] = {
+            "near_threshold": int((ref["near"] > 0).sum()),
+            "matches_oracle": bool(same.all()),
+            "mismatches_outside_band": int((~same & ~(ref["near"] > 0)).sum()),
+            "sequences": int(B),
+            "note": "the timed inputs' walk against the oracle's (from the cpu_baseline leg); near_threshold counts "
+                    "sequences with a uniform within 1e-6 of an acceptance or CDF threshold"}
     return line
 
 
@@ -633,8 +785,8 @@ def oracle_step_times(wl, h, rows_frac: float):
             done += m
         t_attn = (time.perf_counter() - t0) * total_rows / done
         t0 = time.perf_counter()
-        oracle.verify_sample_ragged(h["p"], h["q"], h["tokens"], h["parent_idx"], h["uniforms"], wl.counts)
-        return t_attn + time.perf_counter() - t0, done, total_rows
+        walk = oracle.verify_sample_ragged(h["p"], h["q"], h["tokens"], h["parent_idx"], h["uniforms"], wl.counts)
+        return t_attn + time.perf_counter() - t0, done, total_rows, walk
     total_rows = B * N * Hq
     n = max(1, int(round(total_rows * rows_frac)))
     sel = np.linspace(0, total_rows - 1, n).astype(np.int64)
@@ -644,21 +796,21 @@ def oracle_step_times(wl, h, rows_frac: float):
                           wl.num_kv_heads, wl.dtype, rows=rows)
     t_attn = (time.perf_counter() - t0) * total_rows / n
     t0 = time.perf_counter()
-    oracle.verify_sample(h["p"], h["q"], h["tokens"], h["parent_idx"], h["uniforms"])
+    walk = oracle.verify_sample(h["p"], h["q"], h["tokens"], h["parent_idx"], h["uniforms"])
     t_walk = time.perf_counter() - t0
-    return t_attn + t_walk, n, total_rows
+    return t_attn + t_walk, n, total_rows, walk
 
 
 def cpu_baseline(wl, h, budget_s: float = 20.0):
     import oracle
     cores = oracle.max_threads()
     # calibrate with a small fraction, then size the sample to the budget
-    t_est, n, total = oracle_step_times(wl, h, 1.0 / 64)
+    t_est, n, total, walk = oracle_step_times(wl, h, 1.0 / 64)
     frac = min(1.0, max(1.0 / 64, budget_s / max(t_est, 1e-9)))
     steps, t_sum, rows_done = 0, 0.0, 0
     t_start = time.perf_counter()
     while time.perf_counter() - t_start < budget_s or steps == 0:
-        t, n, total = oracle_step_times(wl, h, frac)
+        t, n, total, walk = oracle_step_times(wl, h, frac)
         t_sum += t
         rows_done += n
         steps += 1
@@ -668,7 +820,7 @@ def cpu_baseline(wl, h, budget_s: float = 20.0):
     # the same step on one core, on a smaller attention sample (a few seconds at most)
     oracle.set_threads(1)
     try:
-        t1, n1, _ = oracle_step_times(wl, h, 1.0 / 256)
+        t1, n1, _, _ = oracle_step_times(wl, h, 1.0 / 256)
     finally:
         oracle.set_threads(cores)
     return {"value": int(wl.counts.sum()) / per_step, "unit": "nodes/s", "cores": cores, "kind": "oracle",
@@ -677,7 +829,8 @@ def cpu_baseline(wl, h, budget_s: float = 20.0):
                       f"{per_step * 1e3:.1f} ms per full step",
             "single_thread": {"value": int(wl.counts.sum()) / t1, "unit": "nodes/s", "cores": 1,
                               "sample": f"one step: attention on {n1} of {total} query rows (time scaled to all "
-                                        f"rows) plus the full acceptance walk; {t1 * 1e3:.1f} ms per full step"}}
+                                        f"rows) plus the full acceptance walk; {t1 * 1e3:.1f} ms per full step"},
+            "walk": walk}
 
 
 def run_reference(args, rank, world):
@@ -687,14 +840,14 @@ def run_reference(args, rank, world):
     wl, h = make_inputs(args.workload, seed=1)
     K, W = args.steps, args.warmup
     budget = 150.0
-    t_est, _, _ = oracle_step_times(wl, h, 1.0 / 64)
+    t_est, _, _, _ = oracle_step_times(wl, h, 1.0 / 64)
     frac = min(1.0, max(1.0 / 1024, budget / max(1, K + W) / max(t_est, 1e-9)))
     for _ in range(W):
         oracle_step_times(wl, h, frac)
     times = []
     n_rows = 0
     for _ in range(K):
-        t, n_rows, total = oracle_step_times(wl, h, frac)
+        t, n_rows, total, _ = oracle_step_times(wl, h, frac)
         times.append(t)
     per_step = sum(times) / K
     value = int(wl.counts.sum()) / per_step
@@ -719,6 +872,7 @@ def main():
     ap.add_argument("--workload", default="l8b", choices=("tiny", "l8b", "l70b", "mix", "long", "ragged"))
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-workload GPU figures")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

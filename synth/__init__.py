@@ -270,6 +270,7 @@ class Workload:
     row_keys: np.ndarray           # int64 [B][N]: generator row key of each node's p/q
     extra: dict = field(default_factory=dict)
     node_counts: np.ndarray | None = None  # int32 [B] nodes per sequence (ragged workloads)
+    tree_k_scale: float = 1.0      # keys of the tree block (positions L_b..L_b+n_b-1) are multiplied by this
 
     @property
     def max_blocks(self) -> int:
@@ -304,7 +305,18 @@ class Workload:
         return out
 
     def k_cache(self) -> np.ndarray:
-        return self._cache(STREAM_K)
+        k = self._cache(STREAM_K)
+        if self.tree_k_scale != 1.0:
+            # scale the tree block's keys in place; a power-of-two factor is exact in bf16 and fp32
+            bf = self.dtype == "bf16"
+            for b in range(self.batch):
+                L, n = int(self.prefix_lens[b]), int(self.counts[b])
+                for t in range(L, L + n):
+                    blk, slot = int(self.block_table[b, t // BLOCK_SIZE]), t % BLOCK_SIZE
+                    row = bf16_to_f32(k[blk, slot]) if bf else k[blk, slot]
+                    row = (row * np.float32(self.tree_k_scale)).astype(np.float32)
+                    k[blk, slot] = (row.view(np.uint32) >> 16).astype(np.uint16) if bf else row
+        return k
 
     def v_cache(self) -> np.ndarray:
         return self._cache(STREAM_V)
@@ -355,14 +367,26 @@ CONFIG_NAMES = ("tiny", "l8b", "l70b", "mix", "long")
 RAGGED_NAMES = ("ragged",)
 
 
-def make(name: str, seed: int | None = None, need_tokens: bool = True) -> Workload:
+UNIT_TREE_K_SCALE = 4.0
+
+
+def make(name: str, seed: int | None = None, need_tokens: bool = True, unit_kv: bool = False) -> Workload:
     """Build the tree, lengths and block table of a named workload.
 
     Heavy tensors (KV cache, p/q) are produced on demand by the Workload
     methods so callers only pay for what they use.  ``seed`` defaults to the
-    workload's index + 1."""
+    workload's index + 1.
+
+    ``unit_kv`` gives the same shapes, tree and block table with K and V drawn
+    from N(0, 1) instead of N(0, 1/128), and the tree block's keys multiplied
+    by ``UNIT_TREE_K_SCALE``: attention outputs are then of order one and each
+    row's ancestors carry a visible share of its softmax mass, so a wrong mask
+    word, split merge or row mapping changes the output far beyond bf16
+    rounding (with the default scales every output is an average of
+    thousands of small values and such mistakes stay below 1e-2)."""
     if name in RAGGED_NAMES:
-        return _make_ragged(name, 10 + RAGGED_NAMES.index(name) if seed is None else seed, need_tokens)
+        wl = _make_ragged(name, 10 + RAGGED_NAMES.index(name) if seed is None else seed, need_tokens)
+        return _unit(wl) if unit_kv else wl
     if name not in CONFIG_NAMES:
         raise ValueError(f"unknown workload {name!r}; choose from {CONFIG_NAMES + RAGGED_NAMES}")
     if seed is None:
@@ -432,6 +456,12 @@ def make(name: str, seed: int | None = None, need_tokens: bool = True) -> Worklo
                 for c in range(1, N):
                     toks[b, c] = categorical(q[b, parents[b, c]], float(u[b, c]))
         wl.tree_tokens = toks
+    return _unit(wl) if unit_kv else wl
+
+
+def _unit(wl: Workload) -> Workload:
+    wl.kv_std = 1.0
+    wl.tree_k_scale = UNIT_TREE_K_SCALE
     return wl
 
 

@@ -13,6 +13,43 @@ import tree_speculative_decoding_07_b200 as tv
 
 BF16_ATOL = 2e-2       # max-abs for bf16 storage (fp32 accumulation)
 F32_RTOL = 1e-5        # fp32 path: max-abs error <= 1e-5 * max |oracle| of the row
+# bf16 path, in addition to the max-abs bound: per (sequence, KV head) block,
+# ||gpu - oracle||_2 <= REL_RMS * ||oracle||_2.  The rounding in the kernel
+# (bf16 P and outputs, 2^-9 relative each) stays near 1e-3 of the block's
+# norm; an all-zero output, a dropped ancestor or a wrong split weight moves
+# the norm of the difference by a large fraction of the output's own norm,
+# however small the outputs are.
+REL_RMS = 1e-2
+
+
+def attention_errors(got: np.ndarray, ref: np.ndarray, block: np.ndarray, dtype: str) -> dict:
+    """Errors of attention rows got against the oracle's ref ([R][D] each);
+    block[r] numbers the (sequence, KV head) block of row r."""
+    got = got.astype(np.float64)
+    err = got - ref
+    out = {"finite": bool(np.isfinite(got).all())}
+    if not out["finite"]:
+        return out
+    out["max_abs"] = float(np.abs(err).max()) if err.size else 0.0
+    if dtype == "bf16":
+        blocks = np.unique(block, return_inverse=True)[1]
+        num = np.bincount(blocks, weights=(err ** 2).sum(axis=1))
+        den = np.bincount(blocks, weights=(ref ** 2).sum(axis=1))
+        out["rel_rms"] = float((np.sqrt(num) / np.maximum(np.sqrt(den), 1e-300)).max()) if num.size else 0.0
+    else:
+        scale = np.maximum(np.abs(ref).max(axis=1, keepdims=True), 1e-30)
+        out["row_rel"] = float((np.abs(err) / scale).max()) if err.size else 0.0
+    return out
+
+
+def attention_ok(e: dict, dtype: str) -> bool:
+    """The parity criterion: max-abs 2e-2 and relative rms 1e-2 per block for
+    bf16, row-relative 1e-5 for fp32."""
+    if not e["finite"]:
+        return False
+    if dtype == "bf16":
+        return e["max_abs"] <= BF16_ATOL and e["rel_rms"] <= REL_RMS
+    return e["row_rel"] <= F32_RTOL
 
 
 def dev(arr: np.ndarray, dtype: str | None = None) -> torch.Tensor:
@@ -58,29 +95,30 @@ class Attn:
         return oracle.tree_attention(self.q, self.k, self.v, self.block_table, self.prefix_lens, self.parent_idx,
                                      self.num_kv_heads, self.dtype, rows=rows)
 
-    def compare(self, gpu: np.ndarray, rows=None) -> float:
-        """Return the worst error against the oracle (absolute for bf16,
-        row-relative for fp32) and assert it is within tolerance."""
+    def row_blocks(self, rows=None) -> np.ndarray:
+        """(sequence, KV head) block number of every compared row."""
+        B, N, Hq = self.q.shape[:3]
+        G = Hq // self.num_kv_heads
+        if rows is not None:
+            rr = np.asarray(rows).reshape(-1, 3)
+            return rr[:, 0] * self.num_kv_heads + rr[:, 2] // G
+        b, _, h = np.meshgrid(np.arange(B), np.arange(N), np.arange(Hq), indexing="ij")
+        return (b * self.num_kv_heads + h // G).reshape(-1)
+
+    def compare(self, gpu: np.ndarray, rows=None) -> dict:
+        """Check the GPU output against the oracle (rows: sampled (b, i, h)
+        triples, else every row) and return the errors."""
         ref = self.oracle(rows)
         if rows is not None:
             rr = np.asarray(rows).reshape(-1, 3)
             got = gpu[rr[:, 0], rr[:, 1], rr[:, 2]]
         else:
             got = gpu.reshape(ref.shape)
-            ref = ref.reshape(-1, ref.shape[-1])
-            got = got.reshape(-1, got.shape[-1])
         ref = ref.reshape(-1, ref.shape[-1])
         got = got.reshape(-1, got.shape[-1])
-        assert np.isfinite(got).all(), "non-finite attention output"
-        err = np.abs(got.astype(np.float64) - ref)
-        if self.dtype == "bf16":
-            worst = float(err.max())
-            assert worst <= BF16_ATOL, f"max-abs {worst} > {BF16_ATOL}"
-        else:
-            scale = np.maximum(np.abs(ref).max(axis=1, keepdims=True), 1e-30)
-            worst = float((err / scale).max())
-            assert worst <= F32_RTOL, f"row-relative {worst} > {F32_RTOL}"
-        return worst
+        e = attention_errors(got, ref, self.row_blocks(rows), self.dtype)
+        assert attention_ok(e, self.dtype), f"attention parity failed: {e}"
+        return e
 
 
 def sample_rows(B, N, Hq, count, seed, must_nodes=()):
@@ -95,8 +133,10 @@ def sample_rows(B, N, Hq, count, seed, must_nodes=()):
     return np.array(rows, dtype=np.int32)
 
 
-def random_attn(seed, B, N, Hq, Hkv, D, prefix_lens, dtype="bf16", permute=True, parents=None, kv_std=None):
-    """Small seeded attention problem with random trees and a paged cache."""
+def random_attn(seed, B, N, Hq, Hkv, D, prefix_lens, dtype="bf16", permute=True, parents=None, kv_std=None,
+                tree_k_scale=1.0):
+    """Small seeded attention problem with random trees and a paged cache;
+    tree_k_scale multiplies the keys of the tree block (positions L_b..L_b+N-1)."""
     rng = np.random.default_rng(seed)
     prefix_lens = np.asarray(prefix_lens, np.int32)
     if parents is None:
@@ -115,6 +155,12 @@ def random_attn(seed, B, N, Hq, Hkv, D, prefix_lens, dtype="bf16", permute=True,
     q = synth.normals(B * N * Hq * D, seed, synth.STREAM_QUERY, bf16=bf).reshape(B, N, Hq, D)
     k = synth.normals(total * 16 * Hkv * D, seed, synth.STREAM_K, std=std, bf16=bf).reshape(total, 16, Hkv, D)
     v = synth.normals(total * 16 * Hkv * D, seed, synth.STREAM_V, std=std, bf16=bf).reshape(total, 16, Hkv, D)
+    if tree_k_scale != 1.0:
+        for b in range(B):
+            for t in range(int(prefix_lens[b]), int(prefix_lens[b]) + N):
+                blk, slot = bt[b, t // 16], t % 16
+                row = (synth.bf16_to_f32(k[blk, slot]) if bf else k[blk, slot]) * np.float32(tree_k_scale)
+                k[blk, slot] = (row.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16) if bf else row
     return Attn(q, k, v, bt, prefix_lens, parents, dtype, Hkv)
 
 

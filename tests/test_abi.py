@@ -111,7 +111,14 @@ def test_sampler_plan_covers_vocab():
         p = tv.tv_verify_sample_plan(tv.TvSampleDesc(1, 64, V))
         assert p.cluster_ctas * p.slice >= V and p.slice % 4 == 0
         assert 32 <= p.threads <= 512 and p.threads % 32 == 0
-        assert p.smem_bytes == 16 * p.slice
+        # two row buffers of p and q, then (when they fit) the gathered child values,
+        # 16 bytes per node; small vocabularies always leave room
+        assert p.smem_bytes in (16 * p.slice, 16 * p.slice + 16 * 64)
+        if V <= 1000:
+            assert p.smem_bytes == 16 * p.slice + 16 * 64
+    # the largest vocabulary leaves no room for the gathered values with 1024 nodes
+    big = tv.tv_verify_sample_plan(tv.TvSampleDesc(1, 1024, 16 * 13824))
+    assert big.smem_bytes == 16 * big.slice
     assert tv.tv_verify_sample_workspace_size(tv.TvSampleDesc(1, 64, 1000)) == 0
 
 

@@ -37,3 +37,18 @@ def test_deepest_paths_respect_node_counts():
     # sequence 1 keeps nodes 0, 1 <- 0, 2 <- 0: depth 1 at best, first deepest node 1
     assert plen.tolist() == [3, 1]
     assert path[0, :3].tolist() == [1, 2, 3] and path[1, :1].tolist() == [1]
+
+
+def test_rotation_copies_exceed_twice_l2():
+    l2 = 126 << 20
+    # the 8B shape reads ~20 MB per step: one pass over the copies must read >= 2 x L2
+    n = bench.rotation_copies(20 << 20, 90 << 20, l2)
+    assert n >= 4 and n * (20 << 20) >= 2 * l2
+    # a step that reads more than L2 by itself still rotates over 4 copies
+    assert bench.rotation_copies(4 << 30, 6 << 30, l2) == 4
+
+
+def test_tensor_flops_counts_every_key_of_every_row():
+    wl = synth.make("l8b", need_tokens=False)
+    # 4 * D * (L + N) * (G * N) per KV head
+    assert bench.tensor_flops(wl) == 4 * 128 * (4096 + 64) * (4 * 64) * 8

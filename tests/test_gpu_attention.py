@@ -24,24 +24,34 @@ def test_tiny_fp32_full_parity():
     print("tiny fp32 row-relative error", err)
 
 
-def test_l8b_full_parity():
-    a = Attn.from_workload(synth.make("l8b", need_tokens=False))
+@pytest.mark.parametrize("unit", [False, True], ids=["default_scale", "unit_kv"])
+def test_l8b_full_parity(unit):
+    """Every row of the Llama-3-8B shape (9 KV splits, 2 row tiles, both mask
+    words); unit_kv makes the outputs of order one (see synth.make)."""
+    a = Attn.from_workload(synth.make("l8b", need_tokens=False, unit_kv=unit))
     err = a.compare(a.run_gpu())
-    print("l8b max-abs error", err)
+    print("l8b", "unit" if unit else "default", err)
 
 
+def _must_nodes(N):
+    # the first and last node of every 32-bit word of the ancestor mask
+    return tuple(sorted({n for w in range((N + 31) // 32) for n in (32 * w, min(N, 32 * w + 32) - 1)}))
+
+
+@pytest.mark.parametrize("unit", [False, True], ids=["default_scale", "unit_kv"])
 @pytest.mark.parametrize("name,count", [("l70b", 384), ("mix", 384), ("long", 256)])
-def test_full_size_sampled_parity(name, count):
-    wl = synth.make(name, need_tokens=False)
+def test_full_size_sampled_parity(name, count, unit):
+    wl = synth.make(name, need_tokens=False, unit_kv=unit)
     a = Attn.from_workload(wl)
     out = a.run_gpu()
     assert np.isfinite(out).all()
     rows = sample_rows(wl.batch, wl.num_nodes, wl.num_q_heads, count, seed=7,
-                       must_nodes=(0, wl.num_nodes - 1) if wl.batch <= 8 else ())
+                       must_nodes=_must_nodes(wl.num_nodes) if wl.batch <= 8 else ())
     err = a.compare(out, rows)
-    print(name, "max-abs error on", len(rows), "rows", err)
+    print(name, "unit" if unit else "default", len(rows), "rows", err)
 
 
+@pytest.mark.parametrize("unit", [False, True], ids=["default_scale", "unit_kv"])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("B,N,Hq,Hkv,D,prefix", [
     (1, 1, 8, 8, 128, [0]),              # plain decode of the root only, empty prefix
@@ -51,15 +61,18 @@ def test_full_size_sampled_parity(name, count):
     (3, 7, 4, 4, 128, [17, 300, 4096]),  # MHA (G = 1), prefixes not multiples of 16
     (2, 16, 64, 8, 128, [2500, 3]),      # G = 8
 ])
-def test_edge_shapes(dtype, B, N, Hq, Hkv, D, prefix):
-    a = random_attn(11 + N, B, N, Hq, Hkv, D, prefix, dtype=dtype)
+def test_edge_shapes(dtype, B, N, Hq, Hkv, D, prefix, unit):
+    a = random_attn(11 + N, B, N, Hq, Hkv, D, prefix, dtype=dtype, kv_std=1.0 if unit else None,
+                    tree_k_scale=synth.UNIT_TREE_K_SCALE if unit else 1.0)
     a.compare(a.run_gpu())
 
 
-def test_chain_tree_matches_oracle():
+@pytest.mark.parametrize("unit", [False, True], ids=["default_scale", "unit_kv"])
+def test_chain_tree_matches_oracle(unit):
     N = 40
     parents = np.array([[-1] + list(range(N - 1))], np.int32)
-    a = random_attn(5, 1, N, 32, 8, 128, [2000], parents=parents)
+    a = random_attn(5, 1, N, 32, 8, 128, [2000], parents=parents, kv_std=1.0 if unit else None,
+                    tree_k_scale=synth.UNIT_TREE_K_SCALE if unit else 1.0)
     a.compare(a.run_gpu())
 
 

@@ -19,6 +19,9 @@ int device_sms() {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// shared memory a block may opt in to on sm_100 (227 KB)
+constexpr int SMEM_PER_BLOCK_OPTIN = 232448;
+
 tv_status check_attn_desc(const tv_attn_desc* d) {
     if (!d) return TV_ERR_INVALID_ARG;
     if (d->batch < 1 || d->num_nodes < 1 || d->num_q_heads < 1 || d->num_kv_heads < 1) return TV_ERR_INVALID_ARG;
@@ -99,9 +102,17 @@ void make_sample_plan(const tv_sample_desc* d, tv_sample_plan* p) {
     p->cluster_ctas = c;
     p->threads = threads;
     p->slice = slice;
-    p->smem_bytes = (int32_t)(4 * sizeof(float) * (size_t)slice);
+    // the two row buffers, then (when they fit) the gathered child values: p(x),
+    // q(x), the uniform and the first child of every node, 16 bytes per node
+    const size_t rows = 4 * sizeof(float) * (size_t)slice;
+    const size_t gathered = 16 * (size_t)d->num_nodes;
+    const bool gather = rows + gathered + tv::sample_static_smem() + 1024 <= (size_t)SMEM_PER_BLOCK_OPTIN;
+    p->smem_bytes = (int32_t)(rows + (gather ? gathered : 0));
     p->launches = 1;
 }
+
+// the walk gathers the child values into shared memory when the plan made room
+bool sample_gathers(const tv_sample_plan& p) { return (size_t)p.smem_bytes > 4 * sizeof(float) * (size_t)p.slice; }
 
 }  // namespace
 
@@ -124,6 +135,7 @@ tv_status verify_sample_common(const tv_sample_desc* desc, const float* p, const
     a.cluster = plan.cluster_ctas; a.threads = plan.threads; a.slice = plan.slice; a.smem_bytes = plan.smem_bytes;
     a.vec4 = (desc->vocab % 4 == 0) && !(reinterpret_cast<uintptr_t>(p) & 15) && !(reinterpret_cast<uintptr_t>(q) & 15);
     a.logits = logits ? 1 : 0;
+    a.gather = sample_gathers(plan) ? 1 : 0;
     int launches = 0;
     cudaError_t e = tv::launch_verify_sample(a, static_cast<cudaStream_t>(stream), &launches);
     return e == cudaSuccess ? TV_OK : TV_ERR_CUDA;

@@ -52,6 +52,7 @@ struct SampleArgs {
     int cluster, threads, slice, smem_bytes;
     int vec4;           // rows start 16-byte aligned and V % 4 == 0
     int logits;         // p and q hold the two models' logits: the walk applies the row softmax
+    int gather;         // every child's p(x), q(x) and uniform are gathered into shared memory first
 };
 
 cudaError_t launch_verify_sample(const SampleArgs& a, cudaStream_t st, int* launches);
@@ -72,6 +73,7 @@ struct CommitArgs {
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st);
 size_t commit_smem_bytes(int N, int row_bytes);
 int sample_max_cluster();
+size_t sample_static_smem();
 
 // Top-k branching: child tokens from each parent's draft distribution (one launch).
 struct FillArgs {

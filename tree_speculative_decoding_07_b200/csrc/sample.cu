@@ -26,6 +26,24 @@
 // same bits and take the same branches.  The bonus draw reuses the per-CTA
 // and per-warp partials of the last pass: the owning CTA, warp and lane are
 // located from them, and one lane scans its few elements.
+//
+// Children.  Every CTA first gathers, for every child c of the tree, the
+// draft token's entries p(x_c), q(x_c) of its parent's rows and its uniform
+// into shared memory (one round of independent loads), so no acceptance test
+// waits on a global load.  With those values the walk knows, on arriving at a
+// node, whether its first child passes the plain test u_c < p(x)/q(x); while
+// it does, the walk moves on without that node's row, and the row load is
+// started only for the node where the first test fails (its residual is
+// needed) or the leaf where the walk ends (its bonus draw).  The logits form
+// needs every visited row's softmax before any test, so it loads each
+// visited row.  When the vocabulary slice leaves no shared memory for the
+// gathered values, each node's children are gathered when the walk reaches it.
+//
+// Exit.  No CTA retires while a peer may still write to its shared memory:
+// every CTA arrives on every peer's exit barrier and waits (bounded) on its
+// own.  A CTA whose bounded wait ran out stops exchanging (no pushes, no
+// waits), so its peers time out once and stop too; the status word records
+// TV_ERR_TIMEOUT.
 #include <cooperative_groups.h>
 
 #include "tv_common.cuh"
@@ -57,6 +75,7 @@ struct SampleShared {
     float row_mp[2], row_mq[2];
     unsigned long long peer_bar[2];
     unsigned long long row_bar[2];
+    unsigned long long exit_bar;
     int timeout;
     int found;
     int wsel;
@@ -82,9 +101,11 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// bounded wait on one phase; false (and the timeout flag set) when it runs out
+// bounded wait on one phase; false (and the timeout flag set) when it runs out,
+// and false at once when an earlier wait of this CTA ran out
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* timeout) {
     if (mbar_try(bar, parity)) return true;
+    if (*timeout) return false;
     const long long t0 = clock64();
     for (;;) {
         if (mbar_try(bar, parity)) return true;
@@ -93,6 +114,21 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
             return false;
         }
     }
+}
+// arrive on the mbarrier at this shared::cluster address (any CTA of the cluster)
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
 }
 __device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
     uint32_t r;
@@ -138,58 +174,71 @@ __device__ __forceinline__ double resid(float p, float q, double c) {
 }
 
 struct Walker {
-    const SampleArgs& a;
     SampleShared& sh;
     float* buf;      // [2][2][slice]: buffer x holds p at buf + 2*x*slice, q right after
+    const float* p;
+    const float* q;
+    int V, N, slice;
     int b, rank, C, lo, n, tid, lane, warp, nwarps, segw;
     bool bulk;
-    int passes;      // cluster exchanges so far
-    int row_uses[2];
-    bool row_pending[2];
+    int passes;        // cluster exchanges so far
+    uint32_t pending;  // bit x: a copy into buffer x is in flight
+    uint32_t phase;    // bit x: parity of the next phase of buffer x's barrier
 
-    __device__ float* ps(int x) const { return buf + (size_t)2 * x * a.slice; }
-    __device__ float* qs(int x) const { return ps(x) + a.slice; }
+    __device__ float* ps(int x) const { return buf + (size_t)2 * x * slice; }
+    __device__ float* qs(int x) const { return ps(x) + slice; }
     __device__ uint32_t row_bar(int x) const { return smem_u32(&sh.row_bar[x]); }
 
-    // Wait until buffer x holds its row (collective).
+    // Wait until buffer x holds its row (collective).  Always waits (bounded), even
+    // after a timeout elsewhere: no copy may land in a buffer that is reused or in a
+    // CTA that has retired.
     __device__ void wait_row(int x) {
-        if (!row_pending[x]) return;
-        mbar_wait(row_bar(x), row_uses[x] & 1, &sh.timeout);
-        ++row_uses[x];
-        row_pending[x] = false;
+        if (!((pending >> x) & 1u)) return;
+        const uint32_t par = (phase >> x) & 1u;
+        if (!mbar_try(row_bar(x), par)) {
+            const long long t0 = clock64();
+            while (!mbar_try(row_bar(x), par)) {
+                if (clock64() - t0 > WAIT_LIMIT) {
+                    sh.timeout = 1;
+                    break;
+                }
+            }
+        }
+        phase ^= 1u << x;
+        pending &= ~(1u << x);
     }
 
     // Start loading this CTA's slice of node u's p and q rows into buffer x (collective).
     __device__ void issue_row(int x, int u) {
         wait_row(x);  // the buffer's previous copy must have landed before it is reused
-        const size_t base = ((size_t)b * a.N + u) * (size_t)a.V + lo;
+        const size_t base = ((size_t)b * N + u) * (size_t)V + lo;
         if (bulk) {
             if (tid == 0) {
                 mbar_expect_tx(row_bar(x), (uint32_t)(8 * n));
                 if (n > 0) {
-                    bulk_load(smem_u32(ps(x)), a.p + base, (uint32_t)(4 * n), row_bar(x));
-                    bulk_load(smem_u32(qs(x)), a.q + base, (uint32_t)(4 * n), row_bar(x));
+                    bulk_load(smem_u32(ps(x)), p + base, (uint32_t)(4 * n), row_bar(x));
+                    bulk_load(smem_u32(qs(x)), q + base, (uint32_t)(4 * n), row_bar(x));
                 }
             }
         } else {
             float* pd = ps(x);
             float* qd = qs(x);
             for (int i = tid; i < n; i += blockDim.x) {
-                pd[i] = __ldg(a.p + base + i);
-                qd[i] = __ldg(a.q + base + i);
+                pd[i] = __ldg(p + base + i);
+                qd[i] = __ldg(q + base + i);
             }
             __syncthreads();
             if (tid == 0) mbar_expect_tx(row_bar(x), 0);
         }
-        row_pending[x] = true;
+        pending |= 1u << x;
     }
 
     // Sum over the whole row of resid(p, q, c) from buffer x; every CTA returns
     // the same value.  Leaves this CTA's per-warp partials in sh.warp_part and
     // every CTA's partial in sh.peer[parity of the pass].
     __device__ double cluster_pass(int x, double c) {
-        const float* p = ps(x);
-        const float* q = qs(x);
+        const float* pr = ps(x);
+        const float* qr = qs(x);
         const int s0 = min(n, warp * segw), s1 = min(n, s0 + segw);
         double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
         // four consecutive elements per lane and step (16-byte shared loads; segw is a
@@ -198,7 +247,7 @@ struct Walker {
         int i = s0 + 4 * lane;
         if (c == 0.0) {
             for (; i + 3 < s1; i += 128) {
-                const float4 pv = *reinterpret_cast<const float4*>(p + i);
+                const float4 pv = *reinterpret_cast<const float4*>(pr + i);
                 a0 += (double)pv.x;
                 a1 += (double)pv.y;
                 a2 += (double)pv.z;
@@ -206,15 +255,15 @@ struct Walker {
             }
         } else {
             for (; i + 3 < s1; i += 128) {
-                const float4 pv = *reinterpret_cast<const float4*>(p + i);
-                const float4 qv = *reinterpret_cast<const float4*>(q + i);
+                const float4 pv = *reinterpret_cast<const float4*>(pr + i);
+                const float4 qv = *reinterpret_cast<const float4*>(qr + i);
                 a0 += pos_part(fma(-c, (double)qv.x, (double)pv.x));
                 a1 += pos_part(fma(-c, (double)qv.y, (double)pv.y));
                 a2 += pos_part(fma(-c, (double)qv.z, (double)pv.z));
                 a3 += pos_part(fma(-c, (double)qv.w, (double)pv.w));
             }
         }
-        for (int e = i; e < s1 && e < i + 4; ++e) a0 += resid(p[e], q[e], c);
+        for (int e = i; e < s1 && e < i + 4; ++e) a0 += resid(pr[e], qr[e], c);
         const double wsum = warp_sum_d((a0 + a1) + (a2 + a3));
         if (lane == 0) sh.warp_part[warp] = wsum;
         __syncthreads();
@@ -230,7 +279,8 @@ struct Walker {
     // st.async completing on the receiver's own mbarrier); every warp then combines
     // the C values with the same shuffle tree -- sums, or maxima when take_max -- so
     // all CTAs and all warps obtain the same bits and take the same branches.  The
-    // per-CTA values stay in sh.peer / sh.peer2 at the parity of the exchange.
+    // per-CTA values stay in sh.peer / sh.peer2 at the parity of the exchange.  Once a
+    // wait of this CTA has run out it neither sends nor waits any more.
     __device__ __forceinline__ void exchange(int nv, double v0, double v1, bool take_max, double& r0, double& r1) {
         const int par = passes & 1;
         const uint32_t use = (uint32_t)(passes >> 1);
@@ -241,7 +291,7 @@ struct Walker {
                     sh.peer[par][0] = v0;
                     sh.peer2[par][0] = v1;
                 }
-            } else {
+            } else if (!sh.timeout) {
                 const uint32_t bar = smem_u32(&sh.peer_bar[par]);
                 if (lane == 0) mbar_expect_tx(bar, (uint32_t)(8 * nv * C));
                 if (lane < C) {
@@ -331,7 +381,7 @@ struct Walker {
 };
 
 template <bool LOGITS>
-__global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a) {
+__global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(const __grid_constant__ SampleArgs a) {
     extern __shared__ float4 sample_dyn[];
     __shared__ SampleShared sh;
     const int C = a.cluster;
@@ -341,6 +391,14 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
     const int N = a.N;
     const int lo = min(a.V, rank * a.slice);
     const int n = min(a.V, lo + a.slice) - lo;
+    float* const rows = reinterpret_cast<float*>(sample_dyn);
+    // the gathered child values follow the two row buffers (a.gather): p(x_c) and
+    // q(x_c) of child c's token in its parent's rows (the raw logits in logits mode),
+    // c's uniform, and each node's first child (nn when it has none)
+    float* const g_p = rows + 4 * (size_t)a.slice;
+    float* const g_q = g_p + N;
+    float* const g_u = g_q + N;
+    int* const g_first = reinterpret_cast<int*>(g_u + N);
 
     if (tid == 0) {
         sh.timeout = 0;
@@ -348,6 +406,7 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
             mbar_init(smem_u32(&sh.row_bar[x]), 1);
             mbar_init(smem_u32(&sh.peer_bar[x]), 1);
         }
+        mbar_init(smem_u32(&sh.exit_bar), (uint32_t)C);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -356,8 +415,8 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
     // kernel has completed and its memory is visible
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    Walker w{a, sh, reinterpret_cast<float*>(sample_dyn), b, rank, C, lo, n, tid, lane, warp, nwarps,
-             ((n + nwarps - 1) / nwarps + 127) / 128 * 128, a.vec4 != 0, 0, {0, 0}, {false, false}};
+    Walker w{sh, rows, a.p, a.q, a.V, N, a.slice, b, rank, C, lo, n, tid, lane, warp, nwarps,
+             ((n + nwarps - 1) / nwarps + 127) / 128 * 128, a.vec4 != 0, 0, 0u, 0u};
     // the root's row is needed unless its first child is accepted: start it now
     w.issue_row(0, 0);
 
@@ -367,6 +426,7 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
     for (int i = tid; i < nn; i += blockDim.x) {
         sh.parent[i] = parent_at(a.parent, b, N, i);
         sh.token[i] = a.tokens[(size_t)b * N + i];
+        if (a.gather) g_first[i] = nn;
     }
     // every CTA's barriers must exist before a peer pushes to them (the first pass);
     // the cluster barrier sits here so the loads above are already in flight
@@ -392,207 +452,271 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(SampleArgs a
                 if (!empty) report(a.status, bad_count ? TV_ERR_INVALID_ARG : TV_ERR_TREE);
             }
         }
-        w.wait_row(0);
-        return;
-    }
-
-    // ---- walk from the root
-    int u = 0, len = 0, x = 0;
-    double cur_c = 0.0, cur_z = 1.0;
-    int last_pass_node = -1;
-    double last_pass_c = -1.0;
-    for (;;) {
-        cur_c = 0.0;
-        cur_z = 1.0;
-        int accepted = -1;
-        int scan = u + 1;
-        if (LOGITS) {
-            // even the first child's test needs the row's softmax normalisers
-            w.wait_row(x);
-            w.prep_row(x);
-        }
-        while (accepted < 0 && scan < nn) {
-            // warp 0 collects the next (up to 32) children of u in ascending order and
-            // gathers their draft tokens' p, q and acceptance draws
-            if (warp == 0) {
-                int found = 0, next = nn;
-                for (int c0 = scan; c0 < nn; c0 += 32) {
-                    const int c = c0 + lane;
-                    const bool kid = c < nn && sh.parent[c] == u;
-                    const unsigned m = __ballot_sync(0xffffffffu, kid);
-                    const int pos = found + __popc(m & ((1u << lane) - 1u));
-                    if (kid && pos < 32) sh.ch_node[pos] = c;
-                    if (found + __popc(m) > 32) {
-                        // resume after the last child taken from this chunk
-                        unsigned mm = m;
-                        for (int t = 0; t < 32 - found; ++t) mm &= mm - 1u;
-                        next = c0 + __ffs(mm) - 1;
-                        found = 32;
-                        break;
-                    }
-                    found += __popc(m);
-                }
-                __syncwarp();
-                if (lane < found) {
-                    const int c = sh.ch_node[lane];
-                    const size_t row = ((size_t)b * N + u) * (size_t)a.V;
-                    if (LOGITS) {
-                        const float ep = expf(__ldg(a.p + row + sh.token[c]) - sh.row_mp[x]);
-                        const float eq = expf(__ldg(a.q + row + sh.token[c]) - sh.row_mq[x]);
-                        sh.ch_p[lane] = (double)(float)((double)ep * sh.row_zp_inv[x]);
-                        sh.ch_q[lane] = (double)(float)((double)eq * sh.row_zq_inv[x]);
-                    } else {
-                        sh.ch_p[lane] = (double)__ldg(a.p + row + sh.token[c]);
-                        sh.ch_q[lane] = (double)__ldg(a.q + row + sh.token[c]);
-                    }
-                    sh.ch_u[lane] = (double)__ldg(a.uniforms + (size_t)b * N + c);
-                }
-                if (lane == 0) {
-                    sh.ch_n = found;
-                    sh.ch_next = next;
-                }
+    } else {
+        if (a.gather) {
+            // every child's draft-token entries and uniform, in one round of loads
+            for (int c = tid + 1; c < nn; c += blockDim.x) {
+                const int pu = sh.parent[c];
+                const size_t at = ((size_t)b * N + pu) * (size_t)a.V + sh.token[c];
+                g_p[c] = __ldg(a.p + at);
+                g_q[c] = __ldg(a.q + at);
+                g_u[c] = __ldg(a.uniforms + (size_t)b * N + c);
+                atomicMin(&g_first[pu], c);
             }
             __syncthreads();
-            const int gn = sh.ch_n;
-            for (int k = 0; k < gn; ++k) {
-                const double px = sh.ch_p[k], qx = sh.ch_q[k], r = sh.ch_u[k];
-                // r < num / (Z q(x)), compared without the fp64 division
-                const double num = cur_c == 0.0 ? px : pos_part(fma(-cur_c, qx, px));
-                const bool acc = qx > 0.0 ? (r * (cur_z * qx) < num) : (num > 0.0);
-                if (acc) {
-                    accepted = sh.ch_node[k];
+        }
+
+        // ---- walk from the root
+        int u = 0, len = 0, x = 0;
+        double cur_c = 0.0, cur_z = 1.0;
+        int last_pass_node = -1;
+        double last_pass_c = -1.0;
+        // From a node the walk has just reached (its distribution is still plain p),
+        // follow every first child that passes its plain test; returns the node where
+        // that stops, whose row the walk needs.  Every thread computes the same steps.
+        auto descend = [&](int v) {
+            if constexpr (!LOGITS) {
+                while (a.gather) {
+                    const int c = g_first[v];
+                    if (c >= nn) break;
+                    const double px = g_p[c], qx = g_q[c], r = g_u[c];
+                    if (!(qx > 0.0 ? (r * qx < px) : (px > 0.0))) break;
+                    if (rank == 0 && tid == 0) path_out[len] = c;
+                    ++len;
+                    v = c;
+                }
+            }
+            return v;
+        };
+        u = descend(0);
+        if (u != 0) {
+            // the root's row (buffer 0) was not needed; this node's is
+            x = 1;
+            w.issue_row(x, u);
+        }
+        for (;;) {
+            cur_c = 0.0;
+            cur_z = 1.0;
+            int accepted = -1;
+            int scan = u + 1;
+            if (LOGITS) {
+                // even the first child's test needs the row's softmax normalisers
+                w.wait_row(x);
+                w.prep_row(x);
+            }
+            while (accepted < 0 && scan < nn) {
+                // warp 0 collects the next (up to 32) children of u in ascending order with
+                // their draft tokens' p, q and acceptance draws
+                if (warp == 0) {
+                    int found = 0, next = nn;
+                    for (int c0 = scan; c0 < nn; c0 += 32) {
+                        const int c = c0 + lane;
+                        const bool kid = c < nn && sh.parent[c] == u;
+                        const unsigned m = __ballot_sync(0xffffffffu, kid);
+                        const int pos = found + __popc(m & ((1u << lane) - 1u));
+                        if (kid && pos < 32) sh.ch_node[pos] = c;
+                        if (found + __popc(m) > 32) {
+                            // resume after the last child taken from this chunk
+                            unsigned mm = m;
+                            for (int t = 0; t < 32 - found; ++t) mm &= mm - 1u;
+                            next = c0 + __ffs(mm) - 1;
+                            found = 32;
+                            break;
+                        }
+                        found += __popc(m);
+                    }
+                    __syncwarp();
+                    if (lane < found) {
+                        const int c = sh.ch_node[lane];
+                        const size_t at = ((size_t)b * N + u) * (size_t)a.V + sh.token[c];
+                        const float vp = a.gather ? g_p[c] : __ldg(a.p + at);
+                        const float vq = a.gather ? g_q[c] : __ldg(a.q + at);
+                        const float vu = a.gather ? g_u[c] : __ldg(a.uniforms + (size_t)b * N + c);
+                        if (LOGITS) {
+                            const float ep = expf(vp - sh.row_mp[x]);
+                            const float eq = expf(vq - sh.row_mq[x]);
+                            sh.ch_p[lane] = (double)(float)((double)ep * sh.row_zp_inv[x]);
+                            sh.ch_q[lane] = (double)(float)((double)eq * sh.row_zq_inv[x]);
+                        } else {
+                            sh.ch_p[lane] = (double)vp;
+                            sh.ch_q[lane] = (double)vq;
+                        }
+                        sh.ch_u[lane] = (double)vu;
+                    }
+                    if (lane == 0) {
+                        sh.ch_n = found;
+                        sh.ch_next = next;
+                    }
+                }
+                __syncthreads();
+                const int gn = sh.ch_n;
+                for (int k = 0; k < gn; ++k) {
+                    const double px = sh.ch_p[k], qx = sh.ch_q[k], r = sh.ch_u[k];
+                    // r < num / (Z q(x)), compared without the fp64 division
+                    const double num = cur_c == 0.0 ? px : pos_part(fma(-cur_c, qx, px));
+                    const bool acc = qx > 0.0 ? (r * (cur_z * qx) < num) : (num > 0.0);
+                    if (acc) {
+                        accepted = sh.ch_node[k];
+                        break;
+                    }
+                    w.wait_row(x);
+                    const double c_new = cur_c + cur_z;
+                    const double z_new = w.cluster_pass(x, c_new);
+                    last_pass_node = u;
+                    last_pass_c = c_new;
+                    if (z_new > 0.0) {
+                        cur_c = c_new;
+                        cur_z = z_new;
+                    }
+                }
+                scan = sh.ch_next;
+                __syncthreads();  // ch_* are rewritten by the next batch
+            }
+            if (accepted < 0) break;
+            if (rank == 0 && tid == 0) path_out[len] = accepted;
+            ++len;
+            u = descend(accepted);
+            x ^= 1;
+            w.issue_row(x, u);  // the row of the node where the walk goes on, into the other buffer
+        }
+
+        // ---- bonus token: first index whose running residual mass exceeds u0 * total
+        w.wait_row(x);
+        double total;
+        if (last_pass_node == u && last_pass_c == cur_c) {
+            total = cur_z;  // the last pass summed exactly this distribution; reuse its partials
+        } else {
+            total = w.cluster_pass(x, cur_c);
+        }
+        const int par = (w.passes - 1) & 1;
+        const double target = (double)__ldg(a.uniforms + (size_t)b * N) * total;
+        int owner = -1, last_pos_cta = -1;
+        double before = 0.0, run = 0.0;
+        for (int k = 0; k < C; ++k) {
+            const double pk = sh.peer[par][k];
+            if (pk > 0.0) last_pos_cta = k;
+            if (owner < 0) {
+                if (run + pk > target) {
+                    owner = k;
+                    before = run;
+                }
+                run += pk;
+            }
+        }
+        const bool fallback = owner < 0;
+        if (fallback) owner = last_pos_cta;
+
+        if (rank == owner) {
+            const float* pr = w.ps(x);
+            const float* qr = w.qs(x);
+            if (tid == 0) {
+                // first warp segment whose running sum crosses the target; the last one
+                // with mass if rounding leaves none
+                int wsel = -1, wlast = -1;
+                double rb = before, rr = before;
+                for (int k = 0; k < nwarps; ++k) {
+                    if (sh.warp_part[k] > 0.0) wlast = k;
+                    if (wsel < 0 && !fallback) {
+                        if (rr + sh.warp_part[k] > target) {
+                            wsel = k;
+                            rb = rr;
+                        }
+                        rr += sh.warp_part[k];
+                    }
+                }
+                sh.wsel = wsel >= 0 ? wsel : wlast;
+                sh.wbefore = wsel >= 0 ? rb : -INFINITY;  // -inf: take the segment's last positive element
+                sh.found = -1;
+            }
+            __syncthreads();
+            if (warp == sh.wsel) {
+                const int s0 = min(n, warp * w.segw), s1 = min(n, s0 + w.segw);
+                const int per = (s1 - s0 + 31) / 32;
+                const int e0 = min(s1, s0 + lane * per), e1 = min(s1, e0 + per);
+                double mine = 0.0;
+                int mylast = -1;
+                for (int i = e0; i < e1; ++i) {
+                    const double v = resid(pr[i], qr[i], cur_c);
+                    mine += v;
+                    if (v > 0.0) mylast = i;
+                }
+                double incl = mine;  // inclusive scan over the lanes
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const double t = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += t;
+                }
+                const bool take_last = sh.wbefore == -INFINITY;
+                const unsigned hit = take_last ? 0u : __ballot_sync(0xffffffffu, sh.wbefore + incl > target);
+                const unsigned pos = __ballot_sync(0xffffffffu, mylast >= 0);
+                int pick = -1;
+                if (hit) {
+                    const int hl = __ffs(hit) - 1;
+                    if (lane == hl) {
+                        double rsum = sh.wbefore + incl - mine;
+                        for (int i = e0; i < e1; ++i) {
+                            const double v = resid(pr[i], qr[i], cur_c);
+                            if (v > 0.0) pick = i;
+                            rsum += v;
+                            if (rsum > target && v > 0.0) break;
+                        }
+                    }
+                    pick = __shfl_sync(0xffffffffu, pick, hl);
+                } else if (pos) {
+                    // rounding left no crossing: the segment's last positive element
+                    const int ll = 31 - __clz(pos);
+                    pick = __shfl_sync(0xffffffffu, mylast, ll);
+                }
+                if (lane == 0) sh.found = pick;
+            }
+            __syncthreads();
+            if (tid == 0) {
+                a.bonus[b] = sh.found >= 0 ? lo + sh.found : -1;
+                a.len[b] = len;
+            }
+            for (int i = len + tid; i < N; i += blockDim.x) path_out[i] = -1;
+        } else if (owner < 0 && rank == 0) {
+            // no mass anywhere (an all-zero distribution)
+            if (tid == 0) {
+                a.bonus[b] = -1;
+                a.len[b] = len;
+            }
+            for (int i = len + tid; i < N; i += blockDim.x) path_out[i] = -1;
+        }
+    }
+
+    // ---- exit: no copy may still be landing in this CTA's shared memory, and no
+    // peer may still send to it, when it retires
+    w.wait_row(0);
+    w.wait_row(1);
+    if (C > 1) {
+        __syncthreads();
+        if (tid == 0) {
+            const uint32_t bar = smem_u32(&sh.exit_bar);
+            for (int k = 0; k < C; ++k) mbar_arrive_remote(mapa(bar, (uint32_t)k));
+            const long long t0 = clock64();
+            while (!mbar_try_cluster(bar, 0)) {
+                if (clock64() - t0 > WAIT_LIMIT) {
+                    sh.timeout = 1;
                     break;
                 }
-                w.wait_row(x);
-                const double c_new = cur_c + cur_z;
-                const double z_new = w.cluster_pass(x, c_new);
-                last_pass_node = u;
-                last_pass_c = c_new;
-                if (z_new > 0.0) {
-                    cur_c = c_new;
-                    cur_z = z_new;
+            }
+            if (sh.timeout) {
+                // exchanges were abandoned: give values a peer pushed before it stopped
+                // time to land before this CTA's shared memory is released
+                const long long t1 = clock64();
+                while (clock64() - t1 < (1ll << 20)) {
                 }
             }
-            scan = sh.ch_next;
-            __syncthreads();  // ch_* are rewritten by the next batch
-        }
-        if (accepted < 0) break;
-        if (rank == 0 && tid == 0) path_out[len] = accepted;
-        ++len;
-        u = accepted;
-        x ^= 1;
-        w.issue_row(x, u);  // prefetch the new node's row into the other buffer
-    }
-
-    // ---- bonus token: first index whose running residual mass exceeds u0 * total
-    w.wait_row(x);
-    double total;
-    if (last_pass_node == u && last_pass_c == cur_c) {
-        total = cur_z;  // the last pass summed exactly this distribution; reuse its partials
-    } else {
-        total = w.cluster_pass(x, cur_c);
-    }
-    const int par = (w.passes - 1) & 1;
-    const double target = (double)__ldg(a.uniforms + (size_t)b * N) * total;
-    int owner = -1, last_pos_cta = -1;
-    double before = 0.0, run = 0.0;
-    for (int k = 0; k < C; ++k) {
-        const double pk = sh.peer[par][k];
-        if (pk > 0.0) last_pos_cta = k;
-        if (owner < 0) {
-            if (run + pk > target) {
-                owner = k;
-                before = run;
-            }
-            run += pk;
-        }
-    }
-    const bool fallback = owner < 0;
-    if (fallback) owner = last_pos_cta;
-
-    if (rank == owner) {
-        const float* p = w.ps(x);
-        const float* q = w.qs(x);
-        if (tid == 0) {
-            // first warp segment whose running sum crosses the target; the last one
-            // with mass if rounding leaves none
-            int wsel = -1, wlast = -1;
-            double rb = before, rr = before;
-            for (int k = 0; k < nwarps; ++k) {
-                if (sh.warp_part[k] > 0.0) wlast = k;
-                if (wsel < 0 && !fallback) {
-                    if (rr + sh.warp_part[k] > target) {
-                        wsel = k;
-                        rb = rr;
-                    }
-                    rr += sh.warp_part[k];
-                }
-            }
-            sh.wsel = wsel >= 0 ? wsel : wlast;
-            sh.wbefore = wsel >= 0 ? rb : -INFINITY;  // -inf: take the segment's last positive element
-            sh.found = -1;
         }
         __syncthreads();
-        if (warp == sh.wsel) {
-            const int s0 = min(n, warp * w.segw), s1 = min(n, s0 + w.segw);
-            const int per = (s1 - s0 + 31) / 32;
-            const int e0 = min(s1, s0 + lane * per), e1 = min(s1, e0 + per);
-            double mine = 0.0;
-            int mylast = -1;
-            for (int i = e0; i < e1; ++i) {
-                const double v = resid(p[i], q[i], cur_c);
-                mine += v;
-                if (v > 0.0) mylast = i;
-            }
-            double incl = mine;  // inclusive scan over the lanes
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const double t = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += t;
-            }
-            const bool take_last = sh.wbefore == -INFINITY;
-            const unsigned hit = take_last ? 0u : __ballot_sync(0xffffffffu, sh.wbefore + incl > target);
-            const unsigned pos = __ballot_sync(0xffffffffu, mylast >= 0);
-            int pick = -1;
-            if (hit) {
-                const int hl = __ffs(hit) - 1;
-                if (lane == hl) {
-                    double rsum = sh.wbefore + incl - mine;
-                    for (int i = e0; i < e1; ++i) {
-                        const double v = resid(p[i], q[i], cur_c);
-                        if (v > 0.0) pick = i;
-                        rsum += v;
-                        if (rsum > target && v > 0.0) break;
-                    }
-                }
-                pick = __shfl_sync(0xffffffffu, pick, hl);
-            } else if (pos) {
-                // rounding left no crossing: the segment's last positive element
-                const int ll = 31 - __clz(pos);
-                pick = __shfl_sync(0xffffffffu, mylast, ll);
-            }
-            if (lane == 0) sh.found = pick;
-        }
-        __syncthreads();
-        if (tid == 0) {
-            a.bonus[b] = sh.found >= 0 ? lo + sh.found : -1;
-            a.len[b] = len;
-        }
-        for (int i = len + tid; i < N; i += blockDim.x) path_out[i] = -1;
-    } else if (owner < 0 && rank == 0) {
-        // no mass anywhere (an all-zero distribution)
-        if (tid == 0) {
-            a.bonus[b] = -1;
-            a.len[b] = len;
-        }
-        for (int i = len + tid; i < N; i += blockDim.x) path_out[i] = -1;
     }
-    // no copy may still be landing in this CTA's shared memory when it retires
-    w.wait_row(x ^ 1);
     if (tid == 0 && sh.timeout) report(a.status, TV_ERR_TIMEOUT);
 }
 
 }  // namespace
+
+size_t sample_static_smem() { return sizeof(SampleShared); }
 
 int sample_max_cluster() {
     static int best = -1;
