@@ -28,10 +28,11 @@
  *  tv_commit_path     after verification, the accepted path joins the cached
  *                     prefix (blog, "KV cache management and prefix sharing";
  *                     glossary, "KV cache management challenges").
- *  tv_tree_shape, tv_tree_fill_topk, tv_tree_select  building the tree that is
- *                     verified (glossary, tree-structure optimisation: top-k
- *                     branching and budget-constrained optimisation; LLM
- *                     Primer VI ch. 9, 9.2: EAGLE-2's dynamic tree).
+ *  tv_tree_shape, tv_tree_fill_topk, tv_tree_select(_device)  building the
+ *                     tree that is verified (glossary, tree-structure
+ *                     optimisation: top-k branching and budget-constrained
+ *                     optimisation; LLM Primer VI ch. 9, 9.2: EAGLE-2's
+ *                     dynamic tree).
  *
  * Ragged batches (trees of different sizes in one call) go through the
  * descriptors' node_counts; a NULL parent_idx means chains (linear
@@ -128,7 +129,8 @@ typedef struct {
 /* How a call will run (host-side query; launches nothing). */
 typedef struct {
     int32_t kernel;              /* 0 = tensor-core (tcgen05) bf16 path, 1 = CUDA-core path */
-    int32_t num_splits;          /* KV splits per (sequence, KV head, row tile) */
+    int32_t num_splits;          /* KV splits per (sequence, KV head, row tile); on the tensor-core
+                                    path the splits of a row tile form one thread-block cluster */
     int32_t row_tiles;           /* 128-row query tiles per (sequence, KV head) */
     int32_t grid_ctas;           /* CTAs in the main launch */
     int32_t launches;            /* kernel launches per call */
@@ -137,11 +139,11 @@ typedef struct {
 
 TV_API tv_status tv_tree_attention_plan(const tv_attn_desc *desc, tv_attn_plan *plan);
 
-/* Device workspace the call needs, in bytes (0 when none).  Ownership stays
- * with the caller; it must be 256-byte aligned, zero-filled before its first
- * use (e.g. one cudaMemset at allocation), and may be reused across calls
- * that are ordered on one stream: every call leaves its synchronisation
- * counters at zero again.  Calls that share a workspace must not overlap. */
+/* Device workspace the call needs, in bytes (0 when none: always so on the
+ * tensor-core path, whose KV splits merge inside a thread-block cluster).
+ * Ownership stays with the caller; it must be 256-byte aligned and may be
+ * reused across calls that are ordered on one stream (a call reads only what
+ * it wrote there itself).  Calls that share a workspace must not overlap. */
 TV_API size_t tv_tree_attention_workspace_size(const tv_attn_desc *desc);
 
 TV_API tv_status tv_tree_attention(const tv_attn_desc *desc, const void *q, const void *paged_k,
@@ -161,18 +163,21 @@ TV_API tv_status tv_tree_attention(const tv_attn_desc *desc, const void *q, cons
  * device), or work recorded into a CUDA graph.  The scratch memory comes from
  * a fixed device array of TV_STATIC_SCRATCH_BYTES inside the library, which
  * every GPU that loads the library holds until the process exits; nothing is
- * allocated or freed by this call.
+ * allocated or freed by this call.  Tensor-core calls (bf16, head_dim 128) need
+ * no scratch; CUDA-core calls with several KV splits need
+ * tv_tree_attention_workspace_size() bytes of it.
  *  - Returns TV_ERR_WORKSPACE, before launching anything, when the problem
- *    needs more scratch than TV_STATIC_SCRATCH_BYTES (see
- *    tv_tree_attention_workspace_size).
+ *    needs more scratch than TV_STATIC_SCRATCH_BYTES (fp32 or bf16 at
+ *    head_dim 128 on the CUDA cores with more than about 4,000 (KV split,
+ *    query row) pairs).
  *  - The first call on each device looks up the array's device address (with
  *    that device current); make that first call before any stream capture.
  *  - All calls share the one array per device, and it keeps the previous
- *    call's contents (the call clears the parts that must start at zero):
+ *    call's contents (every value a call reads it has written itself):
  *    calls that can overlap on the GPU, from any stream or thread, race on it
  *    and must be serialised by the caller.
  */
-#define TV_STATIC_SCRATCH_BYTES (12u << 20)
+#define TV_STATIC_SCRATCH_BYTES (2u << 20)
 
 TV_API tv_status tv_tree_attention_static(const tv_attn_desc *desc, const void *q, const void *paged_k,
                                           const void *paged_v, const int32_t *block_table,
@@ -455,6 +460,38 @@ TV_API tv_status tv_tree_select_batch(int32_t batch, const int32_t *cand_offsets
                                       const int32_t *cand_token, const double *cand_prob, int32_t budget,
                                       int32_t *parent_idx, int32_t *tree_tokens, int32_t *cand_index,
                                       int32_t *node_counts, double *expected_accepted);
+
+/*
+ * tv_tree_select_batch on the device: the same trees, bit for bit, from
+ * candidate arrays that already sit in GPU memory (where the draft model
+ * grew them), so the selection between drafting and verification needs no
+ * round trip to the host.  Section and selection rule as tv_tree_select.
+ *   cand_offsets  [batch + 1] int32: sequence b's candidates are entries
+ *                 cand_offsets[b] .. cand_offsets[b+1]-1 of the candidate
+ *                 arrays (at most max_candidates of them)
+ *   cand_parent, cand_token  int32, cand_prob float32 in [0, 1], as for
+ *                 tv_tree_select (parent indices local to the sequence)
+ * Outputs (device): parent_idx, tree_tokens, cand_index [batch][budget]
+ * int32 (-1 past the tree), node_counts [batch] int32, expected_accepted
+ * [batch] float64 (the sum of the taken scores, scores formed in fp64 from
+ * the fp32 probabilities).  One launch on `stream`, one CTA per sequence,
+ * dynamic shared memory of 16 bytes per candidate slot plus 4 per budget
+ * slot; no workspace.  Host-checked: batch >= 1, budget in [1, 1024],
+ * max_candidates in [0, TV_SELECT_MAX_CANDIDATES], non-null arrays
+ * (TV_ERR_INVALID_ARG / TV_ERR_UNSUPPORTED).  Device-checked, per sequence
+ * (its node count becomes -1, its rows -1, the code goes to *dev_status):
+ * candidates not topological (TV_ERR_TREE), a probability outside [0, 1] or
+ * decreasing offsets (TV_ERR_INVALID_ARG), more than max_candidates
+ * (TV_ERR_UNSUPPORTED).  Ranking is quadratic in the candidates of a sequence
+ * (about a microsecond per thousand candidates squared over 512 threads).
+ */
+#define TV_SELECT_MAX_CANDIDATES 8192
+
+TV_API tv_status tv_tree_select_device(int32_t batch, int32_t max_candidates, const int32_t *cand_offsets,
+                                       const int32_t *cand_parent, const int32_t *cand_token,
+                                       const float *cand_prob, int32_t budget, int32_t *parent_idx,
+                                       int32_t *tree_tokens, int32_t *cand_index, int32_t *node_counts,
+                                       double *expected_accepted, int32_t *dev_status, void *stream);
 
 /* Static string for a status code. */
 TV_API const char *tv_status_string(int32_t status);

@@ -73,6 +73,19 @@ def test_attention_rejects_null_pointers_and_small_workspace():
         assert tv.tv_tree_attention(d, 256, 256, 256, 256, 256, 256, 256, None, need, stream=0) == tv.TV_ERR_WORKSPACE
 
 
+def test_static_attention_refuses_oversize_scratch_on_the_host():
+    # fp32, head_dim 128: 96 query rows x 49 KV splits of partials need more than the fixed array
+    d = _desc(batch=1, num_nodes=32, num_q_heads=3, num_kv_heads=1, head_dim=128, max_blocks_per_seq=800,
+              num_blocks=800, dtype=tv.TV_F32)
+    assert tv.tv_tree_attention_plan(d).workspace_bytes > tv.TV_STATIC_SCRATCH_BYTES
+    a = 256
+    assert tv.tv_tree_attention_static(d, a, a, a, a, a, a, a, None, stream=0) == tv.TV_ERR_WORKSPACE
+    # the tensor-core path (bf16, head_dim 128) needs no scratch at all
+    d = _desc(num_nodes=64, num_q_heads=32, num_kv_heads=8, head_dim=128, max_blocks_per_seq=260,
+              num_blocks=260, dtype=tv.TV_BF16)
+    assert tv.tv_tree_attention_plan(d).workspace_bytes == 0
+
+
 def test_attention_plans():
     # bf16 head_dim 128 runs on the tensor-core kernel, fp32 on the CUDA-core kernel
     d = _desc(num_nodes=64, num_q_heads=32, num_kv_heads=8, head_dim=128, max_blocks_per_seq=260,

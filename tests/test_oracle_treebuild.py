@@ -240,3 +240,23 @@ def test_tree_versus_chain_matches_the_pages():
     for n in (16, 32, 64):
         parent, _, _ = oracle.tree_shape_dp([0.95, 0.03, 0.01], n)
         assert parent.tolist() == [-1] + list(range(n - 1))
+
+
+def test_selection_is_the_first_candidates_of_the_score_order():
+    """With probabilities in [0, 1] every parent precedes its children in the
+    (score descending, index ascending) order, so the selected set is exactly
+    the first budget - 1 candidates of that order (the property the GPU
+    selection relies on), here checked on the oracle's own output."""
+    rng = np.random.default_rng(31)
+    for trial in range(40):
+        M = int(rng.integers(0, 300))
+        par = np.array([int(rng.integers(-1, c)) if c else -1 for c in range(M)], np.int32)
+        prob = (rng.integers(0, 5, M) / 4.0) if trial % 2 else rng.random(M) ** 2
+        tok = np.arange(M, dtype=np.int32)
+        budget = int(rng.integers(1, 80))
+        _, _, index, _ = oracle.select_tree(par, tok, prob, budget)
+        score = np.zeros(M)
+        for c in range(M):
+            score[c] = (score[par[c]] if par[c] >= 0 else 1.0) * prob[c]
+        order = sorted(range(M), key=lambda c: (-score[c], c))
+        assert list(index[1:]) == order[: budget - 1]

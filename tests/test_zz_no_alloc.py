@@ -52,3 +52,22 @@ def test_static_scratch_matches_workspace_path():
         for a, desc, plan, ref in cases:
             out = _static(a, desc, status)
             assert torch.equal(out, ref), (plan.kernel, plan.num_splits)
+
+
+def test_static_scratch_refuses_oversize_problems():
+    """A CUDA-core problem whose split merge needs more than the fixed array
+    (fp32, head_dim 128, 96 query rows x 49 KV splits) is refused before any
+    launch, and the refusal leaves the next call working."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    d = tv.TvAttnDesc(batch=1, num_nodes=32, num_q_heads=3, num_kv_heads=1, head_dim=128, block_size=16,
+                      max_blocks_per_seq=800, num_blocks=800, dtype=tv.TV_F32, softmax_scale=0.0)
+    plan = tv.tv_tree_attention_plan(d)
+    assert plan.workspace_bytes > tv.TV_STATIC_SCRATCH_BYTES
+    buf = torch.zeros(1 << 20, dtype=torch.float32, device="cuda")
+    p = buf.data_ptr()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    assert tv.tv_tree_attention_static(d, p, p, p, p, p, p, p, status) == tv.TV_ERR_WORKSPACE
+    a = random_attn(73, 1, 16, 8, 2, 128, [3000], dtype="f32")
+    a, desc, plan, ref = _case(a)
+    assert torch.equal(_static(a, desc, status), ref)

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libtreeverify.so")
 TV_OK, TV_ERR_INVALID_ARG, TV_ERR_UNSUPPORTED, TV_ERR_TREE = 0, 1, 2, 3
 TV_ERR_BLOCK_TABLE, TV_ERR_WORKSPACE, TV_ERR_CUDA, TV_ERR_TIMEOUT = 4, 5, 6, 7
 TV_BF16, TV_F32 = 0, 1
-TV_STATIC_SCRATCH_BYTES = 12 << 20
+TV_STATIC_SCRATCH_BYTES = 2 << 20
 
 
 class TvAttnDesc(ctypes.Structure):
@@ -83,12 +83,14 @@ def lib() -> ctypes.CDLL:
         L.tv_tree_shape_for_cost.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_double,
                                              ctypes.c_double, P, P, P, P, P]
         L.tv_tree_select_batch.argtypes = [ctypes.c_int32, P, P, P, P, ctypes.c_int32, P, P, P, P, P]
+        L.tv_tree_select_device.argtypes = [ctypes.c_int32, ctypes.c_int32, P, P, P, P, ctypes.c_int32, P, P, P, P,
+                                            P, P, P]
         L.tv_status_string.argtypes = [ctypes.c_int32]
         L.tv_status_string.restype = ctypes.c_char_p
         L.tv_version.restype = ctypes.c_int32
         for name in ("tv_tree_attention_plan", "tv_tree_attention", "tv_tree_attention_static",
                      "tv_verify_sample_plan", "tv_verify_sample", "tv_commit_path", "tv_verify_sample_logits",
-                     "tv_tree_fill_topk", "tv_tree_shape", "tv_tree_select", "tv_tree_select_batch",
+                     "tv_tree_fill_topk", "tv_tree_shape", "tv_tree_select", "tv_tree_select_batch", "tv_tree_select_device",
                      "tv_tree_shape_for_cost", "tv_tree_merge"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -277,6 +279,39 @@ def tree_select_batch(cand_offsets, cand_parent, cand_token, cand_prob, budget: 
                                        _hptr(parent), _hptr(tokens), _hptr(index), _hptr(counts), _hptr(val)))
     if s != TV_OK:
         raise TreeVerifyError(s, "tv_tree_select_batch")
+    return parent, tokens, index, counts, val
+
+
+def tv_tree_select_device(batch: int, max_candidates: int, cand_offsets, cand_parent, cand_token, cand_prob,
+                          budget: int, parent_idx, tree_tokens, cand_index, node_counts, expected_accepted,
+                          dev_status=None, stream=None) -> int:
+    """Device pointers (torch tensors or addresses)."""
+    return int(lib().tv_tree_select_device(int(batch), int(max_candidates), _ptr(cand_offsets), _ptr(cand_parent),
+                                           _ptr(cand_token), _ptr(cand_prob), int(budget), _ptr(parent_idx),
+                                           _ptr(tree_tokens), _ptr(cand_index), _ptr(node_counts),
+                                           _ptr(expected_accepted), _ptr(dev_status), _stream(stream)))
+
+
+def tree_select_device(cand_offsets, cand_parent, cand_token, cand_prob, budget: int, max_candidates=None,
+                       dev_status=None, stream=None):
+    """tv_tree_select_device on CUDA tensors (offsets [B+1] int32, candidates
+    int32 / float32); returns (parent_idx, tree_tokens, cand_index) as
+    [B][budget] int32 tensors, node_counts [B] and expected_accepted [B]
+    (float64), all on the device."""
+    import torch
+    B = cand_offsets.numel() - 1
+    if max_candidates is None:
+        max_candidates = int((cand_offsets[1:] - cand_offsets[:-1]).max().item()) if B > 0 else 0
+    dev = cand_offsets.device
+    parent = torch.empty((B, int(budget)), dtype=torch.int32, device=dev)
+    tokens = torch.empty_like(parent)
+    index = torch.empty_like(parent)
+    counts = torch.empty((B,), dtype=torch.int32, device=dev)
+    val = torch.empty((B,), dtype=torch.float64, device=dev)
+    s = tv_tree_select_device(B, max_candidates, cand_offsets, cand_parent, cand_token, cand_prob, budget, parent,
+                              tokens, index, counts, val, dev_status, stream)
+    if s != TV_OK:
+        raise TreeVerifyError(s, "tv_tree_select_device")
     return parent, tokens, index, counts, val
 
 

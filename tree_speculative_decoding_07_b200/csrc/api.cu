@@ -38,13 +38,12 @@ tv_status check_attn_desc(const tv_attn_desc* d) {
 
 // Which kernel runs and how the KV range is split.
 //  - bf16 with head_dim 128 runs on the tensor cores: 128-row query tiles;
-//    with several KV splits the launch is cooperative and the splits of a
-//    tile merge their partial results through the workspace.
+//    the KV splits of a tile form one thread-block cluster and merge their
+//    partial results through each other's shared memory (no workspace).
 //  - everything else runs on the CUDA cores: 32-row tiles, splits merged by
 //    a second kernel through a global workspace.
-// Splits are chosen so the main launch covers the SMs about once (for the
-// tensor-core path: as many as keep the whole grid resident), and never below
-// 256 tokens per split.
+// Splits are chosen so the main launch covers the SMs about once, and never
+// below 256 tokens per split.
 void make_plan(const tv_attn_desc* d, tv_attn_plan* p) {
     const int G = d->num_q_heads / d->num_kv_heads;
     const int rows = G * d->num_nodes;
@@ -57,7 +56,7 @@ void make_plan(const tv_attn_desc* d, tv_attn_plan* p) {
     const int64_t base = (int64_t)d->batch * d->num_kv_heads * p->row_tiles;
     int64_t splits;
     if (tc) {
-        splits = tv::tc_pick_splits(base, max_tokens, sms);
+        splits = tv::tc_pick_splits(base, d->max_blocks_per_seq, sms);
     } else {
         splits = base >= sms ? 1 : (sms / base);
         const int64_t by_len = (max_tokens + 255) / 256;
@@ -69,7 +68,6 @@ void make_plan(const tv_attn_desc* d, tv_attn_plan* p) {
     p->grid_ctas = (int32_t)(base * splits);
     p->launches = (!tc && splits > 1) ? 2 : 1;
     size_t ws = 0;
-    if (tc) ws = tv::tc_workspace_bytes(base, (int)splits);
     if (!tc && splits > 1) {
         const size_t rows_all = (size_t)d->batch * d->num_nodes * d->num_q_heads;
         ws = align256(sizeof(float) * splits * rows_all * d->head_dim) + align256(sizeof(float) * splits * rows_all);
@@ -203,12 +201,8 @@ tv_status tv_tree_attention(const tv_attn_desc* desc, const void* q, const void*
     a.num_blocks = desc->num_blocks; a.splits = plan.num_splits; a.row_tiles = plan.row_tiles;
     const float scale = desc->softmax_scale > 0.f ? desc->softmax_scale : 1.0f / sqrtf((float)desc->head_dim);
     a.scale_log2 = scale * 1.4426950408889634f;
-    if (plan.workspace_bytes && plan.kernel == 0) {
-        const int64_t groups = (int64_t)a.B * a.Hkv * a.row_tiles;
-        a.o_part = static_cast<float*>(workspace);
-        a.counters = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) +
-                                                 tv::tc_counter_offset(groups, a.splits));
-    } else if (plan.workspace_bytes) {
+    a.blocks_per_split = (desc->max_blocks_per_seq + a.splits - 1) / a.splits;
+    if (plan.workspace_bytes) {
         const size_t rows_all = (size_t)a.B * a.N * a.Hq;
         a.o_part = static_cast<float*>(workspace);
         a.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
@@ -361,6 +355,23 @@ tv_status tv_tree_select_batch(int32_t batch, const int32_t* cand_offsets, const
         node_counts[b] = n;
     }
     return TV_OK;
+}
+
+tv_status tv_tree_select_device(int32_t batch, int32_t max_candidates, const int32_t* cand_offsets,
+                                const int32_t* cand_parent, const int32_t* cand_token, const float* cand_prob,
+                                int32_t budget, int32_t* parent_idx, int32_t* tree_tokens, int32_t* cand_index,
+                                int32_t* node_counts, double* expected_accepted, int32_t* dev_status, void* stream) {
+    if (batch < 1 || max_candidates < 0 || budget < 1) return TV_ERR_INVALID_ARG;
+    if (!cand_offsets || !parent_idx || !tree_tokens || !cand_index || !node_counts || !expected_accepted)
+        return TV_ERR_INVALID_ARG;
+    if (max_candidates > 0 && (!cand_parent || !cand_token || !cand_prob)) return TV_ERR_INVALID_ARG;
+    if (budget > 1024 || max_candidates > TV_SELECT_MAX_CANDIDATES) return TV_ERR_UNSUPPORTED;
+    tv::SelectArgs a = {};
+    a.offsets = cand_offsets; a.cand_parent = cand_parent; a.cand_token = cand_token; a.cand_prob = cand_prob;
+    a.parent_idx = parent_idx; a.tree_tokens = tree_tokens; a.cand_index = cand_index; a.node_counts = node_counts;
+    a.expected = expected_accepted; a.status = dev_status;
+    a.B = batch; a.budget = budget; a.max_cand = max_candidates;
+    return tv::launch_select(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? TV_OK : TV_ERR_CUDA;
 }
 
 tv_status tv_verify_sample(const tv_sample_desc* desc, const float* p, const float* q, const int32_t* tree_tokens,

@@ -7,13 +7,14 @@
 // Decomposition.  The G query heads that share a KV head, times the N tree
 // nodes, form the query rows of one (sequence, KV head): row r is node r / G,
 // head r % G, so each K/V row is read once for all G heads.  A CTA owns one
-// 128-row tile of those rows and one KV split.  With several splits the grid
-// is launched cooperatively (all CTAs resident at once, one per SM); the
-// splits of a tile write their partial results to an L2-resident workspace,
-// count themselves in on a per-tile arrival counter, and once all S have
-// arrived each combines an equal share of the rows (flash-decoding
-// log-sum-exp merge).  The last split to leave resets the counters, so the
-// workspace is ready for the next call.
+// 128-row tile of those rows and one KV split: a fixed range of logical
+// blocks of the block table (known at launch, so the block ids are fetched
+// before the sequence's length arrives).  The S splits of a row tile form one
+// thread-block cluster; when all have finished their tokens, each pushes its
+// normalised partial rows (bf16) and their log-sum-exp into the shared memory
+// of the CTA that owns each row (an equal share per CTA, st.async completing on
+// the owner's mbarrier), and each owner combines its rows from the S partials
+// (flash-decoding log-sum-exp merge).  No global workspace is used.
 //
 // Warp roles (384 threads):
 //   warp 0      TMA producer of K tiles, warp 3 of V tiles: the rows of 8 paged
@@ -40,10 +41,12 @@
 // tree mask is a 128-bit ancestor set per node (anc(i) = anc(parent(i)) |
 // {i}), shifted into column space once per tile; prefix-only tiles skip it.
 //
-// Every wait (mbarrier phase or arrival counter) is bounded (about two
-// seconds of clock); on expiry the CTA records TV_ERR_TIMEOUT, stops issuing
-// work, writes NaN rows, frees its TMEM and still counts itself in and out
-// so no peer is left waiting and the counters return to zero.
+// Every wait (mbarrier phase) is bounded (about two seconds of clock); on
+// expiry the CTA records TV_ERR_TIMEOUT, stops issuing work, drains its copies
+// and MMAs, frees its TMEM, and still takes part in the merge with NaN rows so
+// no peer is left waiting.
+#include <mutex>
+
 #include "tc_device.cuh"
 
 namespace tv {
@@ -72,15 +75,20 @@ constexpr int BAR_PV_DONE = BAR_O_DONE + 2;      // 2: P V of the tile in an S b
 constexpr int BAR_Q_READY = BAR_PV_DONE + 2;     // Q staged
 constexpr int BAR_DRAIN_QK = BAR_Q_READY + 1;    // all S = Q K^T MMAs done
 constexpr int BAR_DRAIN_PV = BAR_DRAIN_QK + 1;   // all P V MMAs done
-constexpr int BAR_COUNT = BAR_DRAIN_PV + 1;
-static_assert(BAR_COUNT == 2 * KST + 2 * VST + 11, "barrier slots overlap");
+constexpr int BAR_FREE = BAR_DRAIN_PV + 1;       // S arrivals: every CTA of the cluster can receive partials
+constexpr int BAR_MERGE = BAR_FREE + 1;          // this CTA's share of partial rows received (transaction count)
+constexpr int BAR_COUNT = BAR_MERGE + 1;
+static_assert(BAR_COUNT == 2 * KST + 2 * VST + 13, "barrier slots overlap");
+// bytes pushed per (partial row, split): 128 bf16 outputs and the fp32 log-sum-exp
+constexpr uint32_t PUSH_BYTES = 2 * HD + 4;
 
 __global__ void __launch_bounds__(TC_THREADS, 1)
-    attn_tc_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+    attn_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tmk,
+                   const __grid_constant__ CUtensorMap tmv) {
     extern __shared__ uint8_t dsmem[];
     __shared__ __align__(8) uint64_t bars[BAR_COUNT];
     __shared__ uint32_t s_tmem;
-    __shared__ int s_abort, s_bad;
+    __shared__ int s_abort, s_bad, s_got;
     __shared__ int32_t s_par[TV_MAX_NODES_ATTN];
     __shared__ __align__(16) int32_t s_ids[2][ID_RING * BLK_PER_TILE];  // block ids, per producer
 
@@ -88,13 +96,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int split = blockIdx.x, tile = blockIdx.y;
     const int b = blockIdx.z / a.Hkv, kvh = blockIdx.z % a.Hkv;
     const int N = a.N, G = a.G, S = a.splits;
-    // the prefix length and the sequence's node count decide everything below:
+    // the prefix length and the sequence's node count decide where the tokens end:
     // both loads are issued before any set-up
     const int L = a.prefix_lens[b];
     bool bad_count;
     const int n = seq_nodes(a.counts, b, N, bad_count);
-    // row tiles past a short tree have no rows; every split of such a tile leaves
-    // here, so no merge waits on it
+    // row tiles past a short tree have no rows; every split of such a tile (the
+    // whole cluster) leaves here, so no merge waits on it
     if (!bad_count && tile * TM >= G * n) return;
     const uint32_t raw = smem_u32(dsmem);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -113,9 +121,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     auto pv_done = [&](int sb) { return bar0 + 8u * (BAR_PV_DONE + sb); };
     const uint32_t q_ready = bar0 + 8u * BAR_Q_READY;
     const uint32_t drain_qk = bar0 + 8u * BAR_DRAIN_QK, drain_pv = bar0 + 8u * BAR_DRAIN_PV;
+    const uint32_t free_bar = bar0 + 8u * BAR_FREE, merge_bar = bar0 + 8u * BAR_MERGE;
     volatile int* abort_flag = &s_abort;
     // results of the softmax groups, consumed by the split merge after the role blocks
-    float o[64];
+    uint32_t pk[32];   // this thread's 64 outputs of its row, as bf16 pairs
     float lse = -INFINITY;
     const int X = warp >= 4 ? (warp - 4) >> 2 : 0;          // softmax group: tokens X*64 .. X*64+63 of a tile
     const int r = ((warp & 3) << 5) + lane;                  // query row in the tile (softmax warps)
@@ -142,6 +151,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         mbar_init(q_ready, 256);
         mbar_init(drain_qk, 1);
         mbar_init(drain_pv, 1);
+        mbar_init(free_bar, (uint32_t)S);
+        mbar_init(merge_bar, 1);
         fence_barrier_init();
     }
     if (warp == 2) {
@@ -151,27 +162,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
         tc_fence_before();
     }
-    // the prefix length decides the split range and so the first block ids; the
-    // tree's parent array is read only after the id copies are issued
-    const int total = L + n;
-    const bool bad_len = L < 0 || (total + TV_BLOCK - 1) / TV_BLOCK > a.max_blocks;
-    int t0, t1;
-    split_range(bad_len ? 0 : total, S, split, t0, t1);
-    const int ntiles = (t1 - t0 + TN - 1) / TN;
-    const int last_blk = (t1 - 1) / TV_BLOCK;
-    // Block ids reach the producers through a shared-memory ring that cp.async
-    // fills ID_AHEAD tiles ahead of use, so no tile's copies wait on a
-    // block-table load (a register loaded one tile earlier would stall every
-    // iteration for one global-memory latency).  The first copies start before
-    // the barrier, overlapping barrier set-up and TMEM allocation.
+    // This split's logical blocks are [blk0, blk_end) of the block table, fixed at
+    // launch, so their ids are fetched without waiting for the prefix length.
+    // They reach the producers through a shared-memory ring that cp.async fills
+    // ID_AHEAD tiles ahead of use, so no tile's copies wait on a block-table load
+    // (a register loaded one tile earlier would stall every iteration for one
+    // global-memory latency).  The first copies start before the barrier,
+    // overlapping barrier set-up and TMEM allocation.
+    const int blk0 = min(a.max_blocks, split * a.blocks_per_split);
+    const int blk_end = min(a.max_blocks, blk0 + a.blocks_per_split);
     const int32_t* bt = a.block_table + (size_t)b * a.max_blocks;
     const int prod = warp == 0 ? 0 : 1;
     auto prefetch_ids = [&](int jt) {
-        if (jt < ntiles && lane < BLK_PER_TILE) {
-            int bi = (t0 + jt * TN) / TV_BLOCK + lane;
-            if (bi > last_blk) bi = last_blk;
+        const int bi = blk0 + jt * BLK_PER_TILE + lane;
+        if (lane < BLK_PER_TILE && bi < blk_end)
             cp_async_4(smem_u32(&s_ids[prod][(jt % ID_RING) * BLK_PER_TILE + lane]), bt + bi);
-        }
         cp_async_commit();  // one group per tile on every lane, empty or not
     };
     if (warp == 0 || warp == 3)
@@ -181,8 +186,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // a kernel launched after this one with programmatic stream serialisation may
     // start its set-up now; it waits for this grid before reading anything
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // the CTAs of the cluster have initialised their barriers (the merge's remote
+    // operations wait for this arrival of every CTA)
+    if (S > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     tc_fence_after();
     const uint32_t tmem = s_tmem;
+    // the split's tokens: [t0, t1) of the sequence's L + n
+    const int total = L + n;
+    const bool bad_len = L < 0 || (total + TV_BLOCK - 1) / TV_BLOCK > a.max_blocks;
+    const int t0 = blk0 * TV_BLOCK;
+    const int t1 = max(t0, min(blk_end * TV_BLOCK, bad_len ? 0 : total));
+    const int ntiles = (t1 - t0 + TN - 1) / TN;
+    const int used_blk = (t1 + TV_BLOCK - 1) / TV_BLOCK;  // blocks holding this split's tokens end here
 
     if (warp == 0 || warp == 3) {
         // ---------------- TMA producers: warp 0 streams K tiles, warp 3 V tiles
@@ -199,11 +214,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             cp_async_wait<ID_AHEAD - 1>();
             __syncwarp();
             if (lane == 0) {
+                // blocks of the tile that hold tokens of the split (the last tile may
+                // hold fewer than 8); rows of the others are masked and never loaded
+                const int nb = min(BLK_PER_TILE, used_blk - (blk0 + j * BLK_PER_TILE));
                 int cur[BLK_PER_TILE];
                 const int32_t* ring = &s_ids[prod][(j % ID_RING) * BLK_PER_TILE];
 #pragma unroll
                 for (int k = 0; k < BLK_PER_TILE; ++k) {
-                    int id = ring[k];
+                    int id = k < nb ? ring[k] : 0;
                     if (id < 0 || id >= a.num_blocks) {
                         bad_id = true;
                         id = 0;
@@ -212,12 +230,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 }
                 const uint32_t full = is_k ? k_full(s) : v_full(s);
                 const uint32_t dst = is_k ? sK(s) : sV(s);
-                mbar_expect_tx(full, TILE_BYTES);
+                mbar_expect_tx(full, (uint32_t)nb * (TILE_BYTES / BLK_PER_TILE));
 #pragma unroll
                 for (int k = 0; k < BLK_PER_TILE; ++k)
+                    if (k < nb)
 #pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        tma_load_4d(dst + h * HALF_BYTES + k * 2048u, map, full, 0, kvh * 2 + h, 0, cur[k]);
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_4d(dst + h * HALF_BYTES + k * 2048u, map, full, 0, kvh * 2 + h, 0, cur[k]);
             }
             __syncwarp();
             // the slot refilled here last held tile j + ID_AHEAD - ID_RING, read before
@@ -247,6 +266,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (ntiles > 0 && lane == 0) {
             bool ok = mbar_wait(q_ready, 0, abort_flag);
             bool issued_any = false;
+            // descriptors of the tiles' first 16-column step; the other steps add a
+            // constant to the address field (addresses stay below 2^18 bytes)
+            const uint64_t dq = sdesc(sQ, 16, 1024);
+            const uint64_t dk0 = sdesc(sK(0), 16, 1024);
             for (int j = 0; ok && j < ntiles; ++j) {
                 const int ks = j % KST, sb = j & 1;
                 // S buffer j % 2 holds P of tile j - 2 until that tile's P V has finished;
@@ -256,11 +279,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 if (ok) ok = mbar_wait(k_full(ks), (j / KST) & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
+                const uint64_t dk = dk0 + (uint64_t)((ks * TILE_BYTES) >> 4);
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k) {
-                    const uint32_t off = (k >> 2) * HALF_BYTES + (k & 3) * 32u;
-                    mma_bf16(tmem + sb * TN, sdesc(sQ + off, 16, 1024), sdesc(sK(ks) + off, 16, 1024), IDESC_QK,
-                             k > 0 ? 1u : 0u);
+                    const uint32_t off = ((k >> 2) * HALF_BYTES + (k & 3) * 32u) >> 4;
+                    mma_bf16(tmem + sb * TN, dq + off, dk + off, IDESC_QK, k > 0 ? 1u : 0u);
                 }
                 mma_commit(s_full(sb));
                 mma_commit(k_empty(ks));
@@ -279,9 +302,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // ---------------- O += P V issuer (one thread)
         if (ntiles > 0 && lane == 0) {
             bool ok = true, issued_any = false;
+            const uint64_t dv0 = sdesc(sV(0), HALF_BYTES, 1024);
             for (int t = 0; ok && t < ntiles; ++t) {
                 const int vs = t % VST;
                 ok = mbar_wait(v_full(vs), (t / VST) & 1, abort_flag);
+                const uint64_t dv = dv0 + (uint64_t)((vs * TILE_BYTES) >> 4);
                 for (int x = 0; ok && x < 2; ++x) {
                     ok = mbar_wait(p_full(x), t & 1, abort_flag);
                     if (!ok) break;
@@ -289,8 +314,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                     for (int k = 0; k < HALF_N / 16; ++k)
                         mma_bf16_ts(tmem + O_COL + x * HD, tmem + (t & 1) * TN + x * HALF_N + k * 8,
-                                    sdesc(sV(vs) + (x * 4 + k) * 2048u, HALF_BYTES, 1024), IDESC_PV,
-                                    (t > 0 || k > 0) ? 1u : 0u);
+                                    dv + (uint64_t)(((x * 4 + k) * 2048u) >> 4), IDESC_PV, (t > 0 || k > 0) ? 1u : 0u);
                     mma_commit(o_done(x));
                     issued_any = true;
                 }
@@ -319,7 +343,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int node = row_ok ? gr / G : 0;
         const int head = kvh * G + (row_ok ? gr % G : 0);
         uint32_t an0 = 0, an1 = 0, an2 = 0, an3 = 0;
-        if (row_ok) {
+        if (row_ok && !a.parent) {
+            // a chain: node i's ancestors are nodes 0..i (the causal tail), no walk needed
+            an0 = below(node + 1, 0);
+            an1 = below(node + 1, 1);
+            an2 = below(node + 1, 2);
+            an3 = below(node + 1, 3);
+        } else if (row_ok) {
             int steps = 0;
             for (int jn = node; jn >= 0 && jn < N && steps <= N; jn = s_par[jn], ++steps) {
                 const uint32_t bit = 1u << (jn & 31);
@@ -380,20 +410,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             // whose scores were read above
             float s4[4] = {0.f, 0.f, 0.f, 0.f};
             {
-                uint32_t pk[32];
+                uint32_t pp[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const float e0 = ex2(fmaf(x[2 * i], sl, -mu));
                     const float e1 = ex2(fmaf(x[2 * i + 1], sl, -mu));
                     s4[(2 * i) & 3] += e0;
                     s4[(2 * i + 1) & 3] += e1;
-                    pk[i] = pack_bf16(e0, e1);
+                    pp[i] = pack_bf16(e0, e1);
                 }
-                tmem_st_x32(tmem + lane_base + sb * TN + X * HALF_N, pk);
+                tmem_st_x32(tmem + lane_base + sb * TN + X * HALF_N, pp);
             }
             l_run = l_run * f + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
             if (lim < TN) {
-                // value rows past the split end may hold stale data: clear this group's ones
+                // value rows past the split end are not loaded (or hold another
+                // sequence's data): clear this group's ones
                 const int tok = X * HALF_N + (r & 63);
                 if (tok >= lim) {
                     const int vs = j % VST;
@@ -452,61 +483,69 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 tmem_ld_x32(tmem + lane_base + O_COL + HD + X * 64 + c32 * 32, rb);
             }
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                o[c32 * 32 + i] = have_o ? (wA * __uint_as_float(ra[i]) + wB * __uint_as_float(rb[i])) * inv
-                                         : (bad ? NAN : 0.f);
+            for (int i = 0; i < 16; ++i) {
+                const float o0 = have_o ? (wA * __uint_as_float(ra[2 * i]) + wB * __uint_as_float(rb[2 * i])) * inv
+                                        : (bad ? NAN : 0.f);
+                const float o1 = have_o ? (wA * __uint_as_float(ra[2 * i + 1]) + wB * __uint_as_float(rb[2 * i + 1])) *
+                                              inv
+                                        : (bad ? NAN : 0.f);
+                pk[c32 * 16 + i] = pack_bf16(o0, o1);
+            }
         }
         tc_fence_before();
-        if (S > 1) {
-            // this split's partial row straight to the workspace: the group's 64
-            // outputs as bf16, and (group A) the row's log-sum-exp
-            const size_t group = ((size_t)b * a.Hkv + kvh) * a.row_tiles + tile;
-            uint8_t* prow = reinterpret_cast<uint8_t*>(a.o_part) + ((group * S + split) * TM + r) * PROW_BYTES;
-            uint4* dst = reinterpret_cast<uint4*>(prow + X * HD);
-#pragma unroll
-            for (int q8 = 0; q8 < 8; ++q8)
-                dst[q8] = make_uint4(pack_bf16(o[q8 * 8 + 0], o[q8 * 8 + 1]), pack_bf16(o[q8 * 8 + 2], o[q8 * 8 + 3]),
-                                     pack_bf16(o[q8 * 8 + 4], o[q8 * 8 + 5]), pack_bf16(o[q8 * 8 + 6], o[q8 * 8 + 7]));
-            if (X == 0) *reinterpret_cast<float*>(prow + 2 * HD) = lse;
-        }
         if (S == 1 && row_ok) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
                                                   (((size_t)b * N + node) * a.Hq + head) * HD + X * 64);
 #pragma unroll
-            for (int q8 = 0; q8 < 8; ++q8) {
-                uint4 v;
-                v.x = pack_bf16(o[q8 * 8 + 0], o[q8 * 8 + 1]);
-                v.y = pack_bf16(o[q8 * 8 + 2], o[q8 * 8 + 3]);
-                v.z = pack_bf16(o[q8 * 8 + 4], o[q8 * 8 + 5]);
-                v.w = pack_bf16(o[q8 * 8 + 6], o[q8 * 8 + 7]);
-                dst[q8] = v;
-            }
+            for (int q8 = 0; q8 < 8; ++q8)
+                dst[q8] = make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]);
         }
     }
 
-    __syncthreads();  // every role finished; all TMEM reads completed
+    __syncthreads();  // every role finished; all TMEM reads completed; the rings are idle
     if (warp == 2) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
     }
     if (S > 1) {
-        // ---- merge the KV splits of this row tile.  Each split has written its
-        // normalised partial rows (bf16) and their log-sum-exp to the workspace; it
-        // counts itself in, and once all S splits are in combines an equal share of
-        // the rows from all S partials.
-        const size_t group = ((size_t)b * a.Hkv + kvh) * a.row_tiles + tile;
-        const uint8_t* part = reinterpret_cast<const uint8_t*>(a.o_part) + group * (size_t)S * TM * PROW_BYTES;
-        unsigned* arrive = a.counters + 2 * group;  // [groups][2]: arrivals, departures
-        __shared__ int s_all_in;
+        // ---- merge the KV splits of this row tile through the cluster's shared memory.
+        // Rows [k R, k R + R) belong to CTA k (split k); each CTA receives, in its idle
+        // K ring, S partial rows (one per split) for each row it owns, laid out
+        // [split][row - k R] with PROW_BYTES per row: 128 bf16 outputs, then the fp32
+        // log-sum-exp.
+        const int R = (TM + S - 1) / S;
+        const int own = max(0, min(TM, (split + 1) * R) - split * R);
+        const uint32_t recv = base + SK_OFF;
+        // every CTA of the cluster has initialised its barriers
+        asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
         if (tid == 0) {
-            count_in(arrive);
-            s_all_in = wait_count(arrive, (unsigned)S, abort_flag) ? 1 : 0;
+            mbar_expect_tx(merge_bar, (uint32_t)(own * S) * PUSH_BYTES);
+            // this CTA's ring is free: tell every CTA of the cluster it may push
+            for (int k = 0; k < S; ++k) mbar_arrive_cluster(mapa_shared(free_bar, (uint32_t)k));
         }
+        if (warp >= 4) {
+            // push once every CTA can receive (NaN rows if this CTA failed: the owners
+            // still get every byte they wait for)
+            if (__all_sync(0xffffffffu, mbar_wait_cluster_bounded(free_bar, 0))) {
+                const int owner = r / R, slot = r % R;
+                const uint32_t row = recv + (uint32_t)((split * R + slot) * PROW_BYTES);
+                const uint32_t dst = mapa_shared(row + X * HD, (uint32_t)owner);
+                const uint32_t mb = mapa_shared(merge_bar, (uint32_t)owner);
+#pragma unroll
+                for (int q8 = 0; q8 < 8; ++q8)
+                    st_async_v4(dst + q8 * 16, pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3], mb);
+                if (X == 0) st_async_b32(mapa_shared(row + 2 * HD, (uint32_t)owner), __float_as_uint(lse), mb);
+            } else if (lane == 0) {
+                *abort_flag = 1;
+            }
+        }
+        // every partial row of this CTA's share has arrived (always waited for, bounded:
+        // no peer may still write to this CTA's shared memory when it retires)
+        if (tid == 0) s_got = mbar_wait_cluster_bounded(merge_bar, 0) ? 1 : 0;
         __syncthreads();
-        if (!s_all_in) {
-            // a peer never arrived: leave this CTA's share of the rows as NaN
-            const int R = (TM + S - 1) / S;
-            const int own = max(0, min(TM, (split + 1) * R) - split * R);
+        const uint8_t* part = base_ptr + SK_OFF;
+        if (!s_got) {
+            *abort_flag = 1;
             for (int item = tid; item < own * (HD / 4); item += TC_THREADS) {
                 const int rt = split * R + item / (HD / 4), gr = tile * TM + rt;
                 if (gr >= G * n) continue;
@@ -517,31 +556,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) +
                                           (((size_t)b * N + node) * a.Hq + head) * HD + (item % (HD / 4)) * 4) = ov;
             }
-        } else
-        switch (S) {
-            case 2: merge_rows<TM, TC_THREADS, 2>(a, part, split, tile, b, kvh, tid, G * n); break;
-            case 3: merge_rows<TM, TC_THREADS, 3>(a, part, split, tile, b, kvh, tid, G * n); break;
-            case 4: merge_rows<TM, TC_THREADS, 4>(a, part, split, tile, b, kvh, tid, G * n); break;
-            case 5: merge_rows<TM, TC_THREADS, 5>(a, part, split, tile, b, kvh, tid, G * n); break;
-            case 6: merge_rows<TM, TC_THREADS, 6>(a, part, split, tile, b, kvh, tid, G * n); break;
-            case 7: merge_rows<TM, TC_THREADS, 7>(a, part, split, tile, b, kvh, tid, G * n); break;
-            case 8: merge_rows<TM, TC_THREADS, 8>(a, part, split, tile, b, kvh, tid, G * n); break;
-            case 9: merge_rows<TM, TC_THREADS, 9>(a, part, split, tile, b, kvh, tid, G * n); break;
-            case 10: merge_rows<TM, TC_THREADS, 10>(a, part, split, tile, b, kvh, tid, G * n); break;
-            case 11: merge_rows<TM, TC_THREADS, 11>(a, part, split, tile, b, kvh, tid, G * n); break;
-            case 12: merge_rows<TM, TC_THREADS, 12>(a, part, split, tile, b, kvh, tid, G * n); break;
-            case 13: merge_rows<TM, TC_THREADS, 13>(a, part, split, tile, b, kvh, tid, G * n); break;
-            case 14: merge_rows<TM, TC_THREADS, 14>(a, part, split, tile, b, kvh, tid, G * n); break;
-            case 15: merge_rows<TM, TC_THREADS, 15>(a, part, split, tile, b, kvh, tid, G * n); break;
-            default: merge_rows<TM, TC_THREADS, 16>(a, part, split, tile, b, kvh, tid, G * n); break;
-        }
-        __syncthreads();
-        if (tid == 0 && atomicAdd(arrive + 1, 1u) == (unsigned)(S - 1)) {
-            // the last split out: every peer has passed its wait, so both counters
-            // can return to zero for the next call
-            arrive[0] = 0u;
-            arrive[1] = 0u;
-            __threadfence();
+        } else {
+            switch (S) {
+                case 2: merge_rows<TM, TC_THREADS, 2>(a, part, R, split, tile, b, kvh, tid, G * n); break;
+                case 3: merge_rows<TM, TC_THREADS, 3>(a, part, R, split, tile, b, kvh, tid, G * n); break;
+                case 4: merge_rows<TM, TC_THREADS, 4>(a, part, R, split, tile, b, kvh, tid, G * n); break;
+                case 5: merge_rows<TM, TC_THREADS, 5>(a, part, R, split, tile, b, kvh, tid, G * n); break;
+                case 6: merge_rows<TM, TC_THREADS, 6>(a, part, R, split, tile, b, kvh, tid, G * n); break;
+                case 7: merge_rows<TM, TC_THREADS, 7>(a, part, R, split, tile, b, kvh, tid, G * n); break;
+                case 8: merge_rows<TM, TC_THREADS, 8>(a, part, R, split, tile, b, kvh, tid, G * n); break;
+                case 9: merge_rows<TM, TC_THREADS, 9>(a, part, R, split, tile, b, kvh, tid, G * n); break;
+                case 10: merge_rows<TM, TC_THREADS, 10>(a, part, R, split, tile, b, kvh, tid, G * n); break;
+                case 11: merge_rows<TM, TC_THREADS, 11>(a, part, R, split, tile, b, kvh, tid, G * n); break;
+                case 12: merge_rows<TM, TC_THREADS, 12>(a, part, R, split, tile, b, kvh, tid, G * n); break;
+                case 13: merge_rows<TM, TC_THREADS, 13>(a, part, R, split, tile, b, kvh, tid, G * n); break;
+                case 14: merge_rows<TM, TC_THREADS, 14>(a, part, R, split, tile, b, kvh, tid, G * n); break;
+                case 15: merge_rows<TM, TC_THREADS, 15>(a, part, R, split, tile, b, kvh, tid, G * n); break;
+                default: merge_rows<TM, TC_THREADS, 16>(a, part, R, split, tile, b, kvh, tid, G * n); break;
+            }
         }
     }
     if (tid == 0) {
@@ -550,76 +582,111 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
 }
 
-bool tc_attrs_ready() {
-    static int state = -1;
-    if (state < 0) {
-        state = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) ==
-                cudaSuccess;
-        cudaGetLastError();
-    }
-    return state == 1;
-}
+// Per-device launch facts, looked up once per device with that device current:
+// whether the kernel's shared-memory and cluster-size attributes are set, and
+// how many clusters of each split count the device holds at once.
+struct TcDeviceInfo {
+    int state = 0;                    // 0 unknown, 1 ready, -1 unusable
+    int clusters[MAX_SPLITS + 1] = {};  // [s]: clusters of s CTAs resident at once (s = 1: CTAs)
+};
+constexpr int MAX_DEVICES = 64;
+std::mutex g_info_mutex;
+TcDeviceInfo g_info[MAX_DEVICES];
 
-// CTAs of this kernel the device holds at once (-1 if it cannot be queried)
-int tc_resident_ctas() {
-    static int cached = 0;
-    if (cached == 0) {
-        int n = -1, per_sm = 0, dev = 0, sms = 0;
-        if (tc_attrs_ready() && cudaGetDevice(&dev) == cudaSuccess &&
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_tc_kernel, TC_THREADS, SMEM_BYTES) ==
-                cudaSuccess)
-            n = per_sm * sms;
+const TcDeviceInfo* tc_device_info() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) {
         cudaGetLastError();
-        cached = n;
+        return nullptr;
     }
-    return cached;
+    std::lock_guard<std::mutex> lock(g_info_mutex);
+    TcDeviceInfo& d = g_info[dev];
+    if (d.state == 0) {
+        d.state = -1;
+        if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) ==
+                cudaSuccess &&
+            cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+            d.state = 1;
+            int per_sm = 0, sms = 0;
+            if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_tc_kernel, TC_THREADS, SMEM_BYTES) ==
+                    cudaSuccess)
+                d.clusters[1] = per_sm * sms;
+            for (int s = 2; s <= MAX_SPLITS; ++s) {
+                cudaLaunchConfig_t cfg = {};
+                cudaLaunchAttribute attr[1];
+                cfg.gridDim = dim3(s, 1, 1);
+                cfg.blockDim = dim3(TC_THREADS, 1, 1);
+                cfg.dynamicSmemBytes = SMEM_BYTES;
+                attr[0].id = cudaLaunchAttributeClusterDimension;
+                attr[0].val.clusterDim.x = s;
+                attr[0].val.clusterDim.y = 1;
+                attr[0].val.clusterDim.z = 1;
+                cfg.attrs = attr;
+                cfg.numAttrs = 1;
+                int c = 0;
+                if (cudaOccupancyMaxActiveClusters(&c, attn_tc_kernel, &cfg) != cudaSuccess) c = 0;
+                d.clusters[s] = c;
+            }
+        }
+        cudaGetLastError();
+    }
+    return &d;
 }
 
 }  // namespace
 
 int tc_rows_per_tile() { return TM; }
 int tc_max_splits() { return MAX_SPLITS; }
-size_t tc_counter_offset(int64_t groups, int splits) {
-    return (size_t)groups * splits * TM * PROW_BYTES;
-}
-size_t tc_workspace_bytes(int64_t groups, int splits) {
-    if (splits <= 1) return 0;
-    return tc_counter_offset(groups, splits) + (((size_t)groups * 2 * sizeof(unsigned) + 255) & ~(size_t)255);
-}
 
-// KV splits per row tile: as many as keep the whole grid resident at once
-// (one wave, which the cooperative merge requires), at most 16, and at least
-// 256 tokens per split.
-int tc_pick_splits(int64_t groups, int64_t max_tokens, int sms) {
-    int cap = tc_resident_ctas();
-    if (cap <= 0) cap = sms;
+// KV splits per row tile (the splits of a tile form one cluster).  Splitting
+// pays only while the grid fills less than half of the GPU.  Among 2..16
+// splits (at least 256 tokens each) take the one with the fewest tiles on the
+// longest path: waves of clusters the device holds at once, times the tiles
+// of one split.  Without a device (host-only planning) every SM is assumed to
+// hold one CTA and a cluster of s CTAs to need s SMs.
+int tc_pick_splits(int64_t groups, int64_t max_blocks, int sms) {
+    const TcDeviceInfo* info = tc_device_info();
+    const bool known = info && info->state == 1 && info->clusters[1] > 0;
+    const int64_t cap = known ? info->clusters[1] : sms;
     if (groups * 2 > cap) return 1;
-    int64_t s = cap / groups;
-    if (s > MAX_SPLITS) s = MAX_SPLITS;
-    const int64_t by_len = max_tokens / 256;
-    if (s > by_len) s = by_len;
-    return s < 1 ? 1 : (int)s;
+    const int64_t tiles1 = (max_blocks + BLK_PER_TILE - 1) / BLK_PER_TILE;
+    int best = 1;
+    int64_t best_cost = tiles1 * ((groups + cap - 1) / cap);
+    for (int s = 2; s <= MAX_SPLITS; ++s) {
+        if (max_blocks < (int64_t)s * 16) break;  // at least 256 tokens per split
+        const int64_t per_wave = known ? info->clusters[s] : sms / s;
+        if (per_wave <= 0) continue;
+        const int64_t bps = (max_blocks + s - 1) / s;
+        const int64_t cost = ((groups + per_wave - 1) / per_wave) * ((bps + BLK_PER_TILE - 1) / BLK_PER_TILE);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = s;
+        }
+    }
+    return best;
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st, int* launches) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
-    if (a.D != HD || a.splits < 1 || a.splits > MAX_SPLITS) return cudaErrorInvalidValue;
+    if (a.D != HD || a.splits < 1 || a.splits > MAX_SPLITS || a.blocks_per_split < 1) return cudaErrorInvalidValue;
     CUtensorMap mk, mv;
     if (!make_kv_map(fn, &mk, a.k, a.Hkv, a.num_blocks) || !make_kv_map(fn, &mv, a.v, a.Hkv, a.num_blocks))
         return cudaErrorInvalidValue;
-    if (!tc_attrs_ready()) return cudaErrorInvalidDeviceFunction;
-    if (a.splits > 1 && (!a.o_part || !a.counters)) return cudaErrorInvalidValue;
+    const TcDeviceInfo* info = tc_device_info();
+    if (!info || info->state != 1) return cudaErrorInvalidDeviceFunction;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attrs[1];
     cfg.gridDim = dim3(a.splits, a.row_tiles, a.B * a.Hkv);
     cfg.blockDim = dim3(TC_THREADS, 1, 1);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = st;
-    // the split merge waits on peers of the same launch: every CTA must be resident
-    attrs[0].id = cudaLaunchAttributeCooperative;
-    attrs[0].val.cooperative = 1;
+    // the splits of a row tile merge through each other's shared memory: one cluster
+    attrs[0].id = cudaLaunchAttributeClusterDimension;
+    attrs[0].val.clusterDim.x = a.splits;
+    attrs[0].val.clusterDim.y = 1;
+    attrs[0].val.clusterDim.z = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = a.splits > 1 ? 1 : 0;
     *launches = 1;

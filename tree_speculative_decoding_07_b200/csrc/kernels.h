@@ -15,13 +15,11 @@ struct AttnArgs {
     const int32_t* parent;  // [B][N]; NULL: every tree is a chain (parent of node i is i - 1)
     const int32_t* counts;  // [B] nodes per sequence (0..N); NULL: N for every sequence
     void* out;
-    float* o_part;      // CUDA-core path: [splits][B][N][Hq][D] fp32 partial outputs (normalised);
-                        // tensor-core path: [groups][splits][128] partial rows of 272 bytes
-                        // (128 bf16 outputs, fp32 log-sum-exp, padding)
-    float* lse_part;    // [splits][B][N][Hq] log2-domain log-sum-exp of each partial
-    unsigned* counters; // tensor-core path: [groups][2] arrival / departure counts, zero between calls
+    float* o_part;      // CUDA-core path: [splits][B][N][Hq][D] fp32 partial outputs (normalised)
+    float* lse_part;    // CUDA-core path: [splits][B][N][Hq] log2-domain log-sum-exp of each partial
     int32_t* status;
     int B, N, Hq, Hkv, G, D, max_blocks, num_blocks, splits, row_tiles;
+    int blocks_per_split;  // tensor-core path: split s covers logical blocks [s * bps, (s + 1) * bps)
     float scale_log2;   // softmax_scale * log2(e)
 };
 
@@ -33,9 +31,7 @@ int simt_rows_per_tile();
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st, int* launches);
 int tc_rows_per_tile();
 int tc_max_splits();
-int tc_pick_splits(int64_t groups, int64_t max_tokens, int sms);
-size_t tc_workspace_bytes(int64_t groups, int splits);
-size_t tc_counter_offset(int64_t groups, int splits);
+int tc_pick_splits(int64_t groups, int64_t max_blocks, int sms);
 
 struct SampleArgs {
     const float* p;
@@ -105,5 +101,22 @@ int tree_merge(int num_seqs, const int32_t* offsets, const int32_t* tokens, int 
 // Dynamic tree selection from a candidate set (host).  Returns the node count, -1 if not topological.
 int tree_select(const int32_t* cand_parent, const int32_t* cand_token, const double* cand_prob, int M, int budget,
                 int32_t* parent_idx, int32_t* tree_tokens, int32_t* cand_index, double* value);
+
+// Dynamic tree selection on the device: one CTA per sequence (one launch).
+struct SelectArgs {
+    const int32_t* offsets;      // [B + 1] candidate ranges
+    const int32_t* cand_parent;  // parent candidate (local to the sequence), -1 for a child of the root
+    const int32_t* cand_token;
+    const float* cand_prob;
+    int32_t* parent_idx;         // [B][budget]
+    int32_t* tree_tokens;        // [B][budget]
+    int32_t* cand_index;         // [B][budget]
+    int32_t* node_counts;        // [B]
+    double* expected;            // [B]
+    int32_t* status;
+    int B, budget, max_cand;
+};
+size_t select_smem_bytes(int max_cand, int budget);
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
 
 }  // namespace tv

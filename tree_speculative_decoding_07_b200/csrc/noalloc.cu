@@ -16,9 +16,14 @@
 
 namespace {
 
-// Fixed scratch: the tensor-core path needs 67,584 bytes per CTA of a split
-// launch plus 8 bytes of counters per row tile, and its launches never exceed
-// the CTAs resident on one GPU (148 on a B200), so 12 MiB covers it with room.
+// Fixed scratch.  Tensor-core calls (bf16, head_dim 128) merge their KV splits
+// through the cluster's shared memory and need none.  CUDA-core calls with
+// several KV splits keep fp32 partial outputs and their log-sum-exp for every
+// (split, query row): 4 * (head_dim + 1) bytes each.  The split count is chosen
+// so splits x query rows stay within 32 rows per SM (4,736 on a 148-SM B200),
+// i.e. at most about 2.4 MB at head_dim 128 and 1.2 MB at 64; 2 MiB covers
+// every head_dim-64 call and head_dim-128 calls up to about 4,000
+// (split, row) pairs, and larger ones are refused with TV_ERR_WORKSPACE.
 __device__ __align__(256) unsigned char g_scratch[TV_STATIC_SCRATCH_BYTES];
 
 constexpr int MAX_DEVICES = 64;
@@ -58,16 +63,8 @@ extern "C" tv_status tv_tree_attention_static(const tv_attn_desc* desc, const vo
     if (plan.workspace_bytes) {
         s = scratch_address(&scratch);
         if (s != TV_OK) return s;
-        if (plan.kernel == 0) {
-            // the split merge's arrival counters must start at zero; the array keeps
-            // whatever the previous call left, so clear them (the partial rows are
-            // always overwritten before they are read)
-            const int64_t groups = (int64_t)desc->batch * desc->num_kv_heads * plan.row_tiles;
-            const size_t off = tv::tc_counter_offset(groups, plan.num_splits);
-            if (cudaMemsetAsync(static_cast<char*>(scratch) + off, 0, plan.workspace_bytes - off,
-                                static_cast<cudaStream_t>(stream)) != cudaSuccess)
-                return TV_ERR_CUDA;
-        }
+        // every partial the merge reads is written earlier in the same call, so
+        // nothing in the array needs clearing
     }
     return tv_tree_attention(desc, q, paged_k, paged_v, block_table, prefix_lens, parent_idx, out, scratch,
                              plan.workspace_bytes ? (size_t)TV_STATIC_SCRATCH_BYTES : 0, dev_status, stream);

@@ -184,49 +184,28 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
     return __all_sync(0xffffffffu, ok);
 }
 
-// per-tile arrival counter: increment after a release fence, bounded
-// acquire spin for the target count
-__device__ __forceinline__ unsigned count_in(unsigned* cnt) {
-    __threadfence();
-    return atomicAdd(cnt, 1u);
-}
-__device__ __forceinline__ bool wait_count(const unsigned* cnt, unsigned target, volatile int* abort_flag) {
-    const long long t0 = clock64();
-    for (;;) {
-        unsigned v;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
-        if (v >= target) return true;
-        if (clock64() - t0 > WAIT_LIMIT) {
-            *abort_flag = 1;
-            return false;
-        }
-        __nanosleep(32);
-    }
-}
-
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
-// Combine rows [split * R, split * R + R) of one ROWS-row tile from the S
-// partials in the workspace (layout [S][ROWS] rows of PROW_BYTES):
+// Combine this CTA's share of one ROWS-row tile, rows [split * R, split * R + own),
+// from the S partials it received into shared memory (layout [S][R] rows of
+// PROW_BYTES: 128 bf16 outputs, then the fp32 log-sum-exp):
 // out = sum_s 2^(lse_s - m) o_s / sum_s 2^(lse_s - m), m = max_s lse_s.
 // Each item is 8 columns of one row, so a thread issues all its loads at once.
 template <int ROWS, int THREADS, int S_>
-__device__ __forceinline__ void merge_rows(const AttnArgs& a, const uint8_t* part, int split, int tile, int b, int kvh,
-                                           int tid, int nrows) {
-    constexpr int R = (ROWS + S_ - 1) / S_;
+__device__ __forceinline__ void merge_rows(const AttnArgs& a, const uint8_t* part, int R, int split, int tile, int b,
+                                           int kvh, int tid, int nrows) {
     constexpr int NC = HD / 8;
     const int own = max(0, min(ROWS, (split + 1) * R) - split * R);
     for (int item = tid; item < own * NC; item += THREADS) {
         const int rr = item / NC, cc = item % NC;
-        const int rt = split * R + rr;
-        const int gr = tile * ROWS + rt;
+        const int gr = tile * ROWS + split * R + rr;
         if (gr >= nrows) continue;  // rows of nodes past the sequence's tree
         float ls[S_];
         uint4 v[S_];
 #pragma unroll
         for (int k = 0; k < S_; ++k) {
-            const uint8_t* prow = part + ((size_t)k * ROWS + rt) * PROW_BYTES;
+            const uint8_t* prow = part + ((size_t)k * R + rr) * PROW_BYTES;
             ls[k] = *reinterpret_cast<const float*>(prow + 2 * HD);
             v[k] = reinterpret_cast<const uint4*>(prow)[cc];
         }
@@ -261,6 +240,51 @@ __device__ __forceinline__ void merge_rows(const AttnArgs& a, const uint8_t* par
         *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + (((size_t)b * a.N + node) * a.Hq + head) * HD +
                                   cc * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
+}
+
+// ---- cluster (distributed shared memory) operations of the split merge
+
+// address of the same shared-memory location in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+// arrive on an mbarrier of any CTA of the cluster (release at cluster scope)
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// Bounded wait (acquire at cluster scope) on a phase of this CTA's mbarrier that
+// other CTAs of the cluster complete.  It does not give up early when this CTA
+// aborted: the bytes a peer pushes must have landed before the CTA retires.
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t parity) {
+    const long long t0 = clock64();
+    for (;;) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (clock64() - t0 > WAIT_LIMIT) return false;
+    }
+}
+// 16 / 4 bytes into the shared memory of a CTA of the cluster, completing that
+// many transaction bytes on the receiver's mbarrier
+__device__ __forceinline__ void st_async_v4(uint32_t remote, uint32_t x, uint32_t y, uint32_t z, uint32_t w,
+                                            uint32_t remote_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     remote),
+                 "r"(x), "r"(y), "r"(z), "r"(w), "r"(remote_bar)
+                 : "memory");
+}
+__device__ __forceinline__ void st_async_b32(uint32_t remote, uint32_t x, uint32_t remote_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote), "r"(x),
+                 "r"(remote_bar)
+                 : "memory");
 }
 
 template <int NV>
