@@ -576,6 +576,42 @@ def measure_config(tv, name: str, seed: int, W: int, K: int, flush, stream, peak
     return res, (wl, h, st, walk, attn_ms, samp_ms)
 
 
+def time_select(tv, flush, stream, W, K, batch=64, per_seq=512, width=8, budget=64):
+    """tv_tree_select_device (the dynamic tree, EAGLE-2) on grown candidate sets:
+    `batch` sequences of `per_seq` candidates, trees of `budget` nodes; its own
+    graph, L2 flushed before each launch."""
+    import torch
+    import synth
+    off, par, tok, prob = synth.grown_candidates(batch, per_seq, width, seed=5)
+    d = to_device({"off": off, "par": par, "tok": tok, "prob": prob})
+    B = batch
+    parent = torch.empty((B, budget), dtype=torch.int32, device="cuda")
+    tokens = torch.empty_like(parent)
+    index = torch.empty_like(parent)
+    counts = torch.empty((B,), dtype=torch.int32, device="cuda")
+    val = torch.empty((B,), dtype=torch.float64, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def call(st):
+        s = tv.tv_tree_select_device(B, per_seq, d["off"], d["par"], d["tok"], d["prob"], budget, parent, tokens,
+                                     index, counts, val, status, st)
+        if s:
+            raise tv.TreeVerifyError(s, "tv_tree_select_device")
+
+    call(stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call(torch.cuda.current_stream())
+    ms = timed_replays(g, flush, stream, W, K)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} from the tree selection")
+    del g
+    return {"us": float(np.mean(ms)) * 1e3, "sequences": B, "candidates_per_sequence": per_seq, "budget": budget,
+            "note": "tv_tree_select_device on level-by-level grown candidates (width 8, best third expanded); "
+                    "mean over launches, L2 flushed before each"}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -638,6 +674,7 @@ def run_ours(args, rank, world, local_rank):
     commit = time_commit(tv, wl, d, flush, stream, W, min(K, 200))
     logits_walk = time_logits_walk(tv, wl, d, flush, stream, W, min(K, 200), walk)
     fill = time_fill_topk(tv, wl, d, flush, stream, W, min(K, 200))
+    select = time_select(tv, flush, stream, W, min(K, 200))
     total_ms = float(sum(step_ms))
 
     # ---- end to end: host (pinned) inputs -> device -> results back, every step
@@ -734,6 +771,7 @@ def run_ours(args, rank, world, local_rank):
         "commit": commit,
         "sample_logits": logits_walk,
         "tree_fill_topk": fill,
+        "tree_select_device": select,
         "e2e": {"value": e2e_value, "unit": "nodes/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": K2},
         "gpu_launches": K * (st.aplan.launches + st.splan.launches),

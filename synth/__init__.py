@@ -538,3 +538,35 @@ def _greedy_budget_tree(seed, N, V, mode, sp, sn, max_depth, width):
     tokens = np.array([created_token[o] for o in order], dtype=np.int32)
     keys = np.array(order, dtype=np.int64)
     return parents, tokens, keys
+
+
+def grown_candidates(batch: int, per_seq: int, width: int, seed: int):
+    """Candidate sets for dynamic tree selection, grown as a draft model would
+    grow them level by level: each level gives `width` children to the best
+    third of the previous level's nodes (by path probability), each child's
+    probability drawn from Philox as u**2 (a draft's top-k tail).  Returns
+    (offsets [B+1], parent [sum], token [sum], prob [sum] float32); parent
+    indices are local to the sequence (-1 = a child of the root)."""
+    par_all, tok_all, prob_all, offs = [], [], [], [0]
+    for b in range(batch):
+        u = uniforms(2 * per_seq, seed, STREAM_TREE, b << 20)
+        par, prob, score = [], [], []
+        frontier = [(-1, 1.0)]
+        while len(par) < per_seq:
+            nxt = []
+            for node, s in frontier:
+                for _ in range(width):
+                    if len(par) >= per_seq:
+                        break
+                    pr = float(np.float32(u[len(par)] ** 2))
+                    par.append(node)
+                    prob.append(pr)
+                    nxt.append((len(par) - 1, s * pr))
+            nxt.sort(key=lambda t: -t[1])
+            frontier = nxt[: max(1, len(nxt) // 3)]
+        par_all += par
+        prob_all += prob
+        tok_all += [int(w % 128256) for w in words(per_seq, seed, STREAM_TOKEN, b << 20)]
+        offs.append(offs[-1] + per_seq)
+    return (np.array(offs, np.int32), np.array(par_all, np.int32), np.array(tok_all, np.int32),
+            np.array(prob_all, np.float32))

@@ -438,7 +438,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             // this group's previous P V must be complete before O is rescaled and
             // before P V of this tile is released (every phase is waited, in order)
             if (j > 0 && !warp_wait(o_done(X), (j - 1) & 1, abort_flag)) break;
-            if (f != 1.f && j > 0) {
+            // tcgen05.ld / st are warp-collective (.sync.aligned): the whole warp rescales
+            // when any of its rows needs it (rows whose max did not move multiply by 1)
+            if (j > 0 && __any_sync(0xffffffffu, f != 1.f)) {
                 tc_fence_after();
 #pragma unroll
                 for (int c4 = 0; c4 < HD / 32; ++c4) {
