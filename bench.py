@@ -716,7 +716,8 @@ def run_ours(args, rank, world, local_rank):
     peak, peak_kind, pk = load_peaks()
     peaks = {"hbm": peak, "bf16_sustained": float(pk.get("bf16_tflops_sustained", FALLBACK_BF16_SUSTAINED))}
     configs = {}
-    if not args.no_configs:
+    # every workload, at one GPU only (under torchrun each rank would repeat them)
+    if not args.no_configs and world == 1:
         for name in ("tiny", "l8b", "l70b", "mix", "long", "ragged"):
             try:
                 r, _ = measure_config(tv, name, 1 + 1000 * rank if name == args.workload else None, W,
