@@ -10,11 +10,12 @@
 // 128-row tile of those rows and one KV split: a fixed range of logical
 // blocks of the block table (known at launch, so the block ids are fetched
 // before the sequence's length arrives).  The S splits of a row tile form one
-// thread-block cluster; when all have finished their tokens, each pushes its
-// normalised partial rows (bf16) and their log-sum-exp into the shared memory
-// of the CTA that owns each row (an equal share per CTA, st.async completing on
-// the owner's mbarrier), and each owner combines its rows from the S partials
-// (flash-decoding log-sum-exp merge).  No global workspace is used.
+// thread-block cluster; when all have finished their tokens, each stages its
+// normalised partial rows (bf16) and their log-sum-exp in its idle V ring and
+// sends each CTA the rows that CTA owns (an equal share per CTA) with one bulk
+// shared-to-shared copy, completing on the owner's mbarrier; each owner
+// combines its rows from the S partials (flash-decoding log-sum-exp merge).
+// No global workspace is used.
 //
 // Warp roles (384 threads):
 //   warp 0      TMA producer of K tiles, warp 3 of V tiles: the rows of 8 paged
@@ -79,8 +80,8 @@ constexpr int BAR_FREE = BAR_DRAIN_PV + 1;       // S arrivals: every CTA of the
 constexpr int BAR_MERGE = BAR_FREE + 1;          // this CTA's share of partial rows received (transaction count)
 constexpr int BAR_COUNT = BAR_MERGE + 1;
 static_assert(BAR_COUNT == 2 * KST + 2 * VST + 13, "barrier slots overlap");
-// bytes pushed per (partial row, split): 128 bf16 outputs and the fp32 log-sum-exp
-constexpr uint32_t PUSH_BYTES = 2 * HD + 4;
+static_assert(TM * PROW_BYTES <= VST * TILE_BYTES, "staged partial rows exceed the V ring");
+static_assert((TM + MAX_SPLITS) * PROW_BYTES <= KST * TILE_BYTES, "received partial rows exceed the K ring");
 
 __global__ void __launch_bounds__(TC_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tmk,
@@ -501,6 +502,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
             for (int q8 = 0; q8 < 8; ++q8)
                 dst[q8] = make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]);
+        } else if (S > 1) {
+            // stage this row's partial in the V ring (every P V has finished: both groups
+            // waited for their last one before the barrier above): row r at r * PROW_BYTES,
+            // group X's 64 outputs at byte X * 128, the log-sum-exp at byte 256
+            const uint32_t row = base + SV_OFF + (uint32_t)r * PROW_BYTES;
+#pragma unroll
+            for (int q8 = 0; q8 < 8; ++q8)
+                st_shared_v4(row + X * HD + q8 * 16, make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]));
+            if (X == 0) st_shared_v4(row + 2 * HD, make_uint4(__float_as_uint(lse), 0u, 0u, 0u));
+            fence_proxy_async();  // the bulk copies (async proxy) read these rows
         }
     }
 
@@ -511,39 +522,39 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     if (S > 1) {
         // ---- merge the KV splits of this row tile through the cluster's shared memory.
-        // Rows [k R, k R + R) belong to CTA k (split k); each CTA receives, in its idle
-        // K ring, S partial rows (one per split) for each row it owns, laid out
-        // [split][row - k R] with PROW_BYTES per row: 128 bf16 outputs, then the fp32
-        // log-sum-exp.
+        // Rows [k R, k R + R) belong to CTA k (split k).  Each CTA has staged its 128
+        // partial rows in its V ring; once every CTA's K ring is idle, each sends CTA k
+        // its rows [k R, k R + own_k) with one bulk copy into k's K ring, laid out
+        // [split][row - k R] with PROW_BYTES per row, completing on k's merge barrier.
         const int R = (TM + S - 1) / S;
         const int own = max(0, min(TM, (split + 1) * R) - split * R);
-        const uint32_t recv = base + SK_OFF;
+        const uint32_t recv = base + SK_OFF, stage = base + SV_OFF;
         // every CTA of the cluster has initialised its barriers
         asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
         if (tid == 0) {
-            mbar_expect_tx(merge_bar, (uint32_t)(own * S) * PUSH_BYTES);
-            // this CTA's ring is free: tell every CTA of the cluster it may push
+            mbar_expect_tx(merge_bar, (uint32_t)(own * S * PROW_BYTES));
+            // this CTA's K ring is idle: every CTA of the cluster may send to it
             for (int k = 0; k < S; ++k) mbar_arrive_cluster(mapa_shared(free_bar, (uint32_t)k));
-        }
-        if (warp >= 4) {
-            // push once every CTA can receive (NaN rows if this CTA failed: the owners
-            // still get every byte they wait for)
-            if (__all_sync(0xffffffffu, mbar_wait_cluster_bounded(free_bar, 0))) {
-                const int owner = r / R, slot = r % R;
-                const uint32_t row = recv + (uint32_t)((split * R + slot) * PROW_BYTES);
-                const uint32_t dst = mapa_shared(row + X * HD, (uint32_t)owner);
-                const uint32_t mb = mapa_shared(merge_bar, (uint32_t)owner);
-#pragma unroll
-                for (int q8 = 0; q8 < 8; ++q8)
-                    st_async_v4(dst + q8 * 16, pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3], mb);
-                if (X == 0) st_async_b32(mapa_shared(row + 2 * HD, (uint32_t)owner), __float_as_uint(lse), mb);
-            } else if (lane == 0) {
+            if (mbar_wait_cluster_bounded(free_bar, 0)) {
+                // NaN rows when this CTA failed: the owners still get every byte they wait for
+                for (int k = 0; k < S; ++k) {
+                    const int own_k = max(0, min(TM, (k + 1) * R) - k * R);
+                    if (own_k > 0)
+                        bulk_copy_cluster(mapa_shared(recv + (uint32_t)(split * R * PROW_BYTES), (uint32_t)k),
+                                          stage + (uint32_t)(k * R * PROW_BYTES), (uint32_t)(own_k * PROW_BYTES),
+                                          mapa_shared(merge_bar, (uint32_t)k));
+                }
+            } else {
                 *abort_flag = 1;
             }
+            // every partial row of this CTA's share has arrived (always waited for, bounded)
+            s_got = mbar_wait_cluster_bounded(merge_bar, 0) ? 1 : 0;
         }
-        // every partial row of this CTA's share has arrived (always waited for, bounded:
-        // no peer may still write to this CTA's shared memory when it retires)
-        if (tid == 0) s_got = mbar_wait_cluster_bounded(merge_bar, 0) ? 1 : 0;
+        __syncthreads();
+        // this CTA has received everything sent to it, so every copy it is the target of
+        // is complete; once all CTAs have arrived here, no copy still reads any CTA's
+        // staged rows (the wait is at the end, after the local merge)
+        asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
         __syncthreads();
         const uint8_t* part = base_ptr + SK_OFF;
         if (!s_got) {
@@ -577,6 +588,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 default: merge_rows<TM, TC_THREADS, 16>(a, part, R, split, tile, b, kvh, tid, G * n); break;
             }
         }
+        asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
     }
     if (tid == 0) {
         if (s_bad) report(a.status, s_bad);

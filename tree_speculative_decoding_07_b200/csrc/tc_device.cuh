@@ -272,18 +272,13 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t
         if (clock64() - t0 > WAIT_LIMIT) return false;
     }
 }
-// 16 / 4 bytes into the shared memory of a CTA of the cluster, completing that
-// many transaction bytes on the receiver's mbarrier
-__device__ __forceinline__ void st_async_v4(uint32_t remote, uint32_t x, uint32_t y, uint32_t z, uint32_t w,
-                                            uint32_t remote_bar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                     remote),
-                 "r"(x), "r"(y), "r"(z), "r"(w), "r"(remote_bar)
-                 : "memory");
-}
-__device__ __forceinline__ void st_async_b32(uint32_t remote, uint32_t x, uint32_t remote_bar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote), "r"(x),
-                 "r"(remote_bar)
+// bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory into the
+// shared memory of a CTA of the cluster, completing on that CTA's mbarrier
+__device__ __forceinline__ void bulk_copy_cluster(uint32_t remote_dst, uint32_t local_src, uint32_t bytes,
+                                                  uint32_t remote_bar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     remote_dst),
+                 "r"(local_src), "r"(bytes), "r"(remote_bar)
                  : "memory");
 }
 
