@@ -216,13 +216,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             __syncwarp();
             if (lane == 0) {
                 // blocks of the tile that hold tokens of the split (the last tile may
-                // hold fewer than 8); rows of the others are masked and never loaded
+                // hold fewer than 8); the others repeat its last block, whose rows past the
+                // split are masked (K) and zeroed (V) like any rows past the split (a copy
+                // of all 8 blocks with a constant byte count measured faster than
+                // issuing only the ones in range)
                 const int nb = min(BLK_PER_TILE, used_blk - (blk0 + j * BLK_PER_TILE));
                 int cur[BLK_PER_TILE];
                 const int32_t* ring = &s_ids[prod][(j % ID_RING) * BLK_PER_TILE];
 #pragma unroll
                 for (int k = 0; k < BLK_PER_TILE; ++k) {
-                    int id = k < nb ? ring[k] : 0;
+                    int id = ring[k < nb ? k : nb - 1];
                     if (id < 0 || id >= a.num_blocks) {
                         bad_id = true;
                         id = 0;
@@ -231,13 +234,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 }
                 const uint32_t full = is_k ? k_full(s) : v_full(s);
                 const uint32_t dst = is_k ? sK(s) : sV(s);
-                mbar_expect_tx(full, (uint32_t)nb * (TILE_BYTES / BLK_PER_TILE));
+                mbar_expect_tx(full, TILE_BYTES);
 #pragma unroll
                 for (int k = 0; k < BLK_PER_TILE; ++k)
-                    if (k < nb)
 #pragma unroll
-                        for (int h = 0; h < 2; ++h)
-                            tma_load_4d(dst + h * HALF_BYTES + k * 2048u, map, full, 0, kvh * 2 + h, 0, cur[k]);
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_4d(dst + h * HALF_BYTES + k * 2048u, map, full, 0, kvh * 2 + h, 0, cur[k]);
             }
             __syncwarp();
             // the slot refilled here last held tile j + ID_AHEAD - ID_RING, read before
@@ -424,8 +426,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
             l_run = l_run * f + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
             if (lim < TN) {
-                // value rows past the split end are not loaded (or hold another
-                // sequence's data): clear this group's ones
+                // value rows past the split end repeat another block or hold data
+                // past the sequence: clear this group's ones
                 const int tok = X * HALF_N + (r & 63);
                 if (tok >= lim) {
                     const int vs = j % VST;
@@ -551,10 +553,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             s_got = mbar_wait_cluster_bounded(merge_bar, 0) ? 1 : 0;
         }
         __syncthreads();
-        // this CTA has received everything sent to it, so every copy it is the target of
-        // is complete; once all CTAs have arrived here, no copy still reads any CTA's
-        // staged rows (the wait is at the end, after the local merge)
-        asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+        // this CTA has received everything sent to it (its merge barrier saw every copy
+        // complete), so once all CTAs have arrived here no copy still reads any CTA's
+        // staged rows; the arrival orders no memory of its own (relaxed) and the wait
+        // is at the end, after the local merge
+        asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
         __syncthreads();
         const uint8_t* part = base_ptr + SK_OFF;
         if (!s_got) {
