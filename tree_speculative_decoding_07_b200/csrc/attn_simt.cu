@@ -11,7 +11,10 @@
 // node-major, so the G query heads sharing a KV head read each K/V row once.
 // Tokens are streamed in chunks of 32 through shared memory, one token per
 // lane; each warp owns 8 query rows and keeps an online softmax (running max
-// and sum in the log2 domain) plus D/32 output columns per lane.
+// and sum in the log2 domain) plus D/32 output columns per lane.  A chunk is
+// loaded in 4-element pieces, every thread issuing all of its loads before it
+// stores any; the warp's 8 rows are computed together (8 independent dot
+// products per token, 8 x D/32 independent accumulations per value row).
 #include "tv_common.cuh"
 #include "kernels.h"
 
@@ -34,7 +37,26 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-template <typename T, int D>
+// four consecutive elements as fp32: one 16-byte (fp32) or 8-byte (bf16) load when
+// VEC, else four scalar loads
+template <typename T, bool VEC> struct Load4;
+template <> struct Load4<float, true> {
+    static __device__ __forceinline__ float4 get(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+};
+template <> struct Load4<__nv_bfloat16, true> {
+    static __device__ __forceinline__ float4 get(const __nv_bfloat16* p) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+        return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y << 16),
+                           __uint_as_float(u.y & 0xFFFF0000u));
+    }
+};
+template <typename T> struct Load4<T, false> {
+    static __device__ __forceinline__ float4 get(const T* p) {
+        return make_float4(Elem<T>::load(p), Elem<T>::load(p + 1), Elem<T>::load(p + 2), Elem<T>::load(p + 3));
+    }
+};
+
+template <typename T, int D, bool VEC>
 __global__ void __launch_bounds__(SIMT_WARPS * 32) attn_simt_kernel(AttnArgs a) {
     constexpr int DPL = D / 32;
     extern __shared__ float simt_smem[];
@@ -103,55 +125,84 @@ __global__ void __launch_bounds__(SIMT_WARPS * 32) attn_simt_kernel(AttnArgs a) 
         for (int dd = 0; dd < DPL; ++dd) acc[rr][dd] = 0.f;
     }
 
+    constexpr int PER = CHUNK * D / 4 / (SIMT_WARPS * 32);  // 4-element pieces per thread and chunk
     for (int c0 = t0; c0 < t1; c0 += CHUNK) {
         __syncthreads();  // previous chunk fully consumed (and Qs/anc written on entry)
-        for (int e = tid; e < CHUNK * D; e += blockDim.x) {
-            const int t = e / D, d = e % D, pos = c0 + t;
-            float kv = 0.f, vv = 0.f;
-            if (pos < t1) {
-                const int blk = a.block_table[(size_t)b * a.max_blocks + pos / TV_BLOCK];
-                if (blk < 0 || blk >= a.num_blocks) {
-                    s_bad = TV_ERR_BLOCK_TABLE;
-                } else {
-                    const size_t off = (((size_t)blk * TV_BLOCK + pos % TV_BLOCK) * a.Hkv + kvh) * D + d;
-                    kv = Elem<T>::load(kg + off);
-                    vv = Elem<T>::load(vg + off);
+        {
+            float4 kq[PER], vq[PER];
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int e = tid + i * SIMT_WARPS * 32;
+                const int t = e / (D / 4), d = (e % (D / 4)) * 4, pos = c0 + t;
+                kq[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                vq[i] = kq[i];
+                if (pos < t1) {
+                    const int blk = a.block_table[(size_t)b * a.max_blocks + pos / TV_BLOCK];
+                    if (blk < 0 || blk >= a.num_blocks) {
+                        s_bad = TV_ERR_BLOCK_TABLE;
+                    } else {
+                        const size_t off = (((size_t)blk * TV_BLOCK + pos % TV_BLOCK) * a.Hkv + kvh) * D + d;
+                        kq[i] = Load4<T, VEC>::get(kg + off);
+                        vq[i] = Load4<T, VEC>::get(vg + off);
+                    }
                 }
             }
-            Ks[t][d] = kv;
-            Vs[t][d] = vv;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int e = tid + i * SIMT_WARPS * 32;
+                const int t = e / (D / 4), d = (e % (D / 4)) * 4;
+                Ks[t][d] = kq[i].x;
+                Ks[t][d + 1] = kq[i].y;
+                Ks[t][d + 2] = kq[i].z;
+                Ks[t][d + 3] = kq[i].w;
+                *reinterpret_cast<float4*>(&Vs[t][d]) = vq[i];
+            }
         }
         __syncthreads();
         const int pos = c0 + lane;
         const bool in_range = pos < t1;
+        // scores of the warp's 8 rows for this lane's token
+        float sc[SIMT_RPW];
+#pragma unroll
+        for (int rr = 0; rr < SIMT_RPW; ++rr) sc[rr] = 0.f;
+#pragma unroll 8
+        for (int d = 0; d < D; ++d) {
+            const float kd = Ks[lane][d];
+#pragma unroll
+            for (int rr = 0; rr < SIMT_RPW; ++rr) sc[rr] = fmaf(Qs[warp * SIMT_RPW + rr][d], kd, sc[rr]);
+        }
+        float pr[SIMT_RPW];
 #pragma unroll
         for (int rr = 0; rr < SIMT_RPW; ++rr) {
-            const int r = warp * SIMT_RPW + rr, gr = r0 + r;
-            if (gr >= rows_total) break;  // warp-uniform
-            const int node = gr / G;
-            float s = 0.f;
-#pragma unroll 16
-            for (int d = 0; d < D; ++d) s = fmaf(Qs[r][d], Ks[lane][d], s);
-            bool ok = in_range;
+            const int gr = r0 + warp * SIMT_RPW + rr;
+            const bool row = gr < rows_total;  // warp-uniform
+            bool ok = in_range && row;
             if (ok && pos >= L) {
                 const int j = pos - L;
-                ok = (anc[node][j >> 5] >> (j & 31)) & 1u;
+                ok = (anc[gr / G][j >> 5] >> (j & 31)) & 1u;
             }
-            s = ok ? s : -INFINITY;
-            const float m_new = fmaxf(m_run[rr], warp_max(s));
-            if (m_new == -INFINITY) continue;  // nothing visible yet for this row
-            const float pr = ok ? exp2f(s - m_new) : 0.f;
-            const float corr = exp2f(m_run[rr] - m_new);
-            l_run[rr] = l_run[rr] * corr + warp_sum(pr);
+            const float sv = ok ? sc[rr] : -INFINITY;
+            const float m_new = fmaxf(m_run[rr], warp_max(sv));
+            // nothing visible yet for this row: its state stays as it was
+            const bool live = m_new != -INFINITY;
+            pr[rr] = (ok && live) ? exp2f(sv - m_new) : 0.f;
+            const float corr = live ? exp2f(m_run[rr] - m_new) : 1.f;
+            l_run[rr] = live ? l_run[rr] * corr + warp_sum(pr[rr]) : l_run[rr];
 #pragma unroll
             for (int dd = 0; dd < DPL; ++dd) acc[rr][dd] *= corr;
-#pragma unroll 8
-            for (int t = 0; t < CHUNK; ++t) {
-                const float pt = __shfl_sync(0xffffffffu, pr, t);
+            m_run[rr] = live ? m_new : m_run[rr];
+        }
+#pragma unroll 4
+        for (int t = 0; t < CHUNK; ++t) {
+            float vt[DPL];
 #pragma unroll
-                for (int dd = 0; dd < DPL; ++dd) acc[rr][dd] = fmaf(pt, Vs[t][lane + 32 * dd], acc[rr][dd]);
+            for (int dd = 0; dd < DPL; ++dd) vt[dd] = Vs[t][lane + 32 * dd];
+#pragma unroll
+            for (int rr = 0; rr < SIMT_RPW; ++rr) {
+                const float pt = __shfl_sync(0xffffffffu, pr[rr], t);
+#pragma unroll
+                for (int dd = 0; dd < DPL; ++dd) acc[rr][dd] = fmaf(pt, vt[dd], acc[rr][dd]);
             }
-            m_run[rr] = m_new;
         }
     }
     __syncthreads();
@@ -215,15 +266,21 @@ constexpr size_t simt_smem_bytes(int D) {
     return sizeof(float) * ((size_t)SIMT_ROWS * D + (size_t)CHUNK * (D + 1) + (size_t)CHUNK * D);
 }
 
-template <typename T, int D>
-cudaError_t launch_dim(const AttnArgs& a, cudaStream_t st) {
-    static cudaError_t attr = cudaFuncSetAttribute(attn_simt_kernel<T, D>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)simt_smem_bytes(D));
+template <typename T, int D, bool VEC>
+cudaError_t launch_vec(const AttnArgs& a, cudaStream_t st) {
+    cudaError_t attr = cudaFuncSetAttribute(attn_simt_kernel<T, D, VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)simt_smem_bytes(D));
     if (attr != cudaSuccess) return attr;
     dim3 grid(a.splits, a.row_tiles, a.B * a.Hkv);
-    attn_simt_kernel<T, D><<<grid, SIMT_WARPS * 32, simt_smem_bytes(D), st>>>(a);
+    attn_simt_kernel<T, D, VEC><<<grid, SIMT_WARPS * 32, simt_smem_bytes(D), st>>>(a);
     return cudaGetLastError();
+}
+
+// vector loads need the caches aligned to 4 elements (16 bytes fp32, 8 bytes bf16)
+template <typename T, int D>
+cudaError_t launch_dim(const AttnArgs& a, cudaStream_t st) {
+    const uintptr_t m = reinterpret_cast<uintptr_t>(a.k) | reinterpret_cast<uintptr_t>(a.v);
+    return (m % (4 * sizeof(T))) == 0 ? launch_vec<T, D, true>(a, st) : launch_vec<T, D, false>(a, st);
 }
 
 template <typename T>

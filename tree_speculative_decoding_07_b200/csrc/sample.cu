@@ -78,8 +78,11 @@ struct SampleShared {
     unsigned long long exit_bar;
     int timeout;
     int found;
+    int found_t;
     int wsel;
     double wbefore;
+    double wofs[MAX_THREADS / 32];  // bonus scan: exclusive prefix of the warps' totals
+    float u0;                       // the bonus draw's uniform, read at launch
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -429,6 +432,7 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(const __grid
         sh.token[i] = a.tokens[(size_t)b * N + i];
         if (a.gather) g_first[i] = nn;
     }
+    if (tid == 0) sh.u0 = __ldg(a.uniforms + (size_t)b * N);
     // every CTA's barriers must exist before a peer pushes to them (the first pass);
     // the cluster barrier sits here so the loads above are already in flight
     if (C > 1)
@@ -590,7 +594,7 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(const __grid
             total = w.cluster_pass(x, cur_c);
         }
         const int par = (w.passes - 1) & 1;
-        const double target = (double)__ldg(a.uniforms + (size_t)b * N) * total;
+        const double target = (double)sh.u0 * total;
         int owner = -1, last_pos_cta = -1;
         double before = 0.0, run = 0.0;
         for (int k = 0; k < C; ++k) {
@@ -628,47 +632,54 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(const __grid
                 sh.wsel = wsel >= 0 ? wsel : wlast;
                 sh.wbefore = wsel >= 0 ? rb : -INFINITY;  // -inf: take the segment's last positive element
                 sh.found = -1;
+                sh.found_t = INT_MAX;
             }
             __syncthreads();
-            if (warp == sh.wsel) {
-                const int s0 = min(n, warp * w.segw), s1 = min(n, s0 + w.segw);
-                const int per = (s1 - s0 + 31) / 32;
-                const int e0 = min(s1, s0 + lane * per), e1 = min(s1, e0 + per);
-                double mine = 0.0;
-                int mylast = -1;
+            // the whole CTA scans the selected segment: each thread a run of at most a
+            // few elements, then an inclusive scan over the threads (lanes, then warps)
+            const int s0 = sh.wsel < 0 ? n : min(n, sh.wsel * w.segw), s1 = min(n, s0 + w.segw);
+            const int per = (s1 - s0 + (int)blockDim.x - 1) / (int)blockDim.x;
+            const int e0 = min(s1, s0 + tid * per), e1 = min(s1, e0 + per);
+            double mine = 0.0;
+            int mylast = -1;
+            for (int i = e0; i < e1; ++i) {
+                const double v = resid(pr[i], qr[i], cur_c);
+                mine += v;
+                if (v > 0.0) mylast = i;
+            }
+            double incl = mine;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const double t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            if (lane == 31) sh.warp_part2[warp] = incl;
+            __syncthreads();
+            if (tid == 0) {
+                double acc = 0.0;
+                for (int k = 0; k < nwarps; ++k) {
+                    sh.wofs[k] = acc;
+                    acc += sh.warp_part2[k];
+                }
+            }
+            __syncthreads();
+            incl += sh.wofs[warp];
+            const bool take_last = sh.wbefore == -INFINITY;
+            // the first thread whose inclusive running sum exceeds the target holds the draw
+            if (!take_last && sh.wbefore + incl > target) atomicMin(&sh.found_t, tid);
+            if (mylast >= 0) atomicMax(&sh.found, mylast);  // the segment's last positive element
+            __syncthreads();
+            const int ft = sh.found_t;
+            if (ft != INT_MAX && tid == ft) {
+                double rsum = sh.wbefore + incl - mine;
+                int pick = -1;
                 for (int i = e0; i < e1; ++i) {
                     const double v = resid(pr[i], qr[i], cur_c);
-                    mine += v;
-                    if (v > 0.0) mylast = i;
+                    if (v > 0.0) pick = i;
+                    rsum += v;
+                    if (rsum > target && v > 0.0) break;
                 }
-                double incl = mine;  // inclusive scan over the lanes
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const double t = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += t;
-                }
-                const bool take_last = sh.wbefore == -INFINITY;
-                const unsigned hit = take_last ? 0u : __ballot_sync(0xffffffffu, sh.wbefore + incl > target);
-                const unsigned pos = __ballot_sync(0xffffffffu, mylast >= 0);
-                int pick = -1;
-                if (hit) {
-                    const int hl = __ffs(hit) - 1;
-                    if (lane == hl) {
-                        double rsum = sh.wbefore + incl - mine;
-                        for (int i = e0; i < e1; ++i) {
-                            const double v = resid(pr[i], qr[i], cur_c);
-                            if (v > 0.0) pick = i;
-                            rsum += v;
-                            if (rsum > target && v > 0.0) break;
-                        }
-                    }
-                    pick = __shfl_sync(0xffffffffu, pick, hl);
-                } else if (pos) {
-                    // rounding left no crossing: the segment's last positive element
-                    const int ll = 31 - __clz(pos);
-                    pick = __shfl_sync(0xffffffffu, mylast, ll);
-                }
-                if (lane == 0) sh.found = pick;
+                sh.found = pick;
             }
             __syncthreads();
             if (tid == 0) {
