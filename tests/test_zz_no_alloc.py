@@ -40,8 +40,8 @@ def test_static_scratch_matches_workspace_path():
     cases = [
         # the Llama-3-8B shape (bf16, tensor cores, several KV splits)
         _case(Attn.from_workload(synth.make("l8b", need_tokens=False))),
-        # fp32 on the CUDA cores: 11 KV splits merged through scratch memory
-        _case(random_attn(71, 1, 16, 8, 2, 128, [3000], dtype="f32")),
+        # fp32 on the CUDA cores: 10 KV splits merged through scratch memory
+        _case(random_attn(71, 1, 16, 8, 2, 128, [600], dtype="f32")),
         # bf16, head_dim 64 (CUDA cores), another split count and batch
         _case(random_attn(72, 3, 9, 16, 4, 64, [700, 2100, 64], dtype="bf16")),
     ]
@@ -68,6 +68,6 @@ def test_static_scratch_refuses_oversize_problems():
     p = buf.data_ptr()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     assert tv.tv_tree_attention_static(d, p, p, p, p, p, p, p, status) == tv.TV_ERR_WORKSPACE
-    a = random_attn(73, 1, 16, 8, 2, 128, [3000], dtype="f32")
+    a = random_attn(73, 1, 16, 8, 2, 128, [600], dtype="f32")
     a, desc, plan, ref = _case(a)
     assert torch.equal(_static(a, desc, status), ref)

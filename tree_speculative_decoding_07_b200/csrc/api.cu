@@ -43,7 +43,8 @@ tv_status check_attn_desc(const tv_attn_desc* d) {
 //  - everything else runs on the CUDA cores: 32-row tiles, splits merged by
 //    a second kernel through a global workspace.
 // Splits are chosen so the main launch covers the SMs about once, and never
-// below 256 tokens per split.
+// below 256 tokens per split on the tensor cores (64 on the CUDA cores, whose
+// tiles stream 32 tokens at a time).
 void make_plan(const tv_attn_desc* d, tv_attn_plan* p) {
     const int G = d->num_q_heads / d->num_kv_heads;
     const int rows = G * d->num_nodes;
@@ -59,7 +60,7 @@ void make_plan(const tv_attn_desc* d, tv_attn_plan* p) {
         splits = tv::tc_pick_splits(base, d->max_blocks_per_seq, sms);
     } else {
         splits = base >= sms ? 1 : (sms / base);
-        const int64_t by_len = (max_tokens + 255) / 256;
+        const int64_t by_len = (max_tokens + 63) / 64;  // at least two 32-token chunks per split
         if (splits > by_len) splits = by_len;
         if (splits < 1) splits = 1;
         if (splits > 64) splits = 64;
