@@ -145,6 +145,15 @@ __device__ __forceinline__ void st_async_f64(uint32_t remote_addr, double v, uin
                  "l"(__double_as_longlong(v)), "r"(remote_bar)
                  : "memory");
 }
+// bring [src, src + bytes) into L2 (16-byte aligned, a multiple of 16 bytes); no data
+// reaches the CTA, so it may run before the previous kernel has finished
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void prefetch_line_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)) : "memory");
+}
 // bulk copy global -> this CTA's shared memory, completing on a local mbarrier
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -412,6 +421,23 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(const __grid
         }
         mbar_init(smem_u32(&sh.exit_bar), (uint32_t)C);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    // Launched with a programmatic dependency, the kernel may start while the previous
+    // kernel still runs: warm L2 (and the address translations) for what the walk
+    // reads first -- this CTA's slice of the root's p and q rows, and the sequence's
+    // tree, tokens and uniforms.  Only prefetches happen before the wait below: the
+    // data is read after it, so a write by the previous kernel is still seen.
+    if (tid == 0 && a.vec4 && n > 0) {
+        const size_t row = (size_t)b * N * (size_t)a.V + lo;  // node 0's row
+        bulk_prefetch_l2(a.p + row, (uint32_t)(4 * n));
+        bulk_prefetch_l2(a.q + row, (uint32_t)(4 * n));
+    }
+    if (rank == 0 && tid < 96) {
+        const int arr = tid / 32, line = tid % 32;  // parents, tokens, uniforms: 32 lines of 128 B each
+        const char* base = arr == 0 ? reinterpret_cast<const char*>(a.parent)
+                                    : arr == 1 ? reinterpret_cast<const char*>(a.tokens)
+                                               : reinterpret_cast<const char*>(a.uniforms);
+        if (base && 128 * line < 4 * N) prefetch_line_l2(base + 4 * (size_t)b * N + 128 * line);
     }
     __syncthreads();
     // the kernel may have been launched while the previous one on the stream was still
