@@ -24,21 +24,27 @@
 //               reach them through a shared-memory ring filled by cp.async
 //               several tiles ahead.
 //   warp 1      S = Q K^T issuer: tcgen05.mma kind::f16, M 128, N 128, 8 x K16,
-//               into one of two TMEM S buffers.
+//               into the TMEM S buffer, reused as soon as both softmax groups
+//               have read the previous tile's scores into registers.
 //   warp 2      O_x += P_x V issuer (one per softmax group, over that group's 64
 //               tokens), and owner of the TMEM allocation (all 512 columns:
-//               S0, S1, O_A, O_B).  The two issuers sit on different SM
-//               sub-partitions; S buffer j % 2 is reused once P V of tile j - 2,
-//               which reads P from it, has finished.
+//               S, two P buffers, O_A, O_B).  The two issuers sit on different SM
+//               sub-partitions.
 //   warps 4-7   softmax group A: columns 0..63 of every S tile
 //   warps 8-11  softmax group B: columns 64..127
 // Each softmax thread owns one query row (its TMEM lane).  The two groups
-// keep separate running maxima / sums and separate O accumulators, so they
-// never wait on each other inside the loop; their halves are merged at the
-// end.  Scores are scaled into the log2 domain by the same FFMA that
+// keep separate running maxima / sums and separate O accumulators, merged at
+// the end like two splits.  Every SM sub-partition holds one warp of each
+// group, and the two take turns at the exponentials of a tile (two named
+// barriers pass the turn): while one warp's exponentials occupy the
+// sub-partition's MUFU unit, the other reads its next scores from TMEM and
+// reduces their maximum, so the unit is not left idle while both wait for
+// scores in step.  Scores are scaled into the log2 domain by the same FFMA that
 // subtracts the running max; the O rescale in TMEM is skipped while the max
-// grows by at most 2^8.  P is written as bf16 pairs into TMEM over the scores
-// just read, and P V takes it from there (the TMEM-A form of the MMA).  The
+// grows by at most 2^8.  P is written as bf16 pairs into a TMEM P buffer of its
+// own (tile j into buffer j % 2), and P V takes it from there (the TMEM-A form
+// of the MMA); since P does not overwrite the scores, S = Q K^T of tile j + 1
+// runs while the softmax of tile j is still computing.  The
 // tree mask is a 128-bit ancestor set per node (anc(i) = anc(parent(i)) |
 // {i}), shifted into column space once per tile; prefix-only tiles skip it.
 //
@@ -61,25 +67,29 @@ constexpr uint32_t SQ_OFF = 0;             // Q: 2 x [128 rows][128 B], swizzled
 constexpr uint32_t SK_OFF = 32768;         // K ring: KST x 32 KB
 constexpr uint32_t SV_OFF = SK_OFF + KST * 32768u;  // V ring: VST x 32 KB
 constexpr uint32_t SMEM_BYTES = SV_OFF + VST * 32768u + 1024;
-constexpr uint32_t TMEM_COLS = 512;        // S0 [0,128), S1 [128,256), O_A [256,384), O_B [384,512)
+constexpr uint32_t TMEM_COLS = 512;        // S [0,128), P0 [128,192), P1 [192,256), O_A [256,384), O_B [384,512)
+constexpr uint32_t P_COL = 128;            // P buffer j % 2: 64 columns of bf16 pairs, group x at x * 32
 constexpr uint32_t O_COL = 256;
+// named barriers passing the turn at the exponentials: group A waits on BAR_TURN_A
+// (B arrives), group B on BAR_TURN_B (A arrives); 0 is __syncthreads, 1 the epilogue's
+constexpr int BAR_TURN_A = 2, BAR_TURN_B = 3;
 
 // mbarrier slots, derived from the ring depths
 constexpr int BAR_K_FULL = 0;                    // KST: K tile landed (TMA transaction count)
 constexpr int BAR_K_EMPTY = BAR_K_FULL + KST;    // KST: S = Q K^T done with the K slot
 constexpr int BAR_V_FULL = BAR_K_EMPTY + KST;    // VST: V tile landed
 constexpr int BAR_V_EMPTY = BAR_V_FULL + VST;    // VST: P V done with the V slot
-constexpr int BAR_S_FULL = BAR_V_EMPTY + VST;    // 2: S buffer written
-constexpr int BAR_P_FULL = BAR_S_FULL + 2;       // 2: group's P written (and O rescaled)
+constexpr int BAR_S_FULL = BAR_V_EMPTY + VST;    // S of the next tile written
+constexpr int BAR_S_FREE = BAR_S_FULL + 1;       // both groups have read S (256 arrivals)
+constexpr int BAR_P_FULL = BAR_S_FREE + 1;       // 2: group's P written (and O rescaled)
 constexpr int BAR_O_DONE = BAR_P_FULL + 2;       // 2: group's P V done
-constexpr int BAR_PV_DONE = BAR_O_DONE + 2;      // 2: P V of the tile in an S buffer done (buffer free)
-constexpr int BAR_Q_READY = BAR_PV_DONE + 2;     // Q staged
+constexpr int BAR_Q_READY = BAR_O_DONE + 2;      // Q staged
 constexpr int BAR_DRAIN_QK = BAR_Q_READY + 1;    // all S = Q K^T MMAs done
 constexpr int BAR_DRAIN_PV = BAR_DRAIN_QK + 1;   // all P V MMAs done
 constexpr int BAR_FREE = BAR_DRAIN_PV + 1;       // S arrivals: every CTA of the cluster can receive partials
 constexpr int BAR_MERGE = BAR_FREE + 1;          // this CTA's share of partial rows received (transaction count)
 constexpr int BAR_COUNT = BAR_MERGE + 1;
-static_assert(BAR_COUNT == 2 * KST + 2 * VST + 13, "barrier slots overlap");
+static_assert(BAR_COUNT == 2 * KST + 2 * VST + 11, "barrier slots overlap");
 static_assert(TM * PROW_BYTES <= VST * TILE_BYTES, "staged partial rows exceed the V ring");
 static_assert((TM + MAX_SPLITS) * PROW_BYTES <= KST * TILE_BYTES, "received partial rows exceed the K ring");
 
@@ -116,10 +126,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     auto k_empty = [&](int s) { return bar0 + 8u * (BAR_K_EMPTY + s); };
     auto v_full = [&](int s) { return bar0 + 8u * (BAR_V_FULL + s); };
     auto v_empty = [&](int s) { return bar0 + 8u * (BAR_V_EMPTY + s); };
-    auto s_full = [&](int s) { return bar0 + 8u * (BAR_S_FULL + s); };
+    const uint32_t s_full = bar0 + 8u * BAR_S_FULL, s_free = bar0 + 8u * BAR_S_FREE;
     auto p_full = [&](int x) { return bar0 + 8u * (BAR_P_FULL + x); };
     auto o_done = [&](int x) { return bar0 + 8u * (BAR_O_DONE + x); };
-    auto pv_done = [&](int sb) { return bar0 + 8u * (BAR_PV_DONE + sb); };
     const uint32_t q_ready = bar0 + 8u * BAR_Q_READY;
     const uint32_t drain_qk = bar0 + 8u * BAR_DRAIN_QK, drain_pv = bar0 + 8u * BAR_DRAIN_PV;
     const uint32_t free_bar = bar0 + 8u * BAR_FREE, merge_bar = bar0 + 8u * BAR_MERGE;
@@ -143,11 +152,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             mbar_init(v_full(s), 1);
             mbar_init(v_empty(s), 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(s_full(s), 1);
-            mbar_init(p_full(s), 128);
-            mbar_init(o_done(s), 1);
-            mbar_init(pv_done(s), 1);
+        mbar_init(s_full, 1);
+        mbar_init(s_free, 256);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(p_full(x), 128);
+            mbar_init(o_done(x), 1);
         }
         mbar_init(q_ready, 256);
         mbar_init(drain_qk, 1);
@@ -274,11 +283,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const uint64_t dq = sdesc(sQ, 16, 1024);
             const uint64_t dk0 = sdesc(sK(0), 16, 1024);
             for (int j = 0; ok && j < ntiles; ++j) {
-                const int ks = j % KST, sb = j & 1;
-                // S buffer j % 2 holds P of tile j - 2 until that tile's P V has finished;
-                // the buffer's barrier cannot run two phases ahead of this wait, because
-                // P V of tile j needs the S tile issued here
-                if (j >= 2) ok = mbar_wait(pv_done(sb), ((j - 2) >> 1) & 1, abort_flag);
+                const int ks = j % KST;
+                // the S buffer is free once both groups have read tile j - 1's scores (they
+                // cannot read tile j's before this commit, so the phases stay in step)
+                if (j >= 1) ok = mbar_wait(s_free, (j - 1) & 1, abort_flag);
                 if (ok) ok = mbar_wait(k_full(ks), (j / KST) & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
@@ -286,9 +294,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k) {
                     const uint32_t off = ((k >> 2) * HALF_BYTES + (k & 3) * 32u) >> 4;
-                    mma_bf16(tmem + sb * TN, dq + off, dk + off, IDESC_QK, k > 0 ? 1u : 0u);
+                    mma_bf16(tmem, dq + off, dk + off, IDESC_QK, k > 0 ? 1u : 0u);
                 }
-                mma_commit(s_full(sb));
+                mma_commit(s_full);
                 mma_commit(k_empty(ks));
                 issued_any = true;
             }
@@ -316,14 +324,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < HALF_N / 16; ++k)
-                        mma_bf16_ts(tmem + O_COL + x * HD, tmem + (t & 1) * TN + x * HALF_N + k * 8,
+                        mma_bf16_ts(tmem + O_COL + x * HD, tmem + P_COL + (t & 1) * 64 + x * 32 + k * 8,
                                     dv + (uint64_t)(((x * 4 + k) * 2048u) >> 4), IDESC_PV, (t > 0 || k > 0) ? 1u : 0u);
                     mma_commit(o_done(x));
                     issued_any = true;
                 }
                 if (!ok) break;
                 mma_commit(v_empty(vs));
-                mma_commit(pv_done(t & 1));
             }
             if (issued_any) {
                 mma_commit(drain_pv);
@@ -376,21 +383,51 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         float m_run = -INFINITY, l_run = 0.f;  // running max in the scaled log2 domain, running sum
         const float sl = a.scale_log2;
+        // The turn protocol: group A's exponentials of tile j follow group B's of tile
+        // j - 1, and B's of tile j follow A's of tile j.  A waits on BAR_TURN_A once per
+        // tile and B arrives there once per tile (before its loop for tile 0, after its
+        // exponentials of tile j for tile j + 1, never after the last tile); B waits on
+        // BAR_TURN_B once per tile and A arrives there once per tile.  Named barriers
+        // have no time limit, so the loop never leaves early: after a failed wait a warp
+        // only keeps passing the turn (`live` is false, and the abort flag makes every
+        // later mbarrier wait return at once), and both groups run all ntiles
+        // iterations.  The waits alternate strictly, so no barrier receives a second
+        // phase's arrivals before its current phase completes.
+        auto turn_wait = [&]() {
+            if (X == 0)
+                asm volatile("bar.sync %0, 256;" ::"n"(BAR_TURN_A) : "memory");
+            else
+                asm volatile("bar.sync %0, 256;" ::"n"(BAR_TURN_B) : "memory");
+        };
+        auto turn_pass = [&](int j) {
+            if (X == 0)
+                asm volatile("bar.arrive %0, 256;" ::"n"(BAR_TURN_B) : "memory");
+            else if (j + 1 < ntiles)
+                asm volatile("bar.arrive %0, 256;" ::"n"(BAR_TURN_A) : "memory");
+        };
+        if (X == 1 && ntiles > 0) asm volatile("bar.arrive %0, 256;" ::"n"(BAR_TURN_A) : "memory");
+        bool live = true;  // warp-uniform: every wait of this warp so far succeeded
         for (int j = 0; j < ntiles; ++j) {
-            const int sb = j & 1;
-            if (!warp_wait(s_full(sb), (j >> 1) & 1, abort_flag)) break;
-            tc_fence_after();
+            live = live && warp_wait(s_full, j & 1, abort_flag);
             float x[HALF_N];
-#pragma unroll
-            for (int c32 = 0; c32 < HALF_N / 32; ++c32) {
-                uint32_t rr[32];
-                tmem_ld_x32(tmem + lane_base + sb * TN + X * HALF_N + c32 * 32, rr);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[c32 * 32 + i] = __uint_as_float(rr[i]);
-            }
             const int tstart = t0 + j * TN;
             const int lim = t1 - tstart;   // tile columns >= lim lie past the split
             const int tree0 = L - tstart;  // tile columns >= tree0 are tree nodes
+            // after a failed wait the loads, exponentials and stores below still run (on
+            // whatever the buffers hold; the CTA's output is NaN then), only the waits and
+            // hand-offs to other roles are skipped
+            tc_fence_after();
+#pragma unroll
+            for (int c32 = 0; c32 < HALF_N / 32; ++c32) {
+                uint32_t rr[32];
+                tmem_ld_x32(tmem + lane_base + X * HALF_N + c32 * 32, rr);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[c32 * 32 + i] = __uint_as_float(rr[i]);
+            }
+            // the scores are in registers (the loads waited): the next tile's S = Q K^T may
+            // overwrite the buffer
+            tc_fence_before();
+            if (live) mbar_arrive(s_free);
             if (lim < TN || tree0 < TN) {
                 uint32_t cm[2];
 #pragma unroll
@@ -408,9 +445,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 m_run = mt;
             }
             const float mu = m_run == -INFINITY ? 0.f : m_run;
-            // exponentials, packed as bf16 pairs (token 2i in the low half of column i) as
-            // they are made, over the first 32 of this group's S columns of the tile,
-            // whose scores were read above
+            turn_wait();
+            // exponentials, packed as bf16 pairs (token 2i in the low half of column i), into
+            // this group's 32 columns of P buffer j % 2; P V of tile j - 2, which read them,
+            // finished before this group released P of tile j - 1 (the o_done wait below)
             float s4[4] = {0.f, 0.f, 0.f, 0.f};
             {
                 uint32_t pp[32];
@@ -422,8 +460,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     s4[(2 * i + 1) & 3] += e1;
                     pp[i] = pack_bf16(e0, e1);
                 }
-                tmem_st_x32(tmem + lane_base + sb * TN + X * HALF_N, pp);
+                tmem_st_x32(tmem + lane_base + P_COL + (j & 1) * 64 + X * 32, pp);
             }
+            turn_pass(j);
+            if (!live) continue;
             l_run = l_run * f + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
             if (lim < TN) {
                 // value rows past the split end repeat another block or hold data
@@ -440,7 +480,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
             // this group's previous P V must be complete before O is rescaled and
             // before P V of this tile is released (every phase is waited, in order)
-            if (j > 0 && !warp_wait(o_done(X), (j - 1) & 1, abort_flag)) break;
+            if (j > 0) live = warp_wait(o_done(X), (j - 1) & 1, abort_flag);
+            if (!live) continue;
             // tcgen05.ld / st are warp-collective (.sync.aligned): the whole warp rescales
             // when any of its rows needs it (rows whose max did not move multiply by 1)
             if (j > 0 && __any_sync(0xffffffffu, f != 1.f)) {
