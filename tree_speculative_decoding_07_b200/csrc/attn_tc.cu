@@ -25,10 +25,15 @@
 //               several tiles ahead.
 //   warp 1      S = Q K^T issuer: tcgen05.mma kind::f16, M 128, N 128, 8 x K16,
 //               into the TMEM S buffer, reused as soon as both softmax groups
-//               have read the previous tile's scores into registers.
+//               have read the previous tile's scores into registers.  Q is
+//               staged in TMEM by the softmax threads (one row each), so the
+//               MMA takes it from there (the TMEM-A form) and reads only the
+//               K tile from shared memory: with both operands in shared memory
+//               each of these MMAs took ~86 cycles against ~68 for the P V
+//               MMAs, which read one.
 //   warp 2      O_x += P_x V issuer (one per softmax group, over that group's 64
 //               tokens), and owner of the TMEM allocation (all 512 columns:
-//               S, two P buffers, O_A, O_B).  The two issuers sit on different SM
+//               S, P, Q, O_A, O_B).  The two issuers sit on different SM
 //               sub-partitions.
 //   warps 4-7   softmax group A: columns 0..63 of every S tile
 //   warps 8-11  softmax group B: columns 64..127
@@ -42,9 +47,10 @@
 // scores in step.  Scores are scaled into the log2 domain by the same FFMA that
 // subtracts the running max; the O rescale in TMEM is skipped while the max
 // grows by at most 2^8.  P is written as bf16 pairs into a TMEM P buffer of its
-// own (tile j into buffer j % 2), and P V takes it from there (the TMEM-A form
-// of the MMA); since P does not overwrite the scores, S = Q K^T of tile j + 1
-// runs while the softmax of tile j is still computing.  The
+// own, once this group's P V of the previous tile has read it, and P V takes it
+// from there (the TMEM-A form of the MMA); since P does not overwrite the
+// scores, S = Q K^T of tile j + 1 runs while the softmax of tile j is still
+// computing.  The
 // tree mask is a 128-bit ancestor set per node (anc(i) = anc(parent(i)) |
 // {i}), shifted into column space once per tile; prefix-only tiles skip it.
 //
@@ -63,12 +69,12 @@ constexpr int TC_THREADS = 384;
 constexpr int HALF_N = TN / 2;   // tokens per softmax group
 constexpr int KST = 3;           // K ring depth
 constexpr int VST = 3;           // V ring depth
-constexpr uint32_t SQ_OFF = 0;             // Q: 2 x [128 rows][128 B], swizzled
-constexpr uint32_t SK_OFF = 32768;         // K ring: KST x 32 KB
+constexpr uint32_t SK_OFF = 0;             // K ring: KST x 32 KB
 constexpr uint32_t SV_OFF = SK_OFF + KST * 32768u;  // V ring: VST x 32 KB
 constexpr uint32_t SMEM_BYTES = SV_OFF + VST * 32768u + 1024;
-constexpr uint32_t TMEM_COLS = 512;        // S [0,128), P0 [128,192), P1 [192,256), O_A [256,384), O_B [384,512)
-constexpr uint32_t P_COL = 128;            // P buffer j % 2: 64 columns of bf16 pairs, group x at x * 32
+constexpr uint32_t TMEM_COLS = 512;        // S [0,128), P [128,192), Q [192,256), O_A [256,384), O_B [384,512)
+constexpr uint32_t P_COL = 128;            // P: 64 columns of bf16 pairs, group x at x * 32
+constexpr uint32_t Q_COL = 192;            // Q: 64 columns of bf16 pairs (dims 2c, 2c + 1 in column c)
 constexpr uint32_t O_COL = 256;
 // named barriers passing the turn at the exponentials: group A waits on BAR_TURN_A
 // (B arrives), group B on BAR_TURN_B (A arrives); 0 is __syncthreads, 1 the epilogue's
@@ -118,7 +124,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const uint32_t raw = smem_u32(dsmem);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* base_ptr = dsmem + (base - raw);
-    const uint32_t sQ = base + SQ_OFF;
     auto sK = [&](int s) { return base + SK_OFF + (uint32_t)s * TILE_BYTES; };
     auto sV = [&](int s) { return base + SV_OFF + (uint32_t)s * TILE_BYTES; };
     const uint32_t bar0 = smem_u32(&bars[0]);
@@ -280,7 +285,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             bool issued_any = false;
             // descriptors of the tiles' first 16-column step; the other steps add a
             // constant to the address field (addresses stay below 2^18 bytes)
-            const uint64_t dq = sdesc(sQ, 16, 1024);
             const uint64_t dk0 = sdesc(sK(0), 16, 1024);
             for (int j = 0; ok && j < ntiles; ++j) {
                 const int ks = j % KST;
@@ -294,7 +298,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k) {
                     const uint32_t off = ((k >> 2) * HALF_BYTES + (k & 3) * 32u) >> 4;
-                    mma_bf16(tmem, dq + off, dk + off, IDESC_QK, k > 0 ? 1u : 0u);
+                    mma_bf16_ts(tmem, tmem + Q_COL + k * 8, dk + off, IDESC_QK, k > 0 ? 1u : 0u);
                 }
                 mma_commit(s_full);
                 mma_commit(k_empty(ks));
@@ -324,7 +328,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < HALF_N / 16; ++k)
-                        mma_bf16_ts(tmem + O_COL + x * HD, tmem + P_COL + (t & 1) * 64 + x * 32 + k * 8,
+                        mma_bf16_ts(tmem + O_COL + x * HD, tmem + P_COL + x * 32 + k * 8,
                                     dv + (uint64_t)(((x * 4 + k) * 2048u) >> 4), IDESC_PV, (t > 0 || k > 0) ? 1u : 0u);
                     mma_commit(o_done(x));
                     issued_any = true;
@@ -373,12 +377,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         {
             const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
                                                               (((size_t)b * N + node) * a.Hq + head) * HD + X * 64);
+            uint32_t qw[32];
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const uint4 v = row_ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-                st_shared_v4(sQ + X * HALF_BYTES + r * 128 + ((c ^ (r & 7)) << 4), v);
+                qw[4 * c] = v.x;
+                qw[4 * c + 1] = v.y;
+                qw[4 * c + 2] = v.z;
+                qw[4 * c + 3] = v.w;
             }
-            fence_proxy_async();
+            tmem_st_x32(tmem + lane_base + Q_COL + X * 32, qw);
+            tmem_wait_st();
+            tc_fence_before();
             mbar_arrive(q_ready);
         }
         float m_run = -INFINITY, l_run = 0.f;  // running max in the scaled log2 domain, running sum
@@ -446,6 +456,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
             const float mu = m_run == -INFINITY ? 0.f : m_run;
             turn_wait();
+            // one P buffer: this group's P V of the previous tile has read it before it is
+            // overwritten (the same wait also frees O for the rescale below)
+            if (j > 0 && live) live = warp_wait(o_done(X), (j - 1) & 1, abort_flag);
             // exponentials, packed as bf16 pairs (token 2i in the low half of column i), into
             // this group's 32 columns of P buffer j % 2; P V of tile j - 2, which read them,
             // finished before this group released P of tile j - 1 (the o_done wait below)
@@ -460,7 +473,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     s4[(2 * i + 1) & 3] += e1;
                     pp[i] = pack_bf16(e0, e1);
                 }
-                tmem_st_x32(tmem + lane_base + P_COL + (j & 1) * 64 + X * 32, pp);
+                tmem_st_x32(tmem + lane_base + P_COL + X * 32, pp);
             }
             turn_pass(j);
             if (!live) continue;
@@ -480,7 +493,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
             // this group's previous P V must be complete before O is rescaled and
             // before P V of this tile is released (every phase is waited, in order)
-            if (j > 0) live = warp_wait(o_done(X), (j - 1) & 1, abort_flag);
             if (!live) continue;
             // tcgen05.ld / st are warp-collective (.sync.aligned): the whole warp rescales
             // when any of its rows needs it (rows whose max did not move multiply by 1)
@@ -503,9 +515,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         asm volatile("bar.sync 1, 256;" ::: "memory");
         bool fail = __any_sync(0xffffffffu, *abort_flag != 0);
         if (ntiles > 0 && !fail) fail = !warp_wait(o_done(X), (ntiles - 1) & 1, abort_flag);
-        // per-row (max, sum) of each group, exchanged through that group's half of the Q
-        // buffer: every S = Q K^T finished before this group's last P V
-        float* pm = reinterpret_cast<float*>(base_ptr + SQ_OFF);
+        // per-row (max, sum) of each group, exchanged through the first K slot: every
+        // K copy was consumed by an S = Q K^T that finished before the loops ended, and
+        // peers write to the K ring only after this CTA reports it free (below)
+        float* pm = reinterpret_cast<float*>(base_ptr + SK_OFF);
         auto s_m = [&](int g) { return pm + g * (HALF_BYTES / 4); };
         auto s_l = [&](int g) { return pm + g * (HALF_BYTES / 4) + TM; };
         s_m(X)[r] = m_run;
