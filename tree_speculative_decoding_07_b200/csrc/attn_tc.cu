@@ -145,6 +145,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int r = ((warp & 3) << 5) + lane;                  // query row in the tile (softmax warps)
 
     // ---- prologue
+    // The softmax threads request their row's 64 query values and one parent index
+    // first of all, so these global-memory latencies overlap the set-up below and the
+    // block-id loads instead of following them (Q goes to TMEM after the barrier).
+    const int gr = tile * TM + r;
+    const bool row_ok = warp >= 4 && gr < G * n;
+    const int node = row_ok ? gr / G : 0;
+    const int head = kvh * G + (row_ok ? gr % G : 0);
+    uint32_t qw[32];
+    {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
+                                                          (((size_t)b * N + node) * a.Hq + head) * HD + X * 64);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 v = row_ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+            qw[4 * c] = v.x;
+            qw[4 * c + 1] = v.y;
+            qw[4 * c + 2] = v.z;
+            qw[4 * c + 3] = v.w;
+        }
+    }
+    const int32_t par_i = (warp >= 4 && tid - 128 < n) ? parent_at(a.parent, b, N, tid - 128) : 0;
     if ((warp == 0 || warp == 3) && lane == 0) prefetch_tensormap(warp == 0 ? &tmk : &tmv);
     if (tid == 0) {
         s_abort = 0;
@@ -196,7 +217,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     };
     if (warp == 0 || warp == 3)
         for (int jt = 0; jt < ID_AHEAD; ++jt) prefetch_ids(jt);
-    for (int i = tid; i < n; i += TC_THREADS) s_par[i] = parent_at(a.parent, b, N, i);
     __syncthreads();
     // a kernel launched after this one with programmatic stream serialisation may
     // start its set-up now; it waits for this grid before reading anything
@@ -348,14 +368,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // ---------------- softmax groups: one thread per query row / TMEM lane
         const int st = tid - 128;  // 0..255
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        if (st < n) s_par[st] = par_i;  // n <= TV_MAX_NODES_ATTN < 256
+        asm volatile("bar.sync 1, 256;" ::: "memory");
         for (int i = st; i < n; i += 256)
             if (!parent_ok(s_par, i)) s_bad = TV_ERR_TREE;
         if (st == 0 && bad_len) s_bad = TV_ERR_BLOCK_TABLE;
         if (st == 0 && bad_count) s_bad = TV_ERR_INVALID_ARG;
-        const int gr = tile * TM + r;
-        const bool row_ok = gr < G * n;
-        const int node = row_ok ? gr / G : 0;
-        const int head = kvh * G + (row_ok ? gr % G : 0);
         uint32_t an0 = 0, an1 = 0, an2 = 0, an3 = 0;
         if (row_ok && !a.parent) {
             // a chain: node i's ancestors are nodes 0..i (the causal tail), no walk needed
@@ -375,17 +393,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
         }
         {
-            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
-                                                              (((size_t)b * N + node) * a.Hq + head) * HD + X * 64);
-            uint32_t qw[32];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 v = row_ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-                qw[4 * c] = v.x;
-                qw[4 * c + 1] = v.y;
-                qw[4 * c + 2] = v.z;
-                qw[4 * c + 3] = v.w;
-            }
             tmem_st_x32(tmem + lane_base + Q_COL + X * 32, qw);
             tmem_wait_st();
             tc_fence_before();
