@@ -599,8 +599,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             // this CTA's K ring is idle: every CTA of the cluster may send to it
             for (int k = 0; k < S; ++k) mbar_arrive_cluster(mapa_shared(free_bar, (uint32_t)k));
             if (mbar_wait_cluster_bounded(free_bar, 0)) {
-                // NaN rows when this CTA failed: the owners still get every byte they wait for
-                for (int k = 0; k < S; ++k) {
+                // NaN rows when this CTA failed: the owners still get every byte they wait for.
+                // CTA s sends to s, s + 1, ... in turn, so no owner receives all S copies
+                // first (with every CTA starting at owner 0 the owners finished one after
+                // another, ~0.15 us apart on l8b)
+                for (int i = 0; i < S; ++i) {
+                    const int k = split + i < S ? split + i : split + i - S;
                     const int own_k = max(0, min(TM, (k + 1) * R) - k * R);
                     if (own_k > 0)
                         bulk_copy_cluster(mapa_shared(recv + (uint32_t)(split * R * PROW_BYTES), (uint32_t)k),
