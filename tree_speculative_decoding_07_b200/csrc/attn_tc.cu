@@ -69,6 +69,7 @@ constexpr int TC_THREADS = 384;
 constexpr int HALF_N = TN / 2;   // tokens per softmax group
 constexpr int KST = 3;           // K ring depth
 constexpr int VST = 3;           // V ring depth
+constexpr int SHORT_SPLIT_TILES = 8;  // splits of at most this many tiles hold their V ring at first
 constexpr uint32_t SK_OFF = 0;             // K ring: KST x 32 KB
 constexpr uint32_t SV_OFF = SK_OFF + KST * 32768u;  // V ring: VST x 32 KB
 constexpr uint32_t SMEM_BYTES = SV_OFF + VST * 32768u + 1024;
@@ -279,9 +280,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             // the slot refilled here last held tile j + ID_AHEAD - ID_RING, read before
             prefetch_ids(j + ID_AHEAD);
             ++issued;
-            // let the first tile land before streaming the rest, so it does not queue
-            // behind every other tile of the launch
-            if (j == 0 && ntiles > 1 && !warp_wait(is_k ? k_full(0) : v_full(0), 0, abort_flag)) break;
+            // A split of a few tiles is bound by its first tiles' latency: its V copies wait
+            // until the first V tile has landed, so they do not queue beside the K tiles the
+            // first S = Q K^T tiles need (l8b with L2 flushed: 23.0 us against 24.6 with
+            // both rings held after their first tile, and 24.1 with neither).  A long split
+            // streams both rings from the start (2-3 % faster on l70b and long).
+            if (j == 0 && !is_k && ntiles > 1 && ntiles <= SHORT_SPLIT_TILES &&
+                !warp_wait(v_full(0), 0, abort_flag))
+                break;
         }
         asm volatile("cp.async.wait_all;" ::: "memory");  // no id copy lands after the ring is abandoned
         if (bad_id) s_bad = TV_ERR_BLOCK_TABLE;
