@@ -81,7 +81,6 @@ struct SampleShared {
     int found_t;
     int wsel;
     double wbefore;
-    double wofs[MAX_THREADS / 32];  // bonus scan: exclusive prefix of the warps' totals
     float u0;                       // the bonus draw's uniform, read at launch
 };
 
@@ -165,6 +164,34 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 #pragma unroll
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
+}
+// inclusive prefix sums over the lanes (lane k gets v_0 + ... + v_k, summed as a tree)
+__device__ __forceinline__ double warp_scan_d(double v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double t = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += t;
+    }
+    return v;
+}
+// The first of n (<= 32) running totals that exceeds a target, from one value per lane:
+// `first` is that lane (-1 if none), `last_pos` the last lane with a positive value, and
+// `before` the running total of the lanes before `first` (0 for lane 0).  Every lane of
+// the warp gets the same results.
+struct Crossing {
+    int first, last_pos;
+    double before;
+};
+__device__ __forceinline__ Crossing first_crossing(double v, int n, double base, double target, int lane) {
+    const double inc = warp_scan_d(lane < n ? v : 0.0, lane);
+    const unsigned cross = __ballot_sync(0xffffffffu, lane < n && base + inc > target);
+    const unsigned pos = __ballot_sync(0xffffffffu, lane < n && v > 0.0);
+    Crossing r;
+    r.first = cross ? __ffs((int)cross) - 1 : -1;
+    r.last_pos = pos ? 31 - __clz((int)pos) : -1;
+    const double prev = __shfl_sync(0xffffffffu, inc, r.first > 0 ? r.first - 1 : 0);
+    r.before = base + (r.first > 0 ? prev : 0.0);
+    return r;
 }
 __device__ __forceinline__ double warp_max_d(double v) {
 #pragma unroll
@@ -621,44 +648,27 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(const __grid
         }
         const int par = (w.passes - 1) & 1;
         const double target = (double)sh.u0 * total;
-        int owner = -1, last_pos_cta = -1;
-        double before = 0.0, run = 0.0;
-        for (int k = 0; k < C; ++k) {
-            const double pk = sh.peer[par][k];
-            if (pk > 0.0) last_pos_cta = k;
-            if (owner < 0) {
-                if (run + pk > target) {
-                    owner = k;
-                    before = run;
-                }
-                run += pk;
-            }
-        }
-        const bool fallback = owner < 0;
-        if (fallback) owner = last_pos_cta;
+        // the CTA whose slice holds the crossing: every warp scans the C slice totals of the
+        // last pass (one per lane), so every thread of every CTA gets the same owner
+        const Crossing oc = first_crossing(lane < C ? sh.peer[par][lane] : 0.0, C, 0.0, target, lane);
+        const bool fallback = oc.first < 0;
+        const int owner = fallback ? oc.last_pos : oc.first;
+        const double before = oc.before;
 
         if (rank == owner) {
             const float* pr = w.ps(x);
             const float* qr = w.qs(x);
-            if (tid == 0) {
+            if (warp == 0) {
                 // first warp segment whose running sum crosses the target; the last one
-                // with mass if rounding leaves none
-                int wsel = -1, wlast = -1;
-                double rb = before, rr = before;
-                for (int k = 0; k < nwarps; ++k) {
-                    if (sh.warp_part[k] > 0.0) wlast = k;
-                    if (wsel < 0 && !fallback) {
-                        if (rr + sh.warp_part[k] > target) {
-                            wsel = k;
-                            rb = rr;
-                        }
-                        rr += sh.warp_part[k];
-                    }
+                // with mass if rounding leaves none (or the CTA was taken as a fallback)
+                const Crossing wc = first_crossing(lane < nwarps ? sh.warp_part[lane] : 0.0, nwarps, before,
+                                                   fallback ? INFINITY : target, lane);
+                if (lane == 0) {
+                    sh.wsel = wc.first >= 0 ? wc.first : wc.last_pos;
+                    sh.wbefore = wc.first >= 0 ? wc.before : -INFINITY;  // -inf: the segment's last positive element
+                    sh.found = -1;
+                    sh.found_t = INT_MAX;
                 }
-                sh.wsel = wsel >= 0 ? wsel : wlast;
-                sh.wbefore = wsel >= 0 ? rb : -INFINITY;  // -inf: take the segment's last positive element
-                sh.found = -1;
-                sh.found_t = INT_MAX;
             }
             __syncthreads();
             // the whole CTA scans the selected segment: each thread a run of at most a
@@ -681,15 +691,12 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(const __grid
             }
             if (lane == 31) sh.warp_part2[warp] = incl;
             __syncthreads();
-            if (tid == 0) {
-                double acc = 0.0;
-                for (int k = 0; k < nwarps; ++k) {
-                    sh.wofs[k] = acc;
-                    acc += sh.warp_part2[k];
-                }
+            {
+                // this warp's offset: the running total of the warps before it
+                const double inc = warp_scan_d(lane < nwarps ? sh.warp_part2[lane] : 0.0, lane);
+                const double prev = __shfl_sync(0xffffffffu, inc, warp > 0 ? warp - 1 : 0);
+                incl += warp > 0 ? prev : 0.0;
             }
-            __syncthreads();
-            incl += sh.wofs[warp];
             const bool take_last = sh.wbefore == -INFINITY;
             // the first thread whose inclusive running sum exceeds the target holds the draw
             if (!take_last && sh.wbefore + incl > target) atomicMin(&sh.found_t, tid);
