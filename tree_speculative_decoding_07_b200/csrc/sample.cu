@@ -45,6 +45,7 @@
 // waits), so its peers time out once and stop too; the status word records
 // TV_ERR_TIMEOUT.
 #include <cooperative_groups.h>
+#include <mutex>
 
 #include "tv_common.cuh"
 #include "kernels.h"
@@ -763,10 +764,23 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(const __grid
 
 size_t sample_static_smem() { return sizeof(SampleShared); }
 
+// The largest cluster (16 CTAs, else the portable 8) that the device can hold, found once per
+// device: the answer and the function attributes set to find it belong to the current device.
+namespace {
+constexpr int MAX_DEVICES = 64;
+std::mutex g_cluster_mutex;
+int g_max_cluster[MAX_DEVICES] = {};  // 0: not yet found
+}  // namespace
+
 int sample_max_cluster() {
-    static int best = -1;
-    if (best >= 0) return best;
-    best = 8;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) {
+        cudaGetLastError();
+        return 8;
+    }
+    std::lock_guard<std::mutex> lock(g_cluster_mutex);
+    if (g_max_cluster[dev]) return g_max_cluster[dev];
+    int best = 8;
     if (cudaFuncSetAttribute(verify_sample_kernel<false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
             cudaSuccess &&
         cudaFuncSetAttribute(verify_sample_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024) ==
@@ -787,6 +801,7 @@ int sample_max_cluster() {
             best = 16;
     }
     cudaGetLastError();
+    g_max_cluster[dev] = best;
     return best;
 }
 
