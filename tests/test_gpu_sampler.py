@@ -105,3 +105,56 @@ def test_bad_tree_is_reported():
     assert int(status.item()) == tv.TV_ERR_TREE
     assert res["accepted_len"][1] == -1 and res["bonus_token"][1] == -1
     assert res["accepted_len"][0] >= 0
+
+
+def test_bonus_draw_finds_the_owner_anywhere_in_the_vocabulary():
+    # The root's only child has p(x) = 0, so it is always rejected, and the bonus token comes
+    # from the residual max(0, p - q).  The residual is zero everywhere except a few chosen
+    # entries, placed at the two ends of a 128,256-entry vocabulary and inside slices far from
+    # the first (the walk spreads the vocabulary over up to 16 CTAs), so the owner of the draw
+    # is found at the edges of the CTA and warp scans.  u0 = 0 takes the first entry with mass.
+    V = 128256
+    spots = [[0], [V - 1], [3 * V // 16 + 5, 12 * V // 16 + 7], [3 * V // 16 + 5, 12 * V // 16 + 7],
+             [V // 2 - 1, V // 2, V // 2 + 1], [7, V - 2]]
+    u0 = [0.5, 0.5, 0.25, 0.75, 0.0, 0.3]
+    B, x = len(spots), 11  # x: the child's draft token
+    q = np.full((B, 2, V), 1.0 / V, np.float32)
+    p = np.full((B, 2, V), 0.5 / V, np.float32)  # below q: no residual mass
+    for s, ks in enumerate(spots):
+        p[s, 0, x] = 0.0
+        for k in ks:
+            p[s, 0, k] = 2.0 / V  # above q: residual mass 1 / V each
+        p[s, 0] /= p[s, 0].sum()
+        p[s, 1] = p[s, 0]
+    tok = np.array([[0, x]] * B, np.int32)
+    par = np.array([[-1, 0]] * B, np.int32)
+    u = np.array([[u0[s], 0.5] for s in range(B)], np.float32)
+    ref = oracle.verify_sample(p, q, tok, par, u)
+    gpu = run_sampler_gpu(p, q, tok, par, u)
+    compare_sampler(gpu, ref, oracle.verify_sample(p, q, tok, par, u, eps=1e-9))
+    want = [0, V - 1, spots[2][0], spots[3][1], spots[4][0], 7]
+    assert list(gpu["bonus_token"]) == want
+    assert (gpu["accepted_len"] == 0).all()
+
+
+def test_bonus_draw_with_u0_just_below_one_takes_the_last_entry_with_mass():
+    # target = u0 * Z sits within rounding of the total: whichever way the sums round, the
+    # draw must be the last entry with residual mass (the oracle's fallback reading)
+    V = 128256
+    B, x = 3, 11
+    last = [V - 1, 9 * V // 16 + 3, 5]
+    q = np.full((B, 2, V), 1.0 / V, np.float32)
+    p = np.full((B, 2, V), 0.5 / V, np.float32)
+    for s in range(B):
+        p[s, 0, x] = 0.0
+        for k in (2, 4 * V // 16 + 1, last[s]):
+            if k <= last[s]:
+                p[s, 0, k] = 2.0 / V
+        p[s, 0] /= p[s, 0].sum()
+        p[s, 1] = p[s, 0]
+    tok = np.array([[0, x]] * B, np.int32)
+    par = np.array([[-1, 0]] * B, np.int32)
+    u = np.array([[np.nextafter(np.float32(1), np.float32(0)), 0.5]] * B, np.float32)
+    gpu = run_sampler_gpu(p, q, tok, par, u)
+    assert list(gpu["bonus_token"]) == last
+    assert (gpu["accepted_len"] == 0).all()
