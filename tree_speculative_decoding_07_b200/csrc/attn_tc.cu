@@ -600,28 +600,30 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint32_t recv = base + SK_OFF, stage = base + SV_OFF;
         // every CTA of the cluster has initialised its barriers
         asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-        if (tid == 0) {
-            mbar_expect_tx(merge_bar, (uint32_t)(own * S * PROW_BYTES));
-            // this CTA's K ring is idle: every CTA of the cluster may send to it
-            for (int k = 0; k < S; ++k) mbar_arrive_cluster(mapa_shared(free_bar, (uint32_t)k));
-            if (mbar_wait_cluster_bounded(free_bar, 0)) {
-                // NaN rows when this CTA failed: the owners still get every byte they wait for.
-                // CTA s sends to s, s + 1, ... in turn, so no owner receives all S copies
-                // first (with every CTA starting at owner 0 the owners finished one after
-                // another, ~0.15 us apart on l8b)
-                for (int i = 0; i < S; ++i) {
-                    const int k = split + i < S ? split + i : split + i - S;
-                    const int own_k = max(0, min(TM, (k + 1) * R) - k * R);
-                    if (own_k > 0)
-                        bulk_copy_cluster(mapa_shared(recv + (uint32_t)(split * R * PROW_BYTES), (uint32_t)k),
-                                          stage + (uint32_t)(k * R * PROW_BYTES), (uint32_t)(own_k * PROW_BYTES),
-                                          mapa_shared(merge_bar, (uint32_t)k));
-                }
-            } else {
-                *abort_flag = 1;
+        if (warp == 0) {
+            bool fr = false;
+            if (lane == 0) {
+                mbar_expect_tx(merge_bar, (uint32_t)(own * S * PROW_BYTES));
+                // this CTA's K ring is idle: every CTA of the cluster may send to it
+                for (int k = 0; k < S; ++k) mbar_arrive_cluster(mapa_shared(free_bar, (uint32_t)k));
+                fr = mbar_wait_cluster_bounded(free_bar, 0);
+                if (!fr) *abort_flag = 1;
             }
+            // NaN rows when this CTA failed: the owners still get every byte they wait for.
+            // Lane i sends to owner s + i (mod S), all at once; CTA s starts at owner s, so no
+            // owner receives all S copies first (with every CTA starting at owner 0 the
+            // owners finished one after another, ~0.15 us apart on l8b)
+            if (__shfl_sync(0xffffffffu, fr ? 1 : 0, 0) && lane < S) {
+                const int k = split + lane < S ? split + lane : split + lane - S;
+                const int own_k = max(0, min(TM, (k + 1) * R) - k * R);
+                if (own_k > 0)
+                    bulk_copy_cluster(mapa_shared(recv + (uint32_t)(split * R * PROW_BYTES), (uint32_t)k),
+                                      stage + (uint32_t)(k * R * PROW_BYTES), (uint32_t)(own_k * PROW_BYTES),
+                                      mapa_shared(merge_bar, (uint32_t)k));
+            }
+            __syncwarp();
             // every partial row of this CTA's share has arrived (always waited for, bounded)
-            s_got = mbar_wait_cluster_bounded(merge_bar, 0) ? 1 : 0;
+            if (lane == 0) s_got = mbar_wait_cluster_bounded(merge_bar, 0) ? 1 : 0;
         }
         __syncthreads();
         // this CTA has received everything sent to it (its merge barrier saw every copy
@@ -630,7 +632,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // is at the end, after the local merge
         asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
         __syncthreads();
-        const uint8_t* part = base_ptr + SK_OFF;
+        const uint32_t part = base + SK_OFF;
         if (!s_got) {
             *abort_flag = 1;
             for (int item = tid; item < own * (HD / 4); item += TC_THREADS) {

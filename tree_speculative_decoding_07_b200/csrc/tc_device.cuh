@@ -147,6 +147,17 @@ __device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&r)[
                  : "memory");
 }
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
@@ -191,9 +202,10 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
 // from the S partials it received into shared memory (layout [S][R] rows of
 // PROW_BYTES: 128 bf16 outputs, then the fp32 log-sum-exp):
 // out = sum_s 2^(lse_s - m) o_s / sum_s 2^(lse_s - m), m = max_s lse_s.
-// Each item is 8 columns of one row, so a thread issues all its loads at once.
+// Each item is 8 columns of one row, so a thread issues all its loads at once; `part` is
+// the shared-memory address of the received rows.
 template <int ROWS, int THREADS, int S_>
-__device__ __forceinline__ void merge_rows(const AttnArgs& a, const uint8_t* part, int R, int split, int tile, int b,
+__device__ __forceinline__ void merge_rows(const AttnArgs& a, uint32_t part, int R, int split, int tile, int b,
                                            int kvh, int tid, int nrows) {
     constexpr int NC = HD / 8;
     const int own = max(0, min(ROWS, (split + 1) * R) - split * R);
@@ -205,9 +217,9 @@ __device__ __forceinline__ void merge_rows(const AttnArgs& a, const uint8_t* par
         uint4 v[S_];
 #pragma unroll
         for (int k = 0; k < S_; ++k) {
-            const uint8_t* prow = part + ((size_t)k * R + rr) * PROW_BYTES;
-            ls[k] = *reinterpret_cast<const float*>(prow + 2 * HD);
-            v[k] = reinterpret_cast<const uint4*>(prow)[cc];
+            const uint32_t prow = part + (uint32_t)(k * R + rr) * PROW_BYTES;
+            ls[k] = ld_shared_f32(prow + 2 * HD);
+            v[k] = ld_shared_v4(prow + 16u * cc);
         }
         float mx = -INFINITY;
         bool nan = false;
