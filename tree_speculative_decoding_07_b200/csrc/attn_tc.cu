@@ -11,11 +11,10 @@
 // blocks of the block table (known at launch, so the block ids are fetched
 // before the sequence's length arrives).  The S splits of a row tile form one
 // thread-block cluster; when all have finished their tokens, each stages its
-// normalised partial rows (bf16) and their log-sum-exp in its idle V ring and
-// sends each CTA the rows that CTA owns (an equal share per CTA) with one bulk
-// shared-to-shared copy, completing on the owner's mbarrier; each owner
-// combines its rows from the S partials (flash-decoding log-sum-exp merge).
-// No global workspace is used.
+// normalised partial rows (bf16) and their log-sum-exp in its idle V ring, and
+// after a cluster barrier each CTA reads the rows it owns (an equal share per
+// CTA) from every CTA's staging in place (distributed shared memory) and
+// combines them (flash-decoding log-sum-exp merge).  No global workspace is used.
 //
 // Warp roles (384 threads):
 //   warp 0      TMA producer of K tiles, warp 3 of V tiles: the rows of 8 paged
@@ -54,10 +53,10 @@
 // tree mask is a 128-bit ancestor set per node (anc(i) = anc(parent(i)) |
 // {i}), shifted into column space once per tile; prefix-only tiles skip it.
 //
-// Every wait (mbarrier phase) is bounded (about two seconds of clock); on
-// expiry the CTA records TV_ERR_TIMEOUT, stops issuing work, drains its copies
-// and MMAs, frees its TMEM, and still takes part in the merge with NaN rows so
-// no peer is left waiting.
+// Every mbarrier wait is bounded (about two seconds of clock); on expiry the
+// CTA records TV_ERR_TIMEOUT, stops issuing work, drains its copies and MMAs,
+// frees its TMEM, and still takes part in the merge with NaN rows, so every CTA
+// of the cluster reaches the merge's two cluster barriers.
 #include <mutex>
 
 #include "tc_device.cuh"
@@ -93,12 +92,9 @@ constexpr int BAR_O_DONE = BAR_P_FULL + 2;       // 2: group's P V done
 constexpr int BAR_Q_READY = BAR_O_DONE + 2;      // Q staged
 constexpr int BAR_DRAIN_QK = BAR_Q_READY + 1;    // all S = Q K^T MMAs done
 constexpr int BAR_DRAIN_PV = BAR_DRAIN_QK + 1;   // all P V MMAs done
-constexpr int BAR_FREE = BAR_DRAIN_PV + 1;       // S arrivals: every CTA of the cluster can receive partials
-constexpr int BAR_MERGE = BAR_FREE + 1;          // this CTA's share of partial rows received (transaction count)
-constexpr int BAR_COUNT = BAR_MERGE + 1;
-static_assert(BAR_COUNT == 2 * KST + 2 * VST + 11, "barrier slots overlap");
+constexpr int BAR_COUNT = BAR_DRAIN_PV + 1;
+static_assert(BAR_COUNT == 2 * KST + 2 * VST + 9, "barrier slots overlap");
 static_assert(TM * PROW_BYTES <= VST * TILE_BYTES, "staged partial rows exceed the V ring");
-static_assert((TM + MAX_SPLITS) * PROW_BYTES <= KST * TILE_BYTES, "received partial rows exceed the K ring");
 
 __global__ void __launch_bounds__(TC_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tmk,
@@ -106,7 +102,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     extern __shared__ uint8_t dsmem[];
     __shared__ __align__(8) uint64_t bars[BAR_COUNT];
     __shared__ uint32_t s_tmem;
-    __shared__ int s_abort, s_bad, s_got;
+    __shared__ int s_abort, s_bad;
     __shared__ int32_t s_par[TV_MAX_NODES_ATTN];
     __shared__ __align__(16) int32_t s_ids[2][ID_RING * BLK_PER_TILE];  // block ids, per producer
 
@@ -137,7 +133,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     auto o_done = [&](int x) { return bar0 + 8u * (BAR_O_DONE + x); };
     const uint32_t q_ready = bar0 + 8u * BAR_Q_READY;
     const uint32_t drain_qk = bar0 + 8u * BAR_DRAIN_QK, drain_pv = bar0 + 8u * BAR_DRAIN_PV;
-    const uint32_t free_bar = bar0 + 8u * BAR_FREE, merge_bar = bar0 + 8u * BAR_MERGE;
     volatile int* abort_flag = &s_abort;
     // results of the softmax groups, consumed by the split merge after the role blocks
     uint32_t pk[32];   // this thread's 64 outputs of its row, as bf16 pairs
@@ -188,8 +183,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         mbar_init(q_ready, 256);
         mbar_init(drain_qk, 1);
         mbar_init(drain_pv, 1);
-        mbar_init(free_bar, (uint32_t)S);
-        mbar_init(merge_bar, 1);
         fence_barrier_init();
     }
     if (warp == 2) {
@@ -222,9 +215,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // a kernel launched after this one with programmatic stream serialisation may
     // start its set-up now; it waits for this grid before reading anything
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    // the CTAs of the cluster have initialised their barriers (the merge's remote
-    // operations wait for this arrival of every CTA)
-    if (S > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     tc_fence_after();
     const uint32_t tmem = s_tmem;
     // the split's tokens: [t0, t1) of the sequence's L + n
@@ -529,8 +519,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         bool fail = __any_sync(0xffffffffu, *abort_flag != 0);
         if (ntiles > 0 && !fail) fail = !warp_wait(o_done(X), (ntiles - 1) & 1, abort_flag);
         // per-row (max, sum) of each group, exchanged through the first K slot: every
-        // K copy was consumed by an S = Q K^T that finished before the loops ended, and
-        // peers write to the K ring only after this CTA reports it free (below)
+        // K copy was consumed by an S = Q K^T that finished before the loops ended
         float* pm = reinterpret_cast<float*>(base_ptr + SK_OFF);
         auto s_m = [&](int g) { return pm + g * (HALF_BYTES / 4); };
         auto s_l = [&](int g) { return pm + g * (HALF_BYTES / 4) + TM; };
@@ -580,7 +569,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             for (int q8 = 0; q8 < 8; ++q8)
                 st_shared_v4(row + X * HD + q8 * 16, make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]));
             if (X == 0) st_shared_v4(row + 2 * HD, make_uint4(__float_as_uint(lse), 0u, 0u, 0u));
-            fence_proxy_async();  // the bulk copies (async proxy) read these rows
         }
     }
 
@@ -591,79 +579,34 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     if (S > 1) {
         // ---- merge the KV splits of this row tile through the cluster's shared memory.
-        // Rows [k R, k R + R) belong to CTA k (split k).  Each CTA has staged its 128
-        // partial rows in its V ring; once every CTA's K ring is idle, each sends CTA k
-        // its rows [k R, k R + own_k) with one bulk copy into k's K ring, laid out
-        // [split][row - k R] with PROW_BYTES per row, completing on k's merge barrier.
+        // Rows [k R, k R + R) belong to CTA k (split k).  Every CTA has staged its 128
+        // partial rows in its V ring; after one cluster barrier (release / acquire) each
+        // CTA reads its rows from every CTA's staging in place and combines them, and a
+        // second one keeps every CTA resident until all have read its rows.  (Copying the
+        // rows to their owners first, once every owner reported its ring idle, took ~2.3 us
+        // after the last split arrived on l8b, against ~1 us for this.)
         const int R = (TM + S - 1) / S;
-        const int own = max(0, min(TM, (split + 1) * R) - split * R);
-        const uint32_t recv = base + SK_OFF, stage = base + SV_OFF;
-        // every CTA of the cluster has initialised its barriers
-        asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-        if (warp == 0) {
-            bool fr = false;
-            if (lane == 0) {
-                mbar_expect_tx(merge_bar, (uint32_t)(own * S * PROW_BYTES));
-                // this CTA's K ring is idle: every CTA of the cluster may send to it
-                for (int k = 0; k < S; ++k) mbar_arrive_cluster(mapa_shared(free_bar, (uint32_t)k));
-                fr = mbar_wait_cluster_bounded(free_bar, 0);
-                if (!fr) *abort_flag = 1;
-            }
-            // NaN rows when this CTA failed: the owners still get every byte they wait for.
-            // Lane i sends to owner s + i (mod S), all at once; CTA s starts at owner s, so no
-            // owner receives all S copies first (with every CTA starting at owner 0 the
-            // owners finished one after another, ~0.15 us apart on l8b)
-            if (__shfl_sync(0xffffffffu, fr ? 1 : 0, 0) && lane < S) {
-                const int k = split + lane < S ? split + lane : split + lane - S;
-                const int own_k = max(0, min(TM, (k + 1) * R) - k * R);
-                if (own_k > 0)
-                    bulk_copy_cluster(mapa_shared(recv + (uint32_t)(split * R * PROW_BYTES), (uint32_t)k),
-                                      stage + (uint32_t)(k * R * PROW_BYTES), (uint32_t)(own_k * PROW_BYTES),
-                                      mapa_shared(merge_bar, (uint32_t)k));
-            }
-            __syncwarp();
-            // every partial row of this CTA's share has arrived (always waited for, bounded)
-            if (lane == 0) s_got = mbar_wait_cluster_bounded(merge_bar, 0) ? 1 : 0;
+        const uint32_t stage = base + SV_OFF;
+        asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+        asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+        switch (S) {
+            case 2: merge_rows<TM, TC_THREADS, 2>(a, stage, R, split, tile, b, kvh, tid, G * n); break;
+            case 3: merge_rows<TM, TC_THREADS, 3>(a, stage, R, split, tile, b, kvh, tid, G * n); break;
+            case 4: merge_rows<TM, TC_THREADS, 4>(a, stage, R, split, tile, b, kvh, tid, G * n); break;
+            case 5: merge_rows<TM, TC_THREADS, 5>(a, stage, R, split, tile, b, kvh, tid, G * n); break;
+            case 6: merge_rows<TM, TC_THREADS, 6>(a, stage, R, split, tile, b, kvh, tid, G * n); break;
+            case 7: merge_rows<TM, TC_THREADS, 7>(a, stage, R, split, tile, b, kvh, tid, G * n); break;
+            case 8: merge_rows<TM, TC_THREADS, 8>(a, stage, R, split, tile, b, kvh, tid, G * n); break;
+            case 9: merge_rows<TM, TC_THREADS, 9>(a, stage, R, split, tile, b, kvh, tid, G * n); break;
+            case 10: merge_rows<TM, TC_THREADS, 10>(a, stage, R, split, tile, b, kvh, tid, G * n); break;
+            case 11: merge_rows<TM, TC_THREADS, 11>(a, stage, R, split, tile, b, kvh, tid, G * n); break;
+            case 12: merge_rows<TM, TC_THREADS, 12>(a, stage, R, split, tile, b, kvh, tid, G * n); break;
+            case 13: merge_rows<TM, TC_THREADS, 13>(a, stage, R, split, tile, b, kvh, tid, G * n); break;
+            case 14: merge_rows<TM, TC_THREADS, 14>(a, stage, R, split, tile, b, kvh, tid, G * n); break;
+            case 15: merge_rows<TM, TC_THREADS, 15>(a, stage, R, split, tile, b, kvh, tid, G * n); break;
+            default: merge_rows<TM, TC_THREADS, 16>(a, stage, R, split, tile, b, kvh, tid, G * n); break;
         }
-        __syncthreads();
-        // this CTA has received everything sent to it (its merge barrier saw every copy
-        // complete), so once all CTAs have arrived here no copy still reads any CTA's
-        // staged rows; the arrival orders no memory of its own (relaxed) and the wait
-        // is at the end, after the local merge
         asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-        __syncthreads();
-        const uint32_t part = base + SK_OFF;
-        if (!s_got) {
-            *abort_flag = 1;
-            for (int item = tid; item < own * (HD / 4); item += TC_THREADS) {
-                const int rt = split * R + item / (HD / 4), gr = tile * TM + rt;
-                if (gr >= G * n) continue;
-                const int node = gr / G, head = kvh * G + gr % G;
-                uint2 ov;
-                ov.x = pack_bf16(NAN, NAN);
-                ov.y = ov.x;
-                *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) +
-                                          (((size_t)b * N + node) * a.Hq + head) * HD + (item % (HD / 4)) * 4) = ov;
-            }
-        } else {
-            switch (S) {
-                case 2: merge_rows<TM, TC_THREADS, 2>(a, part, R, split, tile, b, kvh, tid, G * n); break;
-                case 3: merge_rows<TM, TC_THREADS, 3>(a, part, R, split, tile, b, kvh, tid, G * n); break;
-                case 4: merge_rows<TM, TC_THREADS, 4>(a, part, R, split, tile, b, kvh, tid, G * n); break;
-                case 5: merge_rows<TM, TC_THREADS, 5>(a, part, R, split, tile, b, kvh, tid, G * n); break;
-                case 6: merge_rows<TM, TC_THREADS, 6>(a, part, R, split, tile, b, kvh, tid, G * n); break;
-                case 7: merge_rows<TM, TC_THREADS, 7>(a, part, R, split, tile, b, kvh, tid, G * n); break;
-                case 8: merge_rows<TM, TC_THREADS, 8>(a, part, R, split, tile, b, kvh, tid, G * n); break;
-                case 9: merge_rows<TM, TC_THREADS, 9>(a, part, R, split, tile, b, kvh, tid, G * n); break;
-                case 10: merge_rows<TM, TC_THREADS, 10>(a, part, R, split, tile, b, kvh, tid, G * n); break;
-                case 11: merge_rows<TM, TC_THREADS, 11>(a, part, R, split, tile, b, kvh, tid, G * n); break;
-                case 12: merge_rows<TM, TC_THREADS, 12>(a, part, R, split, tile, b, kvh, tid, G * n); break;
-                case 13: merge_rows<TM, TC_THREADS, 13>(a, part, R, split, tile, b, kvh, tid, G * n); break;
-                case 14: merge_rows<TM, TC_THREADS, 14>(a, part, R, split, tile, b, kvh, tid, G * n); break;
-                case 15: merge_rows<TM, TC_THREADS, 15>(a, part, R, split, tile, b, kvh, tid, G * n); break;
-                default: merge_rows<TM, TC_THREADS, 16>(a, part, R, split, tile, b, kvh, tid, G * n); break;
-            }
-        }
         asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
     }
     if (tid == 0) {

@@ -147,15 +147,24 @@ __device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&r)[
                  : "memory");
 }
 
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+// address of the same shared-memory location in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+// loads from another CTA's shared memory (a shared::cluster address from mapa)
+__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
     uint4 v;
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+    asm volatile("ld.shared::cluster.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
                  : "memory");
     return v;
 }
-__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
     float v;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
     return v;
 }
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
@@ -202,10 +211,11 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
 // from the S partials it received into shared memory (layout [S][R] rows of
 // PROW_BYTES: 128 bf16 outputs, then the fp32 log-sum-exp):
 // out = sum_s 2^(lse_s - m) o_s / sum_s 2^(lse_s - m), m = max_s lse_s.
-// Each item is 8 columns of one row, so a thread issues all its loads at once; `part` is
-// the shared-memory address of the received rows.
+// Each item is 8 columns of one row, so a thread issues all its loads at once; `stage` is
+// the shared-memory address at which every CTA of the cluster staged its partial rows
+// (row r at r * PROW_BYTES), read in place from each CTA (distributed shared memory).
 template <int ROWS, int THREADS, int S_>
-__device__ __forceinline__ void merge_rows(const AttnArgs& a, uint32_t part, int R, int split, int tile, int b,
+__device__ __forceinline__ void merge_rows(const AttnArgs& a, uint32_t stage, int R, int split, int tile, int b,
                                            int kvh, int tid, int nrows) {
     constexpr int NC = HD / 8;
     const int own = max(0, min(ROWS, (split + 1) * R) - split * R);
@@ -217,9 +227,9 @@ __device__ __forceinline__ void merge_rows(const AttnArgs& a, uint32_t part, int
         uint4 v[S_];
 #pragma unroll
         for (int k = 0; k < S_; ++k) {
-            const uint32_t prow = part + (uint32_t)(k * R + rr) * PROW_BYTES;
-            ls[k] = ld_shared_f32(prow + 2 * HD);
-            v[k] = ld_shared_v4(prow + 16u * cc);
+            const uint32_t prow = mapa_shared(stage + (uint32_t)(split * R + rr) * PROW_BYTES, (uint32_t)k);
+            ls[k] = ld_cluster_f32(prow + 2 * HD);
+            v[k] = ld_cluster_v4(prow + 16u * cc);
         }
         float mx = -INFINITY;
         bool nan = false;
@@ -252,46 +262,6 @@ __device__ __forceinline__ void merge_rows(const AttnArgs& a, uint32_t part, int
         *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + (((size_t)b * a.N + node) * a.Hq + head) * HD +
                                   cc * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
-}
-
-// ---- cluster (distributed shared memory) operations of the split merge
-
-// address of the same shared-memory location in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-    return r;
-}
-// arrive on an mbarrier of any CTA of the cluster (release at cluster scope)
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-// Bounded wait (acquire at cluster scope) on a phase of this CTA's mbarrier that
-// other CTAs of the cluster complete.  It does not give up early when this CTA
-// aborted: the bytes a peer pushes must have landed before the CTA retires.
-__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t parity) {
-    const long long t0 = clock64();
-    for (;;) {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}\n"
-            : "=r"(ok)
-            : "r"(bar), "r"(parity)
-            : "memory");
-        if (ok) return true;
-        if (clock64() - t0 > WAIT_LIMIT) return false;
-    }
-}
-// bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory into the
-// shared memory of a CTA of the cluster, completing on that CTA's mbarrier
-__device__ __forceinline__ void bulk_copy_cluster(uint32_t remote_dst, uint32_t local_src, uint32_t bytes,
-                                                  uint32_t remote_bar) {
-    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     remote_dst),
-                 "r"(local_src), "r"(bytes), "r"(remote_bar)
-                 : "memory");
 }
 
 template <int NV>
