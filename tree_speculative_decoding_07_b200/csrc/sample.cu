@@ -487,12 +487,31 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(const __grid
         if (a.gather) g_first[i] = nn;
     }
     if (tid == 0) sh.u0 = __ldg(a.uniforms + (size_t)b * N);
-    // every CTA's barriers must exist before a peer pushes to them (the first pass);
-    // the cluster barrier sits here so the loads above are already in flight
-    if (C > 1)
-        cg::this_cluster().sync();
-    else
-        __syncthreads();
+    __syncthreads();
+    // Every child's draft-token entries and uniform are requested now, before the cluster
+    // barrier, so their latency overlaps it.  Each entry's parent and token are checked one
+    // by one: a malformed tree's values are never used, but no load may leave the rows.
+    // (Up to two children per thread; a tree with more falls back to loading them after
+    // the checks below.)
+    constexpr int GPT = 2;
+    const bool early = a.gather && nn <= GPT * (int)blockDim.x;
+    float gp[GPT], gq[GPT], gu[GPT];
+#pragma unroll
+    for (int k = 0; k < GPT; ++k) {
+        gp[k] = gq[k] = gu[k] = 0.f;
+        const int c = tid + 1 + k * (int)blockDim.x;
+        if (early && c < nn) {
+            const int pu = sh.parent[c], tk = sh.token[c];
+            if (pu >= 0 && pu < c && tk >= 0 && tk < a.V) {
+                const size_t at = ((size_t)b * N + pu) * (size_t)a.V + tk;
+                gp[k] = __ldg(a.p + at);
+                gq[k] = __ldg(a.q + at);
+                gu[k] = __ldg(a.uniforms + (size_t)b * N + c);
+            }
+        }
+    }
+    // every CTA's barriers must exist before a peer pushes to them (the first pass)
+    if (C > 1) cg::this_cluster().sync();
     bool bad_local = false;
     for (int i = tid; i < nn; i += blockDim.x) {
         const int p = sh.parent[i];
@@ -512,7 +531,19 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(const __grid
             }
         }
     } else {
-        if (a.gather) {
+        if (early) {
+#pragma unroll
+            for (int k = 0; k < GPT; ++k) {
+                const int c = tid + 1 + k * (int)blockDim.x;
+                if (c < nn) {
+                    g_p[c] = gp[k];
+                    g_q[c] = gq[k];
+                    g_u[c] = gu[k];
+                    atomicMin(&g_first[sh.parent[c]], c);
+                }
+            }
+            __syncthreads();
+        } else if (a.gather) {
             // every child's draft-token entries and uniform, in one round of loads
             for (int c = tid + 1; c < nn; c += blockDim.x) {
                 const int pu = sh.parent[c];
