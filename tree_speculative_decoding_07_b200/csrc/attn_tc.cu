@@ -162,8 +162,31 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
     }
     const int32_t par_i = (warp >= 4 && tid - 128 < n) ? parent_at(a.parent, b, N, tid - 128) : 0;
+    // The producer warps request the tensor maps and their first block ids before
+    // anything else (a thread that also initialised the barriers issued them only after
+    // its cluster-scope fence); warp 1, idle until the barrier below, initialises the
+    // barriers, and warp 2 allocates TMEM.
     if ((warp == 0 || warp == 3) && lane == 0) prefetch_tensormap(warp == 0 ? &tmk : &tmv);
-    if (tid == 0) {
+    // This split's logical blocks are [blk0, blk_end) of the block table, fixed at
+    // launch, so their ids are fetched without waiting for the prefix length.
+    // They reach the producers through a shared-memory ring that cp.async fills
+    // ID_AHEAD tiles ahead of use, so no tile's copies wait on a block-table load
+    // (a register loaded one tile earlier would stall every iteration for one
+    // global-memory latency).  The first copies start before the barrier,
+    // overlapping barrier set-up and TMEM allocation.
+    const int blk0 = min(a.max_blocks, split * a.blocks_per_split);
+    const int blk_end = min(a.max_blocks, blk0 + a.blocks_per_split);
+    const int32_t* bt = a.block_table + (size_t)b * a.max_blocks;
+    const int prod = warp == 0 ? 0 : 1;
+    auto prefetch_ids = [&](int jt) {
+        const int bi = blk0 + jt * BLK_PER_TILE + lane;
+        if (lane < BLK_PER_TILE && bi < blk_end)
+            cp_async_4(smem_u32(&s_ids[prod][(jt % ID_RING) * BLK_PER_TILE + lane]), bt + bi);
+        cp_async_commit();  // one group per tile on every lane, empty or not
+    };
+    if (warp == 0 || warp == 3)
+        for (int jt = 0; jt < ID_AHEAD; ++jt) prefetch_ids(jt);
+    if (tid == 32) {
         s_abort = 0;
         s_bad = 0;
         for (int s = 0; s < KST; ++s) {
@@ -192,25 +215,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
         tc_fence_before();
     }
-    // This split's logical blocks are [blk0, blk_end) of the block table, fixed at
-    // launch, so their ids are fetched without waiting for the prefix length.
-    // They reach the producers through a shared-memory ring that cp.async fills
-    // ID_AHEAD tiles ahead of use, so no tile's copies wait on a block-table load
-    // (a register loaded one tile earlier would stall every iteration for one
-    // global-memory latency).  The first copies start before the barrier,
-    // overlapping barrier set-up and TMEM allocation.
-    const int blk0 = min(a.max_blocks, split * a.blocks_per_split);
-    const int blk_end = min(a.max_blocks, blk0 + a.blocks_per_split);
-    const int32_t* bt = a.block_table + (size_t)b * a.max_blocks;
-    const int prod = warp == 0 ? 0 : 1;
-    auto prefetch_ids = [&](int jt) {
-        const int bi = blk0 + jt * BLK_PER_TILE + lane;
-        if (lane < BLK_PER_TILE && bi < blk_end)
-            cp_async_4(smem_u32(&s_ids[prod][(jt % ID_RING) * BLK_PER_TILE + lane]), bt + bi);
-        cp_async_commit();  // one group per tile on every lane, empty or not
-    };
-    if (warp == 0 || warp == 3)
-        for (int jt = 0; jt < ID_AHEAD; ++jt) prefetch_ids(jt);
     __syncthreads();
     // a kernel launched after this one with programmatic stream serialisation may
     // start its set-up now; it waits for this grid before reading anything
