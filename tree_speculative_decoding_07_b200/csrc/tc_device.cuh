@@ -208,9 +208,8 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 // Combine this CTA's share of one ROWS-row tile, rows [split * R, split * R + own),
-// from the S partials it received into shared memory (layout [S][R] rows of
-// PROW_BYTES: 128 bf16 outputs, then the fp32 log-sum-exp):
-// out = sum_s 2^(lse_s - m) o_s / sum_s 2^(lse_s - m), m = max_s lse_s.
+// from the S partials (rows of PROW_BYTES: 128 bf16 outputs, then the fp32
+// log-sum-exp): out = sum_s 2^(lse_s - m) o_s / sum_s 2^(lse_s - m), m = max_s lse_s.
 // Each item is 8 columns of one row, so a thread issues all its loads at once; `stage` is
 // the shared-memory address at which every CTA of the cluster staged its partial rows
 // (row r at r * PROW_BYTES), read in place from each CTA (distributed shared memory).
