@@ -40,14 +40,11 @@
 //   warps 8-11  softmax group B: columns 64..127
 // Each softmax thread owns one query row (its TMEM lane).  The two groups
 // keep separate running maxima / sums and separate O accumulators, merged at
-// the end like two splits.  Every SM sub-partition holds one warp of each
-// group, and the two take turns at the exponentials of a tile (two named
-// barriers pass the turn): while one warp's exponentials occupy the
-// sub-partition's MUFU unit, the other reads its next scores from TMEM and
-// reduces their maximum (1-4 % faster than letting both run in step).  Scores
-// are scaled into the log2 domain by the same FFMA that
-// subtracts the running max; the O rescale in TMEM is skipped while the max
-// grows by at most 2^8.  P is written as bf16 pairs into a TMEM P buffer of its
+// the end like two splits.  (Making the two warps that share an SM
+// sub-partition take turns at the exponentials, through named barriers,
+// measured 4 % slower on the l8b step.)  Scores are scaled into the log2
+// domain by the same FFMA that subtracts the running max; the O rescale in
+// TMEM is skipped while the max grows by at most 2^8.  P is written as bf16 pairs into a TMEM P buffer of its
 // own, once this group's P V of the previous tile has read it, and P V takes it
 // from there (the TMEM-A form of the MMA); since P does not overwrite the
 // scores, S = Q K^T of tile j + 1 runs while the softmax of tile j is still
@@ -78,9 +75,6 @@ constexpr uint32_t TMEM_COLS = 512;        // S [0,128), P [128,192), Q [192,256
 constexpr uint32_t P_COL = 128;            // P: 64 columns of bf16 pairs, group x at x * 32
 constexpr uint32_t Q_COL = 192;            // Q: 64 columns of bf16 pairs (dims 2c, 2c + 1 in column c)
 constexpr uint32_t O_COL = 256;
-// named barriers passing the turn at the exponentials: group A waits on BAR_TURN_A
-// (B arrives), group B on BAR_TURN_B (A arrives); 0 is __syncthreads, 1 the epilogue's
-constexpr int BAR_TURN_A = 2, BAR_TURN_B = 3;
 
 // mbarrier slots, derived from the ring depths
 constexpr int BAR_K_FULL = 0;                    // KST: K tile landed (TMA transaction count)
@@ -402,29 +396,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         float m_run = -INFINITY, l_run = 0.f;  // running max in the scaled log2 domain, running sum
         const float sl = a.scale_log2;
-        // The turn protocol: group A's exponentials of tile j follow group B's of tile
-        // j - 1, and B's of tile j follow A's of tile j.  A waits on BAR_TURN_A once per
-        // tile and B arrives there once per tile (before its loop for tile 0, after its
-        // exponentials of tile j for tile j + 1, never after the last tile); B waits on
-        // BAR_TURN_B once per tile and A arrives there once per tile.  Named barriers
-        // have no time limit, so the loop never leaves early: after a failed wait a warp
-        // only keeps passing the turn (`live` is false, and the abort flag makes every
-        // later mbarrier wait return at once), and both groups run all ntiles
-        // iterations.  The waits alternate strictly, so no barrier receives a second
-        // phase's arrivals before its current phase completes.
-        auto turn_wait = [&]() {
-            if (X == 0)
-                asm volatile("bar.sync %0, 256;" ::"n"(BAR_TURN_A) : "memory");
-            else
-                asm volatile("bar.sync %0, 256;" ::"n"(BAR_TURN_B) : "memory");
-        };
-        auto turn_pass = [&](int j) {
-            if (X == 0)
-                asm volatile("bar.arrive %0, 256;" ::"n"(BAR_TURN_B) : "memory");
-            else if (j + 1 < ntiles)
-                asm volatile("bar.arrive %0, 256;" ::"n"(BAR_TURN_A) : "memory");
-        };
-        if (X == 1 && ntiles > 0) asm volatile("bar.arrive %0, 256;" ::"n"(BAR_TURN_A) : "memory");
         bool live = true;  // warp-uniform: every wait of this warp so far succeeded
         for (int j = 0; j < ntiles; ++j) {
             live = live && warp_wait(s_full, j & 1, abort_flag);
@@ -464,7 +435,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 m_run = mt;
             }
             const float mu = m_run == -INFINITY ? 0.f : m_run;
-            turn_wait();
             // one P buffer: this group's P V of the previous tile has read it before it is
             // overwritten (the same wait also frees O for the rescale below)
             if (j > 0 && live) live = warp_wait(o_done(X), (j - 1) & 1, abort_flag);
@@ -484,7 +454,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 }
                 tmem_st_x32(tmem + lane_base + P_COL + X * 32, pp);
             }
-            turn_pass(j);
             if (!live) continue;
             l_run = l_run * f + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
             if (lim < TN) {
