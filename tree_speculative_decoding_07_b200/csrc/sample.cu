@@ -225,6 +225,11 @@ struct Walker {
     int passes;        // cluster exchanges so far
     uint32_t pending;  // bit x: a copy into buffer x is in flight
     uint32_t phase;    // bit x: parity of the next phase of buffer x's barrier
+    // The lane's whole steps of one buffer's row, converted to fp64 by the first pass
+    // over that row (rows of at most four steps per lane): later passes on the same row
+    // neither read shared memory nor convert again.  Steps past the slice hold zeros.
+    int cached = -1;   // buffer whose row rp / rq hold, -1 for none
+    double rp[4][4], rq[4][4];
 
     __device__ float* ps(int x) const { return buf + (size_t)2 * x * slice; }
     __device__ float* qs(int x) const { return ps(x) + slice; }
@@ -250,8 +255,9 @@ struct Walker {
     }
 
     // Start loading this CTA's slice of node u's p and q rows into buffer x (collective).
-    __device__ void issue_row(int x, int u) {
+    __device__ __forceinline__ void issue_row(int x, int u) {
         wait_row(x);  // the buffer's previous copy must have landed before it is reused
+        if (cached == x) cached = -1;
         const size_t base = ((size_t)b * N + u) * (size_t)V + lo;
         if (bulk) {
             if (tid == 0) {
@@ -277,7 +283,7 @@ struct Walker {
     // Sum over the whole row of resid(p, q, c) from buffer x; every CTA returns
     // the same value.  Leaves this CTA's per-warp partials in sh.warp_part and
     // every CTA's partial in sh.peer[parity of the pass].
-    __device__ double cluster_pass(int x, double c) {
+    __device__ __forceinline__ double cluster_pass(int x, double c) {
         const float* pr = ps(x);
         const float* qr = qs(x);
         const int s0 = min(n, warp * segw), s1 = min(n, s0 + segw);
@@ -294,6 +300,35 @@ struct Walker {
                 a2 += (double)pv.z;
                 a3 += (double)pv.w;
             }
+        } else if (segw <= 4 * 128) {
+            if (cached != x) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    float4 pv = make_float4(0.f, 0.f, 0.f, 0.f), qv = pv;
+                    if (i + 128 * k + 3 < s1) {
+                        pv = *reinterpret_cast<const float4*>(pr + i + 128 * k);
+                        qv = *reinterpret_cast<const float4*>(qr + i + 128 * k);
+                    }
+                    rp[k][0] = pv.x;
+                    rp[k][1] = pv.y;
+                    rp[k][2] = pv.z;
+                    rp[k][3] = pv.w;
+                    rq[k][0] = qv.x;
+                    rq[k][1] = qv.y;
+                    rq[k][2] = qv.z;
+                    rq[k][3] = qv.w;
+                }
+                cached = x;
+            }
+            // the same sums in the same order as from shared memory: a zero step adds +0.0
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                a0 += pos_part(fma(-c, rq[k][0], rp[k][0]));
+                a1 += pos_part(fma(-c, rq[k][1], rp[k][1]));
+                a2 += pos_part(fma(-c, rq[k][2], rp[k][2]));
+                a3 += pos_part(fma(-c, rq[k][3], rp[k][3]));
+            }
+            while (i + 3 < s1) i += 128;
         } else {
             for (; i + 3 < s1; i += 128) {
                 const float4 pv = *reinterpret_cast<const float4*>(pr + i);
@@ -363,6 +398,7 @@ struct Walker {
     // p = (float)(e * (1 / Z)); keep M and 1 / Z for the children's p(x), q(x), which
     // the gather computes with the same expression so they equal the converted row.
     __device__ void prep_row(int x) {
+        if (cached == x) cached = -1;  // the row is rewritten in place
         float* pl = ps(x);
         float* ql = qs(x);
         float mp = -INFINITY, mq = -INFINITY;
