@@ -55,7 +55,9 @@ def test_gpu_kernel_is_lossless():
     assert ok1 and ok2
 
 
-@pytest.mark.parametrize("V", [1, 3, 8, 1001, 4097, 65537, 128259])
+# 151,936 (a Qwen2-sized vocabulary) gives each warp more than four 128-entry steps, the
+# shape whose residual passes read shared memory every time instead of registers
+@pytest.mark.parametrize("V", [1, 3, 8, 1001, 4097, 65537, 128259, 151936])
 def test_ragged_vocab_sizes(V):
     rng = np.random.default_rng(V)
     B, parent = 16, [-1, 0, 0, 1, 1, 2, 0, 6]
@@ -107,13 +109,15 @@ def test_bad_tree_is_reported():
     assert res["accepted_len"][0] >= 0
 
 
-def test_bonus_draw_finds_the_owner_anywhere_in_the_vocabulary():
+@pytest.mark.parametrize("V", [128256, 128259, 151936])
+def test_bonus_draw_finds_the_owner_anywhere_in_the_vocabulary(V):
     # The root's only child has p(x) = 0, so it is always rejected, and the bonus token comes
     # from the residual max(0, p - q).  The residual is zero everywhere except a few chosen
     # entries, placed at the two ends of a 128,256-entry vocabulary and inside slices far from
     # the first (the walk spreads the vocabulary over up to 16 CTAs), so the owner of the draw
     # is found at the edges of the CTA and warp scans.  u0 = 0 takes the first entry with mass.
-    V = 128256
+    # At 128,259 the last slice ends inside a lane's four-entry step (summed entry by entry);
+    # at 151,936 each warp's segment is longer than the registers hold.
     spots = [[0], [V - 1], [3 * V // 16 + 5, 12 * V // 16 + 7], [3 * V // 16 + 5, 12 * V // 16 + 7],
              [V // 2 - 1, V // 2, V // 2 + 1], [7, V - 2]]
     u0 = [0.5, 0.5, 0.25, 0.75, 0.0, 0.3]
@@ -137,10 +141,10 @@ def test_bonus_draw_finds_the_owner_anywhere_in_the_vocabulary():
     assert (gpu["accepted_len"] == 0).all()
 
 
-def test_bonus_draw_with_u0_just_below_one_takes_the_last_entry_with_mass():
+@pytest.mark.parametrize("V", [128256, 128259, 151936])
+def test_bonus_draw_with_u0_just_below_one_takes_the_last_entry_with_mass(V):
     # target = u0 * Z sits within rounding of the total: whichever way the sums round, the
     # draw must be the last entry with residual mass (the oracle's fallback reading)
-    V = 128256
     B, x = 3, 11
     last = [V - 1, 9 * V // 16 + 3, 5]
     q = np.full((B, 2, V), 1.0 / V, np.float32)

@@ -23,9 +23,12 @@
 // contiguous per-warp segment, warp shuffle, CTA, then every CTA pushes its
 // partial to all peers with st.async, which completes on the receiver's own
 // mbarrier; every CTA adds the C partials in rank order, so all obtain the
-// same bits and take the same branches.  The bonus draw reuses the per-CTA
-// and per-warp partials of the last pass: the owning CTA, warp and lane are
-// located from them, and one lane scans its few elements.
+// same bits and take the same branches.  The first pass over a row keeps each
+// lane's entries in registers as fp64 (segments of up to four 128-entry
+// steps), so later passes on that row do only the fp64 arithmetic.  The bonus
+// draw reuses the per-CTA and per-warp partials of the last pass: the owning
+// CTA and warp are located from them, the owning CTA scans that warp's
+// segment, and one thread finds the element among its few.
 //
 // Children.  Every CTA first gathers, for every child c of the tree, the
 // draft token's entries p(x_c), q(x_c) of its parent's rows and its uniform
