@@ -68,11 +68,31 @@ def test_edge_shapes(dtype, B, N, Hq, Hkv, D, prefix, unit):
 
 
 @pytest.mark.parametrize("unit", [False, True], ids=["default_scale", "unit_kv"])
-def test_chain_tree_matches_oracle(unit):
-    N = 40
+@pytest.mark.parametrize("N", [40, 128])
+def test_chain_tree_matches_oracle(unit, N):
+    # A chain given by its parent array: its ancestor sets come from a bounded walk plus
+    # pointer jumping (128 nodes: depth 127, every jumping round).  The same chain without
+    # a parent array gets its sets in closed form and must give the same bits.
     parents = np.array([[-1] + list(range(N - 1))], np.int32)
     a = random_attn(5, 1, N, 32, 8, 128, [2000], parents=parents, kv_std=1.0 if unit else None,
                     tree_k_scale=synth.UNIT_TREE_K_SCALE if unit else 1.0)
+    out = a.run_gpu()
+    a.compare(out)
+    a.dpar = None
+    np.testing.assert_array_equal(a.run_gpu(), out)
+
+
+@pytest.mark.parametrize("unit", [False, True], ids=["default_scale", "unit_kv"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_deep_trees_match_oracle(unit, dtype):
+    # caterpillars: each node's parent is the previous node four times in five, else one two
+    # to four places back, so 128-node trees of depth 92-97 with a branch every few levels
+    rng = np.random.default_rng(9)
+    B, N = 3, 128
+    parents = np.array([[-1] + [i - 1 if (i < 2 or rng.random() < 0.8) else i - int(rng.integers(2, min(i, 4) + 1))
+                                for i in range(1, N)] for _ in range(B)], np.int32)
+    a = random_attn(6, B, N, 16, 8, 128, [300, 1500, 4000], dtype=dtype, parents=parents,
+                    kv_std=1.0 if unit else None, tree_k_scale=synth.UNIT_TREE_K_SCALE if unit else 1.0)
     a.compare(a.run_gpu())
 
 
