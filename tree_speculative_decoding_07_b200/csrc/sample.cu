@@ -169,16 +169,17 @@ __device__ __forceinline__ double warp_sum_d(double v) {
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
-// inclusive prefix sums over the lanes (lane k gets v_0 + ... + v_k, summed as a tree)
-__device__ __forceinline__ double warp_scan_d(double v, int lane) {
+// inclusive prefix sums over lanes 0..15 (lane k gets v_0 + ... + v_k, summed as a tree;
+// lanes 16..31 get values that are not used)
+__device__ __forceinline__ double half_scan_d(double v, int lane) {
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
+    for (int o = 1; o < 16; o <<= 1) {
         const double t = __shfl_up_sync(0xffffffffu, v, o);
         if (lane >= o) v += t;
     }
     return v;
 }
-// The first of n (<= 32) running totals that exceeds a target, from one value per lane:
+// The first of n (<= 16) running totals that exceeds a target, from one value per lane:
 // `first` is that lane (-1 if none), `last_pos` the last lane with a positive value, and
 // `before` the running total of the lanes before `first` (0 for lane 0).  Every lane of
 // the warp gets the same results.
@@ -187,7 +188,7 @@ struct Crossing {
     double before;
 };
 __device__ __forceinline__ Crossing first_crossing(double v, int n, double base, double target, int lane) {
-    const double inc = warp_scan_d(lane < n ? v : 0.0, lane);
+    const double inc = half_scan_d(lane < n ? v : 0.0, lane);
     const unsigned cross = __ballot_sync(0xffffffffu, lane < n && base + inc > target);
     const unsigned pos = __ballot_sync(0xffffffffu, lane < n && v > 0.0);
     Crossing r;
@@ -197,9 +198,19 @@ __device__ __forceinline__ Crossing first_crossing(double v, int n, double base,
     r.before = base + (r.first > 0 ? prev : 0.0);
     return r;
 }
-__device__ __forceinline__ double warp_max_d(double v) {
+// Sum and maximum over 16 values (a cluster's CTAs, a CTA's warps: both at most 16).
+// Both half-warps hold the 16 values, so four butterfly levels give every lane the
+// result, with the same pairings, hence the same bits, as a 32-lane butterfly over the
+// values padded with the identity.
+static_assert(MAX_CLUSTER <= 16 && MAX_THREADS / 32 <= 16, "the half-warp reductions take at most 16 values");
+__device__ __forceinline__ double half_sum_d(double v) {
 #pragma unroll
-    for (int o = 16; o; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+    for (int o = 8; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ double half_max_d(double v) {
+#pragma unroll
+    for (int o = 8; o; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
 }
 __device__ __forceinline__ float warp_max_f(float v) {
@@ -347,7 +358,7 @@ struct Walker {
         if (lane == 0) sh.warp_part[warp] = wsum;
         __syncthreads();
         // this CTA's partial: a fixed shuffle tree over its warps (warp 0's value is sent)
-        const double s = warp == 0 ? warp_sum_d(lane < nwarps ? sh.warp_part[lane] : 0.0) : 0.0;
+        const double s = warp == 0 ? half_sum_d((lane & 15) < nwarps ? sh.warp_part[lane & 15] : 0.0) : 0.0;
         double total, unused;
         exchange(1, s, 0.0, false, total, unused);
         return total;
@@ -385,11 +396,12 @@ struct Walker {
             mbar_wait(smem_u32(&sh.peer_bar[par]), use & 1, &sh.timeout);
         }
         const double id = take_max ? -INFINITY : 0.0;
-        const double x0 = lane < C ? sh.peer[par][lane] : id;
-        r0 = take_max ? warp_max_d(x0) : warp_sum_d(x0);
+        const int k = lane & 15;
+        const double x0 = k < C ? sh.peer[par][k] : id;
+        r0 = take_max ? half_max_d(x0) : half_sum_d(x0);
         if (nv == 2) {
-            const double x1 = lane < C ? sh.peer2[par][lane] : id;
-            r1 = take_max ? warp_max_d(x1) : warp_sum_d(x1);
+            const double x1 = k < C ? sh.peer2[par][k] : id;
+            r1 = take_max ? half_max_d(x1) : half_sum_d(x1);
         } else {
             r1 = 0.0;
         }
@@ -418,8 +430,9 @@ struct Walker {
         __syncthreads();
         double Mp, Mq;
         {
-            const double v0 = warp == 0 ? warp_max_d(lane < nwarps ? sh.warp_part[lane] : -INFINITY) : 0.0;
-            const double v1 = warp == 0 ? warp_max_d(lane < nwarps ? sh.warp_part2[lane] : -INFINITY) : 0.0;
+            const int k = lane & 15;
+            const double v0 = warp == 0 ? half_max_d(k < nwarps ? sh.warp_part[k] : -INFINITY) : 0.0;
+            const double v1 = warp == 0 ? half_max_d(k < nwarps ? sh.warp_part2[k] : -INFINITY) : 0.0;
             exchange(2, v0, v1, true, Mp, Mq);
         }
         const float mpf = (float)Mp, mqf = (float)Mq;
@@ -441,8 +454,9 @@ struct Walker {
         __syncthreads();
         double Zp, Zq;
         {
-            const double v0 = warp == 0 ? warp_sum_d(lane < nwarps ? sh.warp_part[lane] : 0.0) : 0.0;
-            const double v1 = warp == 0 ? warp_sum_d(lane < nwarps ? sh.warp_part2[lane] : 0.0) : 0.0;
+            const int k = lane & 15;
+            const double v0 = warp == 0 ? half_sum_d(k < nwarps ? sh.warp_part[k] : 0.0) : 0.0;
+            const double v1 = warp == 0 ? half_sum_d(k < nwarps ? sh.warp_part2[k] : 0.0) : 0.0;
             exchange(2, v0, v1, false, Zp, Zq);
         }
         const double zpi = Zp > 0.0 ? 1.0 / Zp : 0.0, zqi = Zq > 0.0 ? 1.0 / Zq : 0.0;
@@ -764,7 +778,7 @@ __global__ void __launch_bounds__(MAX_THREADS) verify_sample_kernel(const __grid
             __syncthreads();
             {
                 // this warp's offset: the running total of the warps before it
-                const double inc = warp_scan_d(lane < nwarps ? sh.warp_part2[lane] : 0.0, lane);
+                const double inc = half_scan_d(lane < nwarps ? sh.warp_part2[lane] : 0.0, lane);
                 const double prev = __shfl_sync(0xffffffffu, inc, warp > 0 ? warp - 1 : 0);
                 incl += warp > 0 ? prev : 0.0;
             }
